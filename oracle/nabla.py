@@ -1,0 +1,326 @@
+"""Plain fp64 CPU oracle of NABLA-style block-sparse attention.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path imports, calls or links
+this module: only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline
+and reference legs of ``bench.py`` use it.  It shares no code with the CUDA
+path.
+
+Every function writes out a definition from the NABLA technical summary
+("NABLA - Atencion de Bloque Adaptativa al Vecindario para la Generacion
+Eficiente de Video", gist.science/es/paper/2507.13546), cited below as
+"NABLA summary" plus the section.  Arithmetic is float64 throughout, applied to
+the exact float64 values of the bf16 inputs.  Library primitives (a matmul, a
+stable argsort, a cumulative sum, exp) serve as single steps; there is no
+blocking or fusion beyond what each definition states.
+
+Readings taken where the page is silent or garbled (each is listed in
+the design doc too):
+
+* fractal order: one level of P x P grouping, time outermost, patches in
+  row-major order, tokens inside a patch in row-major order; edge patches are
+  clipped to H and W; the sequence is then zero-padded at its end to a
+  multiple of the block size;
+* pooling divides by the number of valid (non-padding) tokens of the block;
+* softmax scale is 1/sqrt(d) in both the reduced map and the attention;
+* CDF rule: sort a row by descending probability (ties: lower block index
+  first) and keep the shortest prefix whose mass reaches 1 - thr; thr == 0
+  keeps every block; if rounding leaves every prefix short of 1 - thr, every
+  block is kept;
+* STA: block I sits at the tile (t, h // P, w // P) of its first token in the
+  fractal order; blocks I, J are in the window when the tile coordinates
+  differ by at most the half-widths in each of t, h, w;
+* padded keys take part in nothing; padded query rows output 0 (LSE 0).
+
+Parity pins (tests/test_oracle_pins.py): a hand-derived permutation, the
+bijection, closed forms for pooling and the reduced map, brute force over all
+subsets for the CDF rule, the aligned tile grid for STA, and a library
+attention (torch scaled_dot_product_attention in float64) for the masked
+softmax.  The end-to-end combination beyond these invariants is
+"parity unpinned": the pages print no worked example.
+"""
+from __future__ import annotations
+
+import math
+from typing import Iterable, Optional, Sequence, Tuple
+
+import numpy as np
+
+AMBIGUITY_MASS = 1e-6      # prefix-mass window around 1 - thr
+AMBIGUITY_TIE_REL = 1e-9   # relative near-tie window around the boundary block's probability
+
+
+# ---------------------------------------------------------------- shapes
+
+def padded_len(N: int, block: int) -> int:
+    return -(-N // block) * block
+
+
+def num_blocks(N: int, block: int) -> int:
+    return padded_len(N, block) // block
+
+
+# ------------------------------------------------------- fractal reorder
+
+def fractal_order(T: int, H: int, W: int, P: int) -> np.ndarray:
+    """Position p of the reordered sequence -> original token n = t*H*W + h*W + w.
+
+    NABLA summary, Metodologia 1 ("Reordenamiento de Tokens (Aplanamiento
+    Fractal)"): tokens of each P x P spatial patch become contiguous and the
+    temporal order is kept.
+    """
+    order = []
+    for t in range(T):
+        for pr in range(-(-H // P)):
+            for pc in range(-(-W // P)):
+                for h in range(pr * P, min((pr + 1) * P, H)):
+                    for w in range(pc * P, min((pc + 1) * P, W)):
+                        order.append(t * H * W + h * W + w)
+    return np.asarray(order, dtype=np.int64)
+
+
+def reorder(x_bnhd: np.ndarray, T: int, H: int, W: int, P: int, block: int) -> np.ndarray:
+    """[B, N, heads, d] in model order -> [B, heads, Npad, d] in fractal order, zero tail."""
+    B, N, heads, d = x_bnhd.shape
+    assert N == T * H * W
+    order = fractal_order(T, H, W, P)
+    y = np.zeros((B, heads, padded_len(N, block), d), dtype=np.float64)
+    for p in range(N):
+        y[:, :, p, :] = x_bnhd[:, order[p], :, :]
+    return y
+
+
+def inverse_reorder(y_bhnd: np.ndarray, T: int, H: int, W: int, P: int) -> np.ndarray:
+    """Undo ``reorder``: [B, heads, Npad, d] -> [B, N, heads, d], padding dropped."""
+    B, heads, _, d = y_bhnd.shape
+    N = T * H * W
+    order = fractal_order(T, H, W, P)
+    x = np.zeros((B, N, heads, d), dtype=np.float64)
+    for p in range(N):
+        x[:, order[p], :, :] = y_bhnd[:, :, p, :]
+    return x
+
+
+# ------------------------------------------------------------- pooling
+
+def block_means(y_bhnd: np.ndarray, N: int, block: int) -> np.ndarray:
+    """Mean of the valid tokens of every block: [B, heads, Npad, d] -> [B, heads, nb, d].
+
+    NABLA summary, Metodologia 2, "Submuestreo": Q and K are averaged over
+    blocks of tokens.
+    """
+    B, heads, Npad, d = y_bhnd.shape
+    nb = Npad // block
+    out = np.zeros((B, heads, nb, d), dtype=np.float64)
+    for I in range(nb):
+        lo = I * block
+        hi = min((I + 1) * block, N)
+        out[:, :, I, :] = y_bhnd[:, :, lo:hi, :].sum(axis=2) / float(hi - lo)
+    return out
+
+
+# ---------------------------------------------------- reduced attention
+
+def reduced_attention(qbar: np.ndarray, kbar: np.ndarray, scale: Optional[float] = None) -> np.ndarray:
+    """Row softmax of the pooled scores: [.., nb, d] x [.., nb, d] -> [.., nb, nb].
+
+    NABLA summary, Metodologia 2, "Atencion Reducida": a full attention map over
+    the pooled block representations.
+    """
+    d = qbar.shape[-1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    s = np.matmul(qbar, np.swapaxes(kbar, -1, -2)) * scale
+    s = s - s.max(axis=-1, keepdims=True)
+    e = np.exp(s)
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+# ------------------------------------------------------- CDF threshold
+
+def cdf_keep(A: np.ndarray, thr: float) -> Tuple[np.ndarray, np.ndarray]:
+    """Binary block mask from a reduced map, plus the ambiguous blocks.
+
+    NABLA summary, Metodologia 2, "Umbralizacion CDF": per row, the blocks are
+    taken in decreasing probability and the shortest prefix whose cumulative
+    mass reaches 1 - thr is kept.
+
+    Returns ``(keep, ambiguous)``, both bool with the shape of ``A``.  A block is
+    ambiguous when the mass of the blocks ranked before it lies within
+    ``AMBIGUITY_MASS`` of 1 - thr (its decision flips under rounding), or when
+    its probability is within ``AMBIGUITY_TIE_REL`` (relative) of the last kept
+    block's (a near-tie can swap which of the two is kept).
+    """
+    if not (0.0 <= thr < 1.0):
+        raise ValueError("thr must lie in [0, 1)")
+    lead = A.shape[:-1]
+    nb = A.shape[-1]
+    rows = A.reshape(-1, nb)
+    keep = np.zeros(rows.shape, dtype=bool)
+    amb = np.zeros(rows.shape, dtype=bool)
+    target = 1.0 - thr
+    for r in range(rows.shape[0]):
+        a = rows[r]
+        if thr == 0.0:
+            keep[r, :] = True
+            continue
+        order = np.argsort(-a, kind="stable")          # descending, ties -> lower J first
+        c = np.cumsum(a[order])                         # c[k-1] = mass of the first k blocks
+        reach = np.nonzero(c >= target)[0]
+        kstar = int(reach[0]) + 1 if reach.size else nb
+        keep[r, order[:kstar]] = True
+        before = np.concatenate([[0.0], c[:-1]])        # mass ranked ahead of each block
+        amb[r, order[np.abs(before - target) <= AMBIGUITY_MASS]] = True
+        vb = a[order[kstar - 1]]
+        near = np.abs(a - vb) <= AMBIGUITY_TIE_REL * vb
+        if near.sum() > 1:
+            amb[r, near] = True
+    return keep.reshape(A.shape), amb.reshape(A.shape)
+
+
+# ------------------------------------------------------------ STA union
+
+def block_tiles(T: int, H: int, W: int, P: int, block: int) -> np.ndarray:
+    """(t, h // P, w // P) of the first token of every block in the fractal order: [nb, 3]."""
+    N = T * H * W
+    order = fractal_order(T, H, W, P)
+    nb = num_blocks(N, block)
+    tiles = np.zeros((nb, 3), dtype=np.int64)
+    for I in range(nb):
+        n = int(order[I * block])
+        t, rem = divmod(n, H * W)
+        h, w = divmod(rem, W)
+        tiles[I] = (t, h // P, w // P)
+    return tiles
+
+
+def sta_mask(T: int, H: int, W: int, P: int, block: int, half: Tuple[int, int, int]) -> np.ndarray:
+    """Static sliding-tile window over blocks: [nb, nb] bool.
+
+    NABLA summary, Metodologia 3 ("Integracion Hibrida con STA"): the final mask
+    is the union of the adaptive mask and a static window mask.
+    """
+    tiles = block_tiles(T, H, W, P, block)
+    nb = tiles.shape[0]
+    m = np.zeros((nb, nb), dtype=bool)
+    for I in range(nb):
+        for J in range(nb):
+            m[I, J] = all(abs(int(tiles[I, a]) - int(tiles[J, a])) <= half[a] for a in range(3))
+    return m
+
+
+# ----------------------------------------------------------- block mask
+
+def block_mask(q_bhnd: np.ndarray, k_bhnd: np.ndarray, T: int, H: int, W: int, P: int, block: int,
+               thr: float, sta: Optional[Tuple[int, int, int]] = None,
+               scale: Optional[float] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """Reduced map -> CDF mask (-> union with STA).  Returns ``(keep, ambiguous)`` [B, heads, nb, nb].
+
+    Blocks that the STA window keeps are never ambiguous: the union keeps them
+    whatever the CDF rule decides.
+    """
+    N = T * H * W
+    qbar = block_means(q_bhnd, N, block)
+    kbar = block_means(k_bhnd, N, block)
+    A = reduced_attention(qbar, kbar, scale)
+    keep, amb = cdf_keep(A, thr)
+    if sta is not None:
+        m = sta_mask(T, H, W, P, block, sta)
+        keep = keep | m[None, None]
+        amb = amb & ~m[None, None]
+    return keep, amb
+
+
+def mask_to_lists(keep: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """Bool [.., nb, nb] -> (kv_count [.., nb] int32, kv_idx [.., nb, nb] int32 ascending, -1 tail)."""
+    nb = keep.shape[-1]
+    flat = keep.reshape(-1, nb)
+    count = flat.sum(axis=1).astype(np.int32)
+    idx = np.full(flat.shape, -1, dtype=np.int32)
+    for r in range(flat.shape[0]):
+        js = np.nonzero(flat[r])[0]
+        idx[r, :js.size] = js
+    return count.reshape(keep.shape[:-1]), idx.reshape(keep.shape)
+
+
+def lists_to_mask(kv_count: np.ndarray, kv_idx: np.ndarray, nb: int) -> np.ndarray:
+    """Inverse of ``mask_to_lists`` (entries past ``kv_count`` are ignored)."""
+    cnt = kv_count.reshape(-1)
+    idx = kv_idx.reshape(-1, kv_idx.shape[-1])
+    keep = np.zeros((cnt.size, nb), dtype=bool)
+    for r in range(cnt.size):
+        keep[r, idx[r, :cnt[r]]] = True
+    return keep.reshape(kv_count.shape + (nb,))
+
+
+# ------------------------------------------------- block-sparse attention
+
+def masked_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, keep: np.ndarray, N: int, block: int,
+                     scale: Optional[float] = None,
+                     blocks: Optional[Iterable[Tuple[int, int, int]]] = None
+                     ) -> Tuple[np.ndarray, np.ndarray]:
+    """Softmax attention restricted to the kept N x N tiles.
+
+    NABLA summary, Metodologia 2, "Expansion": the block mask, expanded to
+    tokens, says which attention tiles are computed; a query in block I attends
+    to every valid key of every kept block J, with a softmax over exactly those
+    keys.
+
+    ``q, k, v``: [B, heads, Npad, d] (fractal order).  ``keep``: [B, heads, nb, nb].
+    ``blocks``: optional iterable of (b, head, I) to compute; others stay 0.
+    Returns ``(O [B, heads, Npad, d], lse [B, heads, Npad])`` (natural log);
+    padded query rows have O = 0 and lse = 0.
+    """
+    B, heads, Npad, d = q.shape
+    nb = Npad // block
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    O = np.zeros_like(q, dtype=np.float64)
+    lse = np.zeros((B, heads, Npad), dtype=np.float64)
+    if blocks is None:
+        blocks = [(b, h, I) for b in range(B) for h in range(heads) for I in range(nb)]
+    for (b, h, I) in blocks:
+        qlo, qhi = I * block, min((I + 1) * block, N)
+        if qhi <= qlo:
+            continue
+        cols = []
+        for J in np.nonzero(keep[b, h, I])[0]:
+            klo, khi = int(J) * block, min((int(J) + 1) * block, N)
+            cols.extend(range(klo, khi))
+        cols = np.asarray(cols, dtype=np.int64)
+        if cols.size == 0:
+            continue
+        s = (q[b, h, qlo:qhi, :] @ k[b, h, cols, :].T) * scale
+        m = s.max(axis=1, keepdims=True)
+        e = np.exp(s - m)
+        z = e.sum(axis=1, keepdims=True)
+        O[b, h, qlo:qhi, :] = (e @ v[b, h, cols, :]) / z
+        lse[b, h, qlo:qhi] = (m + np.log(z))[:, 0]
+    return O, lse
+
+
+# ------------------------------------------------------------ full path
+
+def nabla_attention(q_bnhd: np.ndarray, k_bnhd: np.ndarray, v_bnhd: np.ndarray,
+                    T: int, H: int, W: int, P: int, block: int, thr: float,
+                    sta: Optional[Tuple[int, int, int]] = None,
+                    scale: Optional[float] = None):
+    """The whole path on model-order inputs: reorder, mask, attention, inverse reorder.
+
+    Returns ``(O [B, N, heads, d], keep, ambiguous)``.
+    """
+    N = T * H * W
+    q = reorder(q_bnhd, T, H, W, P, block)
+    k = reorder(k_bnhd, T, H, W, P, block)
+    v = reorder(v_bnhd, T, H, W, P, block)
+    keep, amb = block_mask(q, k, T, H, W, P, block, thr, sta, scale)
+    O, _ = masked_attention(q, k, v, keep, N, block, scale)
+    return inverse_reorder(O, T, H, W, P), keep, amb
+
+
+def density(keep: np.ndarray) -> float:
+    return float(keep.sum()) / float(keep.size)
+
+
+def attention_flops(N: int, d: int, heads: int, B: int, dens: float) -> float:
+    """Effective FLOPs of one block-sparse call: 4 * N^2 * d * heads * B * density."""
+    return 4.0 * N * N * d * heads * B * dens

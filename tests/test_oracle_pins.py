@@ -1,0 +1,334 @@
+"""Pins for the fp64 oracle against facts that do not come from the oracle itself:
+hand-derived values (tests/golden), closed forms, brute force over all subsets,
+special cases that reduce to a library routine (torch SDPA in float64), and
+invariants.  CPU only.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+from oracle import nabla
+
+
+def _read_golden(path):
+    kv = {}
+    with open(path) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, *vals = line.split()
+            kv[key] = [int(v) for v in vals]
+    return kv
+
+
+# ------------------------------------------------------------------ reorder
+
+def test_fractal_order_matches_hand_derivation(golden_dir):
+    g = _read_golden(os.path.join(golden_dir, "fractal_order_T2_H3_W5_P2.txt"))
+    T, H, W, P = g["T"][0], g["H"][0], g["W"][0], g["P"][0]
+    assert oracle.fractal_order(T, H, W, P).tolist() == g["order"]
+
+
+def test_fractal_order_landmarks():
+    o = oracle.fractal_order(1, 16, 16, 8)
+    # second patch of the first patch row starts with token (t=0, h=0, w=8)
+    assert o[64] == 8
+    # second patch row starts with token (0, 8, 0)
+    assert o[128] == 8 * 16
+    # inside a patch: row-major
+    assert o[:10].tolist() == [0, 1, 2, 3, 4, 5, 6, 7, 16, 17]
+
+
+@pytest.mark.parametrize("T,H,W,P", [(4, 16, 16, 8), (2, 24, 40, 8)])
+def test_aligned_blocks_are_single_patches(T, H, W, P):
+    o = oracle.fractal_order(T, H, W, P)
+    bs = P * P
+    for I in range(len(o) // bs):
+        toks = o[I * bs:(I + 1) * bs]
+        t = toks // (H * W)
+        h = (toks % (H * W)) // W
+        w = toks % W
+        assert len(set(t.tolist())) == 1
+        assert len(set((h // P).tolist())) == 1 and len(set((w // P).tolist())) == 1
+        assert sorted(set(h.tolist())) == list(range(h.min(), h.min() + P))
+
+
+@pytest.mark.parametrize("T,H,W,P,bs", [(1, 3, 5, 2, 4), (2, 7, 9, 4, 16), (3, 10, 13, 8, 64), (2, 8, 8, 8, 64)])
+def test_reorder_is_a_bijection(T, H, W, P, bs):
+    rng = np.random.default_rng(0)
+    N = T * H * W
+    o = oracle.fractal_order(T, H, W, P)
+    assert sorted(o.tolist()) == list(range(N))
+    x = rng.standard_normal((2, N, 3, 4))
+    y = oracle.reorder(x, T, H, W, P, bs)
+    assert y.shape == (2, 3, nabla.padded_len(N, bs), 4)
+    assert np.all(y[:, :, N:, :] == 0.0)
+    assert np.array_equal(oracle.inverse_reorder(y, T, H, W, P), x)
+    # reorder moves whole token rows: position p holds the token the order names
+    p = N // 2
+    assert np.array_equal(y[1, 2, p], x[1, o[p], 2])
+
+
+# ------------------------------------------------------------------ pooling
+
+def test_block_means_closed_forms():
+    # constant -> the constant; ramp value = position -> midpoint of valid positions
+    N, bs, d = 70, 64, 3
+    Npad = nabla.padded_len(N, bs)
+    y = np.zeros((1, 1, Npad, d))
+    y[0, 0, :N, 0] = 2.5
+    y[0, 0, :N, 1] = np.arange(N)
+    y[0, 0, N:, :] = 1e9        # padding must not leak into the means
+    m = oracle.block_means(y, N, bs)
+    assert m.shape == (1, 1, 2, d)
+    assert np.allclose(m[0, 0, :, 0], 2.5, rtol=0, atol=1e-15)
+    assert m[0, 0, 0, 1] == (0 + 63) / 2
+    assert m[0, 0, 1, 1] == (64 + 69) / 2
+    assert np.all(m[0, 0, :, 2] == 0.0)
+
+
+# --------------------------------------------------------- reduced attention
+
+def test_reduced_attention_closed_forms():
+    # equal pooled keys -> uniform rows
+    kb = np.tile(np.array([[0.3, -1.0, 2.0, 0.5]]), (5, 1))
+    qb = np.random.default_rng(1).standard_normal((5, 4))
+    A = oracle.reduced_attention(qb, kb)
+    assert np.allclose(A, 1 / 5, atol=1e-15)
+    # two blocks, d = 2: s = (q.k0, q.k1)/sqrt(2) = (sqrt(2), 0) -> logistic
+    qb = np.array([[1.0, 0.0]])
+    kb = np.array([[2.0, 0.0], [0.0, 0.0]])
+    A = oracle.reduced_attention(qb, kb)
+    want0 = 1.0 / (1.0 + math.exp(-math.sqrt(2.0)))
+    assert abs(A[0, 0] - want0) < 1e-15 and abs(A[0, 1] - (1 - want0)) < 1e-15
+    # a transposed operand would break the asymmetric case: q only sees its own row
+    qb = np.array([[1.0, 0.0], [0.0, 0.0]])
+    kb = np.array([[0.0, 0.0], [3.0, 0.0]])
+    A = oracle.reduced_attention(qb, kb)
+    assert A[0, 1] > 0.8 and np.allclose(A[1], 0.5)
+
+
+def test_reduced_attention_rows_are_distributions():
+    rng = np.random.default_rng(2)
+    A = oracle.reduced_attention(rng.standard_normal((3, 40, 16)) * 4, rng.standard_normal((3, 40, 16)) * 4)
+    assert np.all(A > 0)
+    assert np.allclose(A.sum(-1), 1.0, atol=1e-12)
+    # against torch's softmax in float64 (a different library routine)
+    qb = rng.standard_normal((40, 16))
+    kb = rng.standard_normal((40, 16))
+    ref = torch.softmax(torch.from_numpy(qb @ kb.T / 4.0), dim=-1).numpy()
+    assert np.allclose(oracle.reduced_attention(qb, kb), ref, rtol=1e-13, atol=1e-15)
+
+
+# ------------------------------------------------------------ CDF threshold
+
+def test_cdf_matches_hand_examples(golden_dir):
+    with open(os.path.join(golden_dir, "cdf_threshold_examples.txt")) as f:
+        rows = [l for l in f if l.strip() and not l.startswith("#")]
+    assert len(rows) == 5
+    for line in rows:
+        thr, probs, kept = [p.strip() for p in line.split("|")]
+        A = np.array([float(x) for x in probs.split()])[None]
+        keep, _ = oracle.cdf_keep(A, float(thr))
+        assert np.nonzero(keep[0])[0].tolist() == [int(x) for x in kept.split()], line
+
+
+def test_cdf_is_minimal_by_brute_force():
+    rng = np.random.default_rng(3)
+    for trial in range(300):
+        nb = int(rng.integers(1, 11))
+        A = rng.dirichlet(np.full(nb, float(rng.choice([0.3, 1.0, 3.0]))))[None]
+        thr = float(rng.uniform(0.0, 0.95))
+        keep, amb = oracle.cdf_keep(A, thr)
+        if amb.any():
+            continue
+        target = 1.0 - thr
+        best_k, best_mass = None, -1.0
+        for k in range(1, nb + 1):
+            masses = [sum(A[0, list(c)]) for c in itertools.combinations(range(nb), k)]
+            if max(masses) >= target - 1e-12:
+                best_k, best_mass = k, max(masses)
+                break
+        if thr == 0.0:
+            best_k = nb
+        assert keep.sum() == best_k, (A, thr)
+        # the kept set carries the largest mass among sets of that size
+        assert abs(A[0, keep[0]].sum() - best_mass) < 1e-12
+
+
+def test_cdf_extremes():
+    rng = np.random.default_rng(4)
+    A = rng.dirichlet(np.ones(30), size=4)
+    keep, _ = oracle.cdf_keep(A, 0.0)
+    assert keep.all()
+    keep, _ = oracle.cdf_keep(A, 1.0 - 1e-12)
+    assert np.array_equal(keep, A == A.max(axis=1, keepdims=True))
+    with pytest.raises(ValueError):
+        oracle.cdf_keep(A, 1.0)
+
+
+def test_cdf_flags_blocks_near_the_threshold():
+    # ranked: 0.4 (J0), 0.25 (J3), 0.2 (J1), 0.15 (J2); prefix mass ahead of each:
+    # J0 0, J3 0.4, J1 0.65, J2 0.85.  Target 0.6000005 is far from all of them.
+    A = np.array([[0.4, 0.2, 0.15, 0.25]])
+    keep, amb = oracle.cdf_keep(A, 1.0 - 0.6000005)
+    assert not amb.any()
+    A = np.array([[0.4, 0.2, 0.15, 0.25]])
+    keep, amb = oracle.cdf_keep(A, 1.0 - 0.65 + 4e-7)   # target 0.6499996 ~ prefix 0.65 before J1
+    assert amb[0, 1] and not amb[0, 0]
+
+
+# ----------------------------------------------------------------- STA
+
+def test_sta_on_aligned_grid_is_the_tile_window():
+    T, H, W, P = 3, 24, 24, 8
+    bs = P * P
+    nPr, nPc = H // P, W // P
+    m = oracle.sta_mask(T, H, W, P, bs, (1, 1, 1))
+    nb = T * nPr * nPc
+    assert m.shape == (nb, nb)
+    for I in range(nb):
+        tI, rI, cI = I // (nPr * nPc), (I // nPc) % nPr, I % nPc
+        for J in range(nb):
+            tJ, rJ, cJ = J // (nPr * nPc), (J // nPc) % nPr, J % nPc
+            want = abs(tI - tJ) <= 1 and abs(rI - rJ) <= 1 and abs(cI - cJ) <= 1
+            assert m[I, J] == want
+    # an interior block sees exactly 27 tiles; a corner block 8
+    assert m[1 * nPr * nPc + 1 * nPc + 1].sum() == 27
+    assert m[0].sum() == 2 * 2 * 2
+
+
+def test_hybrid_mask_contains_both_parts():
+    rng = np.random.default_rng(5)
+    T, H, W, P, bs = 2, 12, 20, 4, 16
+    N = T * H * W
+    q = oracle.reorder(rng.standard_normal((1, N, 2, 8)), T, H, W, P, bs)
+    k = oracle.reorder(rng.standard_normal((1, N, 2, 8)), T, H, W, P, bs)
+    keep_a, _ = oracle.block_mask(q, k, T, H, W, P, bs, 0.3)
+    keep_h, _ = oracle.block_mask(q, k, T, H, W, P, bs, 0.3, sta=(1, 1, 1))
+    sta = oracle.sta_mask(T, H, W, P, bs, (1, 1, 1))
+    assert np.array_equal(keep_h, keep_a | sta[None, None])
+
+
+# ------------------------------------------------------------- attention
+
+def _sdpa_rows(q, k, v, keymask, scale):
+    """torch SDPA in float64 with a boolean mask (True = take part)."""
+    out = F.scaled_dot_product_attention(torch.from_numpy(q)[None, None], torch.from_numpy(k)[None, None],
+                                         torch.from_numpy(v)[None, None],
+                                         attn_mask=torch.from_numpy(keymask)[None, None], scale=scale)
+    return out[0, 0].numpy()
+
+
+@pytest.mark.parametrize("N,bs", [(96, 32), (100, 32)])
+def test_masked_attention_equals_library_attention(N, bs):
+    rng = np.random.default_rng(6)
+    d, heads = 16, 2
+    Npad = nabla.padded_len(N, bs)
+    nb = Npad // bs
+    q = rng.standard_normal((1, heads, Npad, d)) * 2
+    k = rng.standard_normal((1, heads, Npad, d)) * 2
+    v = rng.standard_normal((1, heads, Npad, d))
+    keep = rng.random((1, heads, nb, nb)) < 0.5
+    keep[..., np.arange(nb), np.arange(nb)] = True
+    O, lse = oracle.masked_attention(q, k, v, keep, N, bs)
+    scale = 1 / math.sqrt(d)
+    for h in range(heads):
+        tokmask = np.kron(keep[0, h], np.ones((bs, bs), dtype=bool))[:N, :N]
+        ref = _sdpa_rows(q[0, h, :N], k[0, h, :N], v[0, h, :N], tokmask, scale)
+        assert np.allclose(O[0, h, :N], ref, rtol=1e-12, atol=1e-12)
+        s = (q[0, h, :N] @ k[0, h, :N].T) * scale
+        s[~tokmask] = -np.inf
+        ref_lse = torch.logsumexp(torch.from_numpy(s), dim=-1).numpy()
+        assert np.allclose(lse[0, h, :N], ref_lse, rtol=1e-12, atol=1e-12)
+    assert np.all(O[:, :, N:] == 0) and np.all(lse[:, :, N:] == 0)
+
+
+def test_attention_special_cases():
+    rng = np.random.default_rng(7)
+    N, bs, d = 120, 32, 8
+    Npad = nabla.padded_len(N, bs)
+    nb = Npad // bs
+    q = rng.standard_normal((1, 1, Npad, d))
+    k = rng.standard_normal((1, 1, Npad, d))
+    # V constant -> output is that constant
+    v = np.full((1, 1, Npad, d), -0.75)
+    keep = rng.random((1, 1, nb, nb)) < 0.6
+    keep[..., np.arange(nb), np.arange(nb)] = True
+    O, _ = oracle.masked_attention(q, k, v, keep, N, bs)
+    assert np.allclose(O[0, 0, :N], -0.75, atol=1e-14)
+    # a single kept block whose keys are identical -> mean of that block's valid V
+    J = nb - 1                                   # the ragged last block (24 valid keys)
+    k2 = k.copy()
+    k2[0, 0, J * bs:] = k[0, 0, J * bs]
+    v2 = rng.standard_normal((1, 1, Npad, d))
+    keep2 = np.zeros((1, 1, nb, nb), dtype=bool)
+    keep2[..., J] = True
+    O2, _ = oracle.masked_attention(q, k2, v2, keep2, N, bs)
+    assert np.allclose(O2[0, 0, :N], v2[0, 0, J * bs:N].mean(axis=0), atol=1e-13)
+
+
+def test_thr_zero_pipeline_is_dense_attention_in_model_order():
+    """thr = 0 keeps every block; reorder -> attention -> inverse must then equal
+    dense attention applied directly to the model-order tokens."""
+    rng = np.random.default_rng(8)
+    T, H, W, P, bs = 2, 6, 10, 4, 16
+    N, heads, d = T * H * W, 2, 8
+    q = rng.standard_normal((1, N, heads, d))
+    k = rng.standard_normal((1, N, heads, d))
+    v = rng.standard_normal((1, N, heads, d))
+    O, keep, amb = oracle.nabla_attention(q, k, v, T, H, W, P, bs, 0.0)
+    assert keep.all() and not amb.any()
+    for h in range(heads):
+        ref = _sdpa_rows(q[0, :, h], k[0, :, h], v[0, :, h], np.ones((N, N), dtype=bool), 1 / math.sqrt(d))
+        assert np.allclose(O[0, :, h], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_lists_roundtrip():
+    rng = np.random.default_rng(9)
+    keep = rng.random((2, 3, 7, 7)) < 0.4
+    cnt, idx = oracle.mask_to_lists(keep)
+    assert np.array_equal(oracle.lists_to_mask(cnt, idx, 7), keep)
+    for r in range(cnt.size):
+        row = idx.reshape(-1, 7)[r]
+        c = cnt.reshape(-1)[r]
+        assert np.all(np.diff(row[:c]) > 0) and np.all(row[c:] == -1)
+
+
+# ------------------------------------------------ planted mistakes are caught
+
+def test_pins_catch_an_off_by_one_cdf(monkeypatch):
+    def bad(A, thr):  # keeps one block too few
+        keep, amb = orig(A, thr)
+        for r in np.ndindex(keep.shape[:-1]):
+            js = np.nonzero(keep[r])[0]
+            if len(js) > 1:
+                weakest = js[np.argmin(A[r][js])]
+                keep[r + (weakest,)] = False
+        return keep, amb
+    orig = nabla.cdf_keep
+    monkeypatch.setattr(oracle, "cdf_keep", bad)
+    with pytest.raises(AssertionError):
+        test_cdf_is_minimal_by_brute_force()
+
+
+def test_pins_catch_a_transposed_patch_order(monkeypatch, golden_dir):
+    def bad(T, H, W, P):  # patches column-major instead of row-major
+        order = []
+        for t in range(T):
+            for pc in range(-(-W // P)):
+                for pr in range(-(-H // P)):
+                    for h in range(pr * P, min((pr + 1) * P, H)):
+                        for w in range(pc * P, min((pc + 1) * P, W)):
+                            order.append(t * H * W + h * W + w)
+        return np.asarray(order)
+    monkeypatch.setattr(oracle, "fractal_order", bad)
+    with pytest.raises(AssertionError):
+        test_fractal_order_matches_hand_derivation(golden_dir)
