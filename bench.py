@@ -1,0 +1,422 @@
+"""Benchmark of the NABLA block-sparse attention path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload wan480p] [--impl ours|reference]
+
+A step is one pass of the whole path over one batch of seeded synthetic
+input: reorder Q, K, V -> block mask (pool, reduced attention, CDF threshold)
+-> block-sparse attention -> inverse reorder.  Inputs are resident in HBM when
+the timed region starts; L2 is flushed (a 2x-L2 buffer write) between steps,
+outside the per-step CUDA events.  ``value`` is the effective throughput
+4 * N^2 * d * heads * B * density / step time (TFLOP/s), summed over ranks.
+With N > 1 GPUs (torchrun) every rank runs an independent replica of the
+workload with its own seed (weak scaling; the path has no exchange step).
+
+``e2e`` is the same metric through the public API with host buffers: each
+step copies Q, K, V from pinned host memory, runs the path and copies the
+output back.  ``--impl reference`` times the fp64 CPU oracle instead, on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "block-sparse attn fwd ms & effective TFLOPS (% bf16 peak), Wan-480p shape"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_LAUNCHES_PER_STEP = 7   # reorder x3, pool, mask, attention, inverse reorder
+
+
+# ------------------------------------------------------------------ helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def attn_source_hash() -> str:
+    h = hashlib.sha256()
+    for fn in sorted(os.listdir(os.path.join(ROOT, "block_sparse_attention_fractal_b200", "csrc"))):
+        if fn.startswith("attn") or fn.endswith((".cuh", ".h")):
+            with open(os.path.join(ROOT, "block_sparse_attention_fractal_b200", "csrc", fn), "rb") as f:
+                h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if the
+    kernel sources have not changed since it was taken (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    ent = rec.get(kernel)
+    if not ent or ent.get("source_hash") != attn_source_hash():
+        return None
+    return ent.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def aggregate(per_rank_ms, per_rank_flops):
+    """Whole-job throughput: total effective FLOPs over the slowest rank's time."""
+    t = max(per_rank_ms)
+    return sum(per_rank_flops) / (t * 1e-3) / 1e12, t
+
+
+# ------------------------------------------------------------------ oracle timing
+
+def oracle_step_estimate(w, q, k, v, kv_count, kv_idx, budget_s=15.0, seed=0):
+    """Times the fp64 oracle on a bounded sample of one step of workload `w`
+    and extrapolates to a whole step.  Returns (seconds per step, description)."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    nb = w.nb
+    t0 = time.perf_counter()
+    # reorder: time a slice of the heads and scale
+    q64 = q[:, :, :1].to(torch.float64).numpy()
+    t = time.perf_counter()
+    y = oracle.reorder(q64, w.T, w.H, w.W, w.patch, w.block)
+    t_reorder = (time.perf_counter() - t) * w.heads * 3
+    # mask: one head in full
+    k64 = k[:, :, :1].to(torch.float64).numpy()
+    t = time.perf_counter()
+    yk = oracle.reorder(k64, w.T, w.H, w.W, w.patch, w.block)
+    t_mask_reorder = time.perf_counter() - t
+    t = time.perf_counter()
+    keep1, _ = oracle.block_mask(y, yk, w.T, w.H, w.W, w.patch, w.block, w.thr, w.sta) if not w.iid else (None, None)
+    t_mask = (time.perf_counter() - t) * w.heads * w.B
+    # attention: sample query blocks of head 0 until the budget is used
+    v64 = v[:, :, :1].to(torch.float64).numpy()
+    yv = oracle.reorder(v64, w.T, w.H, w.W, w.patch, w.block)
+    keep = oracle.lists_to_mask(kv_count[:, :1].numpy(), kv_idx[:, :1].numpy(), nb)
+    per_block, done = [], 0
+    t = time.perf_counter()
+    order = rng.permutation(nb)
+    for I in order:
+        oracle.masked_attention(y, yk, yv, keep, w.N, w.block, blocks=[(0, 0, int(I))])
+        done += 1
+        if time.perf_counter() - t > budget_s * 0.6 or done >= nb:
+            break
+    t_attn = (time.perf_counter() - t) / done * nb * w.heads * w.B
+    t_inverse = t_reorder / 3.0
+    total = t_reorder + t_mask + t_attn + t_inverse
+    desc = (f"fp64 oracle: reorder of 1 head x3 tensors, mask of 1 head in full, attention of {done} of "
+            f"{nb * w.heads * w.B} query blocks; extrapolated linearly to one whole step "
+            f"(wall {time.perf_counter() - t0:.1f} s)")
+    return total, desc
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------ main legs
+
+def run_reference(args, w):
+    """--impl reference: the fp64 oracle on host cores, a bounded sample per step."""
+    import block_sparse_attention_fractal_b200.synth as synth
+    q, k, v = synth.make_qkv(w)
+    if w.iid:
+        cnt, idx = synth.random_block_lists(w.B, w.heads, w.nb, 0.2, w.seed)
+    else:
+        import oracle
+        # the oracle's own mask for head 0 decides the sampled attention work
+        y = oracle.reorder(q[:, :, :1].double().numpy(), w.T, w.H, w.W, w.patch, w.block)
+        yk = oracle.reorder(k[:, :, :1].double().numpy(), w.T, w.H, w.W, w.patch, w.block)
+        keep, _ = oracle.block_mask(y, yk, w.T, w.H, w.W, w.patch, w.block, w.thr, w.sta)
+        c, i = oracle.mask_to_lists(keep)
+        cnt, idx = torch.from_numpy(c), torch.from_numpy(i)
+    dens = float(cnt[:, :1].sum()) / (w.B * 1 * w.nb * w.nb)
+    flops = 4.0 * w.N * w.N * w.d * w.heads * w.B * dens
+    budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    times = []
+    for s in range(args.warmup + args.steps):
+        t, desc = oracle_step_estimate(w, q, k, v, cnt, idx, budget_s=budget, seed=s)
+        if s >= args.warmup:
+            times.append(t)
+    step_s = statistics.mean(times)
+    value = flops / step_s / 1e12
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "density": dens},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, w, rank, world, dist):
+    import block_sparse_attention_fractal_b200 as bsa
+    import block_sparse_attention_fractal_b200.synth as synth
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wr = dataclasses.replace(w, seed=w.seed + 1000 * rank) if rank else w
+    q_h, k_h, v_h = synth.make_qkv(wr)
+    q_pin, k_pin, v_pin = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+    qd, kd, vd = q_pin.to(dev), k_pin.to(dev), v_pin.to(dev)
+    out = torch.empty_like(qd)
+    out_pin = torch.empty_like(q_pin).pin_memory()
+    shape = bsa.make_shape(w.B, w.T, w.H, w.W, w.heads, w.d, w.block, w.patch)
+    plan = bsa.NablaAttention(shape, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 64 << 20), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    sweep_lists = None
+    if w.iid:
+        dens_req = args.density if args.density is not None else 0.2
+        sweep_lists = synth.random_block_lists(w.B, w.heads, plan.nb, dens_req, w.seed)
+        plan.kv_count.copy_(sweep_lists[0])
+        plan.kv_idx.copy_(sweep_lists[1])
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def step(times=None):
+        e = [ev() for _ in range(5)] if times is not None else None
+        if e: e[0].record(stream)
+        bsa.reorder(shape, qd, plan.q)
+        bsa.reorder(shape, kd, plan.k)
+        bsa.reorder(shape, vd, plan.v)
+        if e: e[1].record(stream)
+        if not w.iid:
+            plan.mask_step(w.thr, w.sta)
+        if e: e[2].record(stream)
+        plan.attention_step()
+        if e: e[3].record(stream)
+        bsa.inverse_reorder(shape, plan.o, out)
+        if e:
+            e[4].record(stream)
+            times.append(e)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if plan.status() != 0:
+        raise RuntimeError("device status not OK after warm-up")
+    dens = float(plan.kv_count.sum().item()) / (w.B * w.heads * plan.nb * plan.nb)
+    flops_step = 4.0 * w.N * w.N * w.d * w.heads * w.B * dens
+
+    # ---- device-timed steps
+    events = []
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clocks:
+        for _ in range(args.steps):
+            flush.fill_(1)
+            step(events)
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    parts = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in events])  # ms
+    step_ms = float(parts.sum(axis=1).sum())   # total over K steps
+    per_rank = torch.tensor([step_ms], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(per_rank, op=dist.ReduceOp.MAX)
+    t_max = float(per_rank.item())
+    total_flops = flops_step * args.steps * world
+    value = total_flops / (t_max * 1e-3) / 1e12
+    ms_per_step = t_max / args.steps
+    br = parts.mean(axis=0)
+    attn_ms = float(br[2])
+
+    # ---- end to end through the public API with host buffers
+    h2d = 3 * q_pin.numel() * q_pin.element_size()
+    d2h = out_pin.numel() * out_pin.element_size()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = ev(), ev()
+    e0.record(stream)
+    for _ in range(args.steps):
+        qd.copy_(q_pin, non_blocking=True)
+        kd.copy_(k_pin, non_blocking=True)
+        vd.copy_(v_pin, non_blocking=True)
+        plan(qd, kd, vd, w.thr, w.sta, out=out) if not w.iid else step()
+        out_pin.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_t = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+        dist.barrier()
+    e2e_value = total_flops / (float(e2e_t.item()) * 1e-3) / 1e12
+    if plan.status() != 0:
+        raise RuntimeError("device status not OK after the timed steps")
+
+    if rank != 0:
+        return
+    peaks, src = load_peaks()
+    peak_tf = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak_tf_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    attn_tf = flops_step / (attn_ms * 1e-3) / 1e12
+    traffic = recorded_traffic("attn")
+    qk_bytes = 2 * w.B * w.heads * w.N * w.d * 2
+    kept = float(plan.kv_count.sum().item())
+    mask_bytes = qk_bytes + 2 * 2 * w.B * w.heads * plan.nb * w.d * 8 + 4 * (kept + w.B * w.heads * plan.nb)
+    mask_ms = float(br[1])
+    reorder_bytes = 3 * 2 * (w.B * w.heads * w.N * w.d * 2) + 3 * 2 * w.B * w.heads * (plan.Npad - w.N) * w.d
+    cpu = None
+    if args.cpu_baseline:
+        cnt_cpu, idx_cpu = plan.kv_count.cpu(), plan.kv_idx.cpu()
+        t_cpu, desc = oracle_step_estimate(w, q_h, k_h, v_h, cnt_cpu, idx_cpu, budget_s=args.cpu_budget)
+        cpu = {"value": flops_step / t_cpu / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": desc}
+    clk = clocks.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {
+            "workload": w.name, "B": w.B, "T": w.T, "H": w.H, "W": w.W, "N": w.N, "Npad": plan.Npad,
+            "heads": w.heads, "d": w.d, "block": w.block, "patch": w.patch, "thr": w.thr,
+            "sta": list(w.sta) if w.sta else None, "density": dens, "parallelism": f"replicas x{world}",
+            "l2": "flushed between steps (write of a 2x L2 buffer, outside the step events)",
+            "attn_ms": attn_ms, "attn_tflops": attn_tf, "attn_pct_bf16_peak": 100.0 * attn_tf / peak_tf,
+            "breakdown_ms": {"reorder_qkv": float(br[0]), "mask": mask_ms, "attn": attn_ms,
+                             "inverse_reorder": float(br[3])},
+            "mask_gbs": mask_bytes / (mask_ms * 1e-3) / 1e9 if mask_ms > 0 else None,
+            "mask_pct_hbm": 100.0 * mask_bytes / (mask_ms * 1e-3) / 1e9 / hbm if mask_ms > 0 else None,
+            "reorder_gbs": reorder_bytes / (float(br[0]) * 1e-3) / 1e9,
+            "mask_precision": "f64 pooled means, dots and masses",
+        },
+        "roofline": {"bound": "tensor", "achieved": attn_tf, "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": attn_tf / peak_tf, "traffic": traffic,
+                     "kernel": "attention", "peak_source": f"{src} bf16 burst",
+                     "frac_of_sustained": attn_tf / peak_tf_sus},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": KERNEL_LAUNCHES_PER_STEP * args.steps if not w.iid else 5 * args.steps,
+        "clocks": clk,
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="wan480p")
+    ap.add_argument("--density", type=float, default=None, help="density-sweep workload: kept fraction")
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    from block_sparse_attention_fractal_b200 import synth
+    w = synth.WORKLOADS[args.workload]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, w)
+        return 0
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist_mod
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        import datetime
+        dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+        dist = dist_mod
+    else:
+        torch.cuda.set_device(0)
+    try:
+        run_ours(args, w, rank, world, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

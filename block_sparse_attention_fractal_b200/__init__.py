@@ -1,0 +1,76 @@
+"""B200-native NABLA-style block-sparse attention for video diffusion transformers.
+
+The compute path is libbsa.so (hand-written CUDA for sm_100a, C ABI in
+include/bsa.h); this package only marshals torch tensors into it.
+
+    import block_sparse_attention_fractal_b200 as bsa
+    shape = bsa.make_shape(B, T, H, W, heads, d, block, patch)
+    plan = bsa.NablaAttention(shape, device="cuda")
+    out = plan(q, k, v, thr=0.2)            # q, k, v: [B, T*H*W, heads, d] bf16
+
+The four steps can also be called one by one: ``reorder``,
+``build_block_mask``, ``attn_fwd``, ``inverse_reorder``.
+"""
+from __future__ import annotations
+
+from typing import Optional, Tuple
+
+import torch
+
+from ._lib import (BsaError, Shape, attn_fwd, build_block_mask, check_device_status, inverse_reorder,  # noqa: F401
+                   lib, make_shape, num_blocks, padded_len, reorder, seq_len, validate_shape, workspace_bytes,
+                   workspace_init, LIB_PATH)
+
+__all__ = ["BsaError", "Shape", "make_shape", "NablaAttention", "reorder", "inverse_reorder", "build_block_mask",
+           "attn_fwd", "check_device_status", "workspace_bytes", "workspace_init", "padded_len", "num_blocks",
+           "seq_len", "validate_shape", "LIB_PATH"]
+
+
+class NablaAttention:
+    """Owns the device buffers of one shape and runs the whole path on the
+    current stream: reorder Q, K, V -> block mask -> block-sparse attention ->
+    inverse reorder.  Buffers are allocated once (torch) and reused."""
+
+    def __init__(self, shape: Shape, device="cuda", with_mask: bool = False, with_lse: bool = False):
+        st = validate_shape(shape)
+        if st != 0:
+            raise BsaError(st, "bsa_validate_shape")
+        self.shape = shape
+        dev = torch.device(device)
+        B, heads, d = shape.B, shape.heads, shape.d
+        Npad, nb = padded_len(shape), num_blocks(shape)
+        self.N, self.Npad, self.nb = seq_len(shape), Npad, nb
+        kw = dict(device=dev)
+        self.q = torch.empty(B, heads, Npad, d, dtype=torch.bfloat16, **kw)
+        self.k = torch.empty_like(self.q)
+        self.v = torch.empty_like(self.q)
+        self.o = torch.empty_like(self.q)
+        self.kv_count = torch.empty(B, heads, nb, dtype=torch.int32, **kw)
+        self.kv_idx = torch.empty(B, heads, nb, nb, dtype=torch.int32, **kw)
+        self.mask = torch.empty(B, heads, nb, nb, dtype=torch.uint8, **kw) if with_mask else None
+        self.lse = torch.empty(B, heads, Npad, dtype=torch.float32, **kw) if with_lse else None
+        ws_bytes = workspace_bytes(shape)
+        self.ws = torch.empty((ws_bytes + 15) // 16 * 16, dtype=torch.uint8, **kw)
+        workspace_init(self.ws)
+
+    def mask_step(self, thr: float, sta: Optional[Tuple[int, int, int]] = None) -> None:
+        build_block_mask(self.shape, self.q, self.k, thr, sta, self.kv_count, self.kv_idx, self.mask, self.ws)
+
+    def attention_step(self, scale: float = 0.0) -> None:
+        attn_fwd(self.shape, self.q, self.k, self.v, self.kv_count, self.kv_idx, scale, self.o, self.lse, self.ws)
+
+    def __call__(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, thr: float,
+                 sta: Optional[Tuple[int, int, int]] = None, scale: float = 0.0,
+                 out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        reorder(self.shape, q, self.q)
+        reorder(self.shape, k, self.k)
+        reorder(self.shape, v, self.v)
+        self.mask_step(thr, sta)
+        self.attention_step(scale)
+        if out is None:
+            out = torch.empty_like(q)
+        inverse_reorder(self.shape, self.o, out)
+        return out
+
+    def status(self) -> int:
+        return check_device_status(self.ws)

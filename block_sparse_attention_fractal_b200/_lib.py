@@ -1,0 +1,146 @@
+"""ctypes binding of libbsa.so: argument marshalling only.
+
+Every function takes torch tensors (device memory owned by the caller), passes
+their raw pointers, sizes and the current CUDA stream to the C ABI declared in
+include/bsa.h, and raises ``BsaError`` on a non-OK status.  There is no
+fallback: if the shared library is missing, importing this module fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbsa.so")
+
+BSA_OK = 0
+STATUS_NAMES = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_UNSUPPORTED", 3: "BSA_ERR_CUDA",
+                4: "BSA_ERR_DEVICE_INDEX", 5: "BSA_ERR_TIMEOUT"}
+
+
+class BsaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+
+
+class Shape(ctypes.Structure):
+    """bsa_shape: B, T, H, W, heads, d, block, patch."""
+    _fields_ = [(n, ctypes.c_int32) for n in ("B", "T", "H", "W", "heads", "d", "block", "patch")]
+
+    def __repr__(self) -> str:
+        return "Shape(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libbsa.so not built ({LIB_PATH}); run python -m block_sparse_attention_fractal_b200.build")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.c_void_p
+    S = ctypes.POINTER(Shape)
+    st = ctypes.c_int
+    sig = {
+        "bsa_validate_shape": (st, [S]),
+        "bsa_seq_len": (ctypes.c_int64, [S]),
+        "bsa_padded_len": (ctypes.c_int64, [S]),
+        "bsa_num_blocks": (ctypes.c_int64, [S]),
+        "bsa_workspace_bytes": (ctypes.c_size_t, [S]),
+        "bsa_workspace_init": (st, [P, ctypes.c_size_t, P]),
+        "bsa_reorder": (st, [S, P, P, P]),
+        "bsa_inverse_reorder": (st, [S, P, P, P]),
+        "bsa_build_block_mask": (st, [S, P, P, ctypes.c_float, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                      P, P, P, P, ctypes.c_size_t, P]),
+        "bsa_attn_fwd": (st, [S, P, P, P, P, P, ctypes.c_float, P, P, P, ctypes.c_size_t, P]),
+        "bsa_check_device_status": (st, [P, P]),
+        "bsa_status_string": (ctypes.c_char_p, [st]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libbsa must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(device: Optional[torch.device] = None) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _check(status: int, where: str) -> None:
+    if status != BSA_OK:
+        raise BsaError(status, where)
+
+
+def make_shape(B: int, T: int, H: int, W: int, heads: int, d: int, block: int, patch: int) -> Shape:
+    return Shape(B, T, H, W, heads, d, block, patch)
+
+
+def validate_shape(s: Shape) -> int:
+    return lib.bsa_validate_shape(ctypes.byref(s))
+
+
+def seq_len(s: Shape) -> int:
+    return lib.bsa_seq_len(ctypes.byref(s))
+
+
+def padded_len(s: Shape) -> int:
+    return lib.bsa_padded_len(ctypes.byref(s))
+
+
+def num_blocks(s: Shape) -> int:
+    return lib.bsa_num_blocks(ctypes.byref(s))
+
+
+def workspace_bytes(s: Shape) -> int:
+    return lib.bsa_workspace_bytes(ctypes.byref(s))
+
+
+def workspace_init(ws: torch.Tensor) -> None:
+    _check(lib.bsa_workspace_init(_ptr(ws), ws.numel() * ws.element_size(), _stream(ws.device)),
+           "bsa_workspace_init")
+
+
+def reorder(s: Shape, x_bnhd: torch.Tensor, y_bhnd: torch.Tensor) -> None:
+    _check(lib.bsa_reorder(ctypes.byref(s), _ptr(x_bnhd), _ptr(y_bhnd), _stream(x_bnhd.device)), "bsa_reorder")
+
+
+def inverse_reorder(s: Shape, y_bhnd: torch.Tensor, x_bnhd: torch.Tensor) -> None:
+    _check(lib.bsa_inverse_reorder(ctypes.byref(s), _ptr(y_bhnd), _ptr(x_bnhd), _stream(y_bhnd.device)),
+           "bsa_inverse_reorder")
+
+
+def build_block_mask(s: Shape, q_bhnd: torch.Tensor, k_bhnd: torch.Tensor, thr: float,
+                     sta: Optional[Tuple[int, int, int]], kv_count: torch.Tensor, kv_idx: torch.Tensor,
+                     mask: Optional[torch.Tensor], ws: torch.Tensor) -> None:
+    st_t, st_h, st_w = sta if sta is not None else (-1, -1, -1)
+    _check(lib.bsa_build_block_mask(ctypes.byref(s), _ptr(q_bhnd), _ptr(k_bhnd), float(thr), st_t, st_h, st_w,
+                                    _ptr(kv_count), _ptr(kv_idx), _ptr(mask), _ptr(ws),
+                                    ws.numel() * ws.element_size(), _stream(q_bhnd.device)),
+           "bsa_build_block_mask")
+
+
+def attn_fwd(s: Shape, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, kv_count: torch.Tensor,
+             kv_idx: torch.Tensor, scale: float, o: torch.Tensor, lse: Optional[torch.Tensor],
+             ws: torch.Tensor) -> None:
+    _check(lib.bsa_attn_fwd(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(kv_count), _ptr(kv_idx),
+                            float(scale), _ptr(o), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(),
+                            _stream(q.device)),
+           "bsa_attn_fwd")
+
+
+def check_device_status(ws: torch.Tensor) -> int:
+    """Synchronises the current stream; returns the device status (0 = OK) and clears it."""
+    return lib.bsa_check_device_status(_ptr(ws), _stream(ws.device))

@@ -1,0 +1,178 @@
+// C ABI of libbsa (declared in include/bsa.h): argument checking, workspace
+// layout and kernel launches.  No entry point allocates, frees or
+// synchronises, except bsa_check_device_status.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.h"
+
+using bsa::Ctrl;
+using bsa::Dims;
+
+namespace {
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+bsa_status check_shape(const bsa_shape* s, Dims* out) {
+  if (s == nullptr) return BSA_ERR_INVALID_ARG;
+  if (s->B < 1 || s->T < 1 || s->H < 1 || s->W < 1 || s->heads < 1 || s->patch < 1) return BSA_ERR_INVALID_ARG;
+  if (s->d != 64 && s->d != 128) return BSA_ERR_INVALID_ARG;
+  if (s->block != 64 && s->block != 128) return BSA_ERR_INVALID_ARG;
+  const int64_t N = (int64_t)s->T * s->H * s->W;
+  if (N > (int64_t)1 << 30) return BSA_ERR_UNSUPPORTED;
+  const int64_t Npad = (N + s->block - 1) / s->block * s->block;
+  const int64_t elems = (int64_t)s->B * s->heads * Npad * s->d;
+  if (elems > ((int64_t)1 << 40)) return BSA_ERR_UNSUPPORTED;
+  if ((int64_t)s->B * s->heads > 65535 * 64 || s->heads > 65535 || s->B > 65535) return BSA_ERR_UNSUPPORTED;
+  if (out != nullptr) {
+    out->B = s->B;
+    out->T = s->T;
+    out->H = s->H;
+    out->W = s->W;
+    out->heads = s->heads;
+    out->d = s->d;
+    out->bs = s->block;
+    out->P = s->patch;
+    out->N = (int)N;
+    out->Npad = (int)Npad;
+    out->nb = (int)(Npad / s->block);
+  }
+  return BSA_OK;
+}
+
+size_t pooled_bytes(const Dims& g) { return (size_t)g.B * g.heads * g.nb * g.d * sizeof(double); }
+
+size_t workspace_bytes(const Dims& g) { return sizeof(Ctrl) + 2 * pooled_bytes(g); }
+
+bsa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+bsa_status bsa_validate_shape(const bsa_shape* s) {
+  Dims g;
+  bsa_status st = check_shape(s, &g);
+  if (st != BSA_OK) return st;
+  if (g.nb > BSA_MAX_BLOCKS) return BSA_ERR_UNSUPPORTED;
+  return BSA_OK;
+}
+
+int64_t bsa_seq_len(const bsa_shape* s) {
+  Dims g;
+  return check_shape(s, &g) == BSA_OK ? g.N : -1;
+}
+
+int64_t bsa_padded_len(const bsa_shape* s) {
+  Dims g;
+  return check_shape(s, &g) == BSA_OK ? g.Npad : -1;
+}
+
+int64_t bsa_num_blocks(const bsa_shape* s) {
+  Dims g;
+  return check_shape(s, &g) == BSA_OK ? g.nb : -1;
+}
+
+size_t bsa_workspace_bytes(const bsa_shape* s) {
+  Dims g;
+  return check_shape(s, &g) == BSA_OK ? workspace_bytes(g) : 0;
+}
+
+bsa_status bsa_workspace_init(void* workspace, size_t ws_bytes, bsa_stream_t stream) {
+  if (workspace == nullptr || !aligned16(workspace) || ws_bytes < sizeof(Ctrl)) return BSA_ERR_INVALID_ARG;
+  return from_cuda(cudaMemsetAsync(workspace, 0, sizeof(Ctrl), (cudaStream_t)stream));
+}
+
+bsa_status bsa_reorder(const bsa_shape* s, const void* x_bnhd, void* y_bhnd, bsa_stream_t stream) {
+  Dims g;
+  bsa_status st = check_shape(s, &g);
+  if (st != BSA_OK) return st;
+  if (x_bnhd == nullptr || y_bhnd == nullptr || !aligned16(x_bnhd) || !aligned16(y_bhnd) || x_bnhd == y_bhnd)
+    return BSA_ERR_INVALID_ARG;
+  return from_cuda(bsa::launch_reorder(g, x_bnhd, y_bhnd, (cudaStream_t)stream));
+}
+
+bsa_status bsa_inverse_reorder(const bsa_shape* s, const void* y_bhnd, void* x_bnhd, bsa_stream_t stream) {
+  Dims g;
+  bsa_status st = check_shape(s, &g);
+  if (st != BSA_OK) return st;
+  if (x_bnhd == nullptr || y_bhnd == nullptr || !aligned16(x_bnhd) || !aligned16(y_bhnd) || x_bnhd == y_bhnd)
+    return BSA_ERR_INVALID_ARG;
+  return from_cuda(bsa::launch_inverse_reorder(g, y_bhnd, x_bnhd, (cudaStream_t)stream));
+}
+
+bsa_status bsa_build_block_mask(const bsa_shape* s, const void* q_bhnd, const void* k_bhnd, float thr,
+                                int32_t sta_t, int32_t sta_h, int32_t sta_w, int32_t* kv_count, int32_t* kv_idx,
+                                uint8_t* mask_or_null, void* workspace, size_t ws_bytes, bsa_stream_t stream) {
+  Dims g;
+  bsa_status st = check_shape(s, &g);
+  if (st != BSA_OK) return st;
+  if (g.nb > BSA_MAX_BLOCKS) return BSA_ERR_UNSUPPORTED;
+  if (!(thr >= 0.0f && thr < 1.0f)) return BSA_ERR_INVALID_ARG;
+  if (q_bhnd == nullptr || k_bhnd == nullptr || kv_count == nullptr || kv_idx == nullptr || workspace == nullptr)
+    return BSA_ERR_INVALID_ARG;
+  if (!aligned16(q_bhnd) || !aligned16(k_bhnd) || !aligned16(kv_count) || !aligned16(kv_idx) ||
+      !aligned16(workspace))
+    return BSA_ERR_INVALID_ARG;
+  if (ws_bytes < workspace_bytes(g)) return BSA_ERR_INVALID_ARG;
+  const bool sta = sta_t >= 0 && sta_h >= 0 && sta_w >= 0;
+  double* qbar = (double*)((char*)workspace + sizeof(Ctrl));
+  double* kbar = qbar + pooled_bytes(g) / sizeof(double);
+  cudaStream_t cs = (cudaStream_t)stream;
+  cudaError_t e = bsa::launch_pool(g, q_bhnd, k_bhnd, qbar, kbar, cs);
+  if (e != cudaSuccess) return BSA_ERR_CUDA;
+  e = bsa::launch_mask(g, qbar, kbar, (double)thr, sta ? sta_t : -1, sta ? sta_h : -1, sta ? sta_w : -1, kv_count,
+                       kv_idx, mask_or_null, cs);
+  return from_cuda(e);
+}
+
+bsa_status bsa_attn_fwd(const bsa_shape* s, const void* q, const void* k, const void* v, const int32_t* kv_count,
+                        const int32_t* kv_idx, float scale, void* o, float* lse_or_null, void* workspace,
+                        size_t ws_bytes, bsa_stream_t stream) {
+  Dims g;
+  bsa_status st = check_shape(s, &g);
+  if (st != BSA_OK) return st;
+  if (g.nb > BSA_MAX_BLOCKS) return BSA_ERR_UNSUPPORTED;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || kv_count == nullptr || kv_idx == nullptr ||
+      workspace == nullptr)
+    return BSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(kv_count) ||
+      !aligned16(kv_idx) || !aligned16(workspace) || (lse_or_null != nullptr && !aligned16(lse_or_null)))
+    return BSA_ERR_INVALID_ARG;
+  if (ws_bytes < workspace_bytes(g)) return BSA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return BSA_ERR_INVALID_ARG;
+  if (scale == 0.0f) scale = (float)(1.0 / std::sqrt((double)g.d));
+  Ctrl* ctrl = (Ctrl*)workspace;
+  return from_cuda(bsa::launch_attn_mma(g, q, k, v, kv_count, kv_idx, scale, o, lse_or_null, ctrl,
+                                        (cudaStream_t)stream));
+}
+
+bsa_status bsa_check_device_status(void* workspace, bsa_stream_t stream) {
+  if (workspace == nullptr || !aligned16(workspace)) return BSA_ERR_INVALID_ARG;
+  cudaStream_t cs = (cudaStream_t)stream;
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return BSA_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return BSA_ERR_CUDA;
+  if (word != 0u) {
+    if (cudaMemset(workspace, 0, sizeof(Ctrl)) != cudaSuccess) return BSA_ERR_CUDA;
+  }
+  if (word & bsa::kErrTimeout) return BSA_ERR_TIMEOUT;
+  if (word & (bsa::kErrIndex | bsa::kErrCount)) return BSA_ERR_DEVICE_INDEX;
+  return BSA_OK;
+}
+
+const char* bsa_status_string(bsa_status st) {
+  switch (st) {
+    case BSA_OK: return "BSA_OK";
+    case BSA_ERR_INVALID_ARG: return "BSA_ERR_INVALID_ARG";
+    case BSA_ERR_UNSUPPORTED: return "BSA_ERR_UNSUPPORTED";
+    case BSA_ERR_CUDA: return "BSA_ERR_CUDA";
+    case BSA_ERR_DEVICE_INDEX: return "BSA_ERR_DEVICE_INDEX";
+    case BSA_ERR_TIMEOUT: return "BSA_ERR_TIMEOUT";
+  }
+  return "BSA_ERR_UNKNOWN";
+}
+
+}  // extern "C"

@@ -1,0 +1,25 @@
+// Internal launchers of libbsa (host side).  Argument checking happens in
+// bsa_api.cu before any of these is called.
+#pragma once
+
+#include <cuda_runtime.h>
+#include "common.cuh"
+
+namespace bsa {
+
+cudaError_t launch_reorder(const Dims& g, const void* x_bnhd, void* y_bhnd, cudaStream_t st);
+cudaError_t launch_inverse_reorder(const Dims& g, const void* y_bhnd, void* x_bnhd, cudaStream_t st);
+
+// Block means of Q and K (double) into `qbar`, `kbar` [B, heads, nb, d].
+cudaError_t launch_pool(const Dims& g, const void* q, const void* k, double* qbar, double* kbar, cudaStream_t st);
+
+// Reduced attention + CDF threshold (+ STA union) -> KV lists.
+cudaError_t launch_mask(const Dims& g, const double* qbar, const double* kbar, double thr, int sta_t, int sta_h,
+                        int sta_w, int32_t* kv_count, int32_t* kv_idx, uint8_t* mask, cudaStream_t st);
+
+// Block-sparse attention on the legacy warp-level mma.sync tensor-core path
+// (baseline kernel; any supported shape).
+cudaError_t launch_attn_mma(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
+                            const int32_t* kv_idx, float scale, void* o, float* lse, Ctrl* ctrl, cudaStream_t st);
+
+}  // namespace bsa

@@ -1,0 +1,334 @@
+// Adaptive block mask (NABLA summary, Metodologia 2 and 3):
+//   pool_kernel: block means of Q and K ("Submuestreo"), double precision;
+//   mask_kernel: reduced attention softmax(qbar kbar^T / sqrt(d)) per row
+//                ("Atencion Reducida"), the CDF threshold ("Umbralizacion CDF"),
+//                the optional STA union, and the ascending KV index lists that
+//                the attention kernel walks ("Expansion").
+//
+// Precision: bf16 values summed in double are exact, so the block means equal
+// the exact mean rounded once.  Dot products, exp and the probability masses
+// are double, which keeps every threshold decision within ~1e-15 of the exact
+// one; only rows whose prefix mass sits that close to 1 - thr can differ from
+// an exact evaluation.
+#include <cfloat>
+#include <cmath>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace bsa {
+
+namespace {
+
+// ---------------------------------------------------------------- pooling
+
+constexpr int kPoolThreads = 256;
+
+// grid (nb, heads, 2*B): z = 2*b + {0: Q, 1: K}.  Each thread accumulates 8
+// columns of one 16-byte vector over every (256/vec)-th row of the block.
+template <int D, int BS>
+__global__ void __launch_bounds__(kPoolThreads) pool_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
+                                                            double* __restrict__ qbar, double* __restrict__ kbar,
+                                                            Dims g) {
+  constexpr int kVec = D / 8;
+  constexpr int kRowsPerPass = kPoolThreads / kVec;
+  constexpr int kIters = BS / kRowsPerPass;
+  __shared__ double part[kRowsPerPass][D];
+
+  const int I = blockIdx.x;
+  const int head = blockIdx.y;
+  const int which = blockIdx.z & 1;
+  const int b = blockIdx.z >> 1;
+  const uint4* src = which ? k : q;
+  double* dst = which ? kbar : qbar;
+  const size_t bh = (size_t)b * g.heads + head;
+  const int lo = I * BS;
+  const int cnt = min(BS, g.N - lo);
+  const int c = threadIdx.x % kVec;
+  const int r0 = threadIdx.x / kVec;
+
+  uint4 raw[kIters];
+#pragma unroll
+  for (int it = 0; it < kIters; ++it) {
+    const int r = r0 + it * kRowsPerPass;
+    raw[it] = (r < cnt) ? __ldcs(src + (bh * g.Npad + lo + r) * kVec + c) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  double acc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = 0.0;
+#pragma unroll
+  for (int it = 0; it < kIters; ++it) {
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[it]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(h2[j]);
+      acc[2 * j] += (double)f.x;
+      acc[2 * j + 1] += (double)f.y;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) part[r0][c * 8 + j] = acc[j];
+  __syncthreads();
+  for (int col = threadIdx.x; col < D; col += kPoolThreads) {
+    double s = 0.0;
+#pragma unroll 8
+    for (int i = 0; i < kRowsPerPass; ++i) s += part[i][col];
+    dst[(bh * g.nb + I) * D + col] = s / (double)cnt;
+  }
+}
+
+// ------------------------------------------------------------- mask rows
+
+constexpr int kMaskRows = 16;                 // query-block rows per CTA (one warp each)
+constexpr int kMaskThreads = 32 * kMaskRows;  // 512
+constexpr int kMaxJ = BSA_MAX_BLOCKS / 32;
+
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ int warp_sum(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ double warp_max(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ unsigned long long warp_max(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long w = __shfl_xor_sync(0xffffffffu, v, o);
+    v = w > v ? w : v;
+  }
+  return v;
+}
+
+__device__ __forceinline__ void block_tile(int I, const Dims& g, int& t, int& th, int& tw) {
+  const int n = fractal_token(I * g.bs, g.H, g.W, g.P);
+  const int HW = g.H * g.W;
+  t = n / HW;
+  const int rem = n - t * HW;
+  const int h = rem / g.W;
+  th = h / g.P;
+  tw = (rem - h * g.W) / g.P;
+}
+
+// grid (ceil(nb / kMaskRows), heads, B).  Dynamic smem: qbar rows
+// [kMaskRows][D] then scores [kMaskRows][nb], both double.
+template <int D>
+__global__ void __launch_bounds__(kMaskThreads) mask_kernel(const double* __restrict__ qbar,
+                                                            const double* __restrict__ kbar, Dims g, double thr,
+                                                            double scale, int sta_t, int sta_h, int sta_w,
+                                                            int32_t* __restrict__ kv_count,
+                                                            int32_t* __restrict__ kv_idx, uint8_t* __restrict__ mask) {
+  extern __shared__ __align__(16) double smem[];
+  double* qs = smem;                       // [kMaskRows][D]
+  double* sc = smem + kMaskRows * D;       // [kMaskRows][nb]
+  const int nb = g.nb;
+  const int head = blockIdx.y;
+  const int b = blockIdx.z;
+  const size_t bh = (size_t)b * g.heads + head;
+  const int I0 = blockIdx.x * kMaskRows;
+  const int rows = min(kMaskRows, nb - I0);
+
+  for (int i = threadIdx.x; i < kMaskRows * D; i += kMaskThreads) {
+    const int r = i / D;
+    qs[i] = (r < rows) ? qbar[(bh * nb + I0 + r) * D + (i % D)] : 0.0;
+  }
+  __syncthreads();
+
+  // Phase 1: scores s[r][J] = scale * qbar_r . kbar_J; each thread owns whole
+  // columns J and reuses every kbar element across the CTA's rows.
+  const double2* q2 = reinterpret_cast<const double2*>(qs);
+  for (int J = threadIdx.x; J < nb; J += kMaskThreads) {
+    const double2* k2 = reinterpret_cast<const double2*>(kbar + (bh * nb + J) * D);
+    double acc[kMaskRows];
+#pragma unroll
+    for (int r = 0; r < kMaskRows; ++r) acc[r] = 0.0;
+#pragma unroll 4
+    for (int c = 0; c < D / 2; ++c) {
+      const double2 kv = __ldg(k2 + c);
+#pragma unroll
+      for (int r = 0; r < kMaskRows; ++r) {
+        const double2 qv = q2[r * (D / 2) + c];
+        acc[r] = fma(qv.x, kv.x, acc[r]);
+        acc[r] = fma(qv.y, kv.y, acc[r]);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kMaskRows; ++r) sc[r * nb + J] = acc[r] * scale;
+  }
+  __syncthreads();
+
+  // Phase 2: one warp per row.  Lane L holds J = L + 32 i.
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= rows) return;
+  const int I = I0 + warp;
+  const double* srow = sc + warp * nb;
+
+  double a[kMaxJ];
+  double mx = -DBL_MAX;
+#pragma unroll
+  for (int i = 0; i < kMaxJ; ++i) {
+    const int J = lane + 32 * i;
+    a[i] = (J < nb) ? srow[J] : -DBL_MAX;
+    mx = fmax(mx, a[i]);
+  }
+  mx = warp_max(mx);
+  double z = 0.0;
+#pragma unroll
+  for (int i = 0; i < kMaxJ; ++i) {
+    const int J = lane + 32 * i;
+    a[i] = (J < nb) ? exp(a[i] - mx) : 0.0;
+    z += a[i];
+  }
+  z = warp_sum(z);
+#pragma unroll
+  for (int i = 0; i < kMaxJ; ++i) a[i] = a[i] / z;  // A = e / sum(e), a true division
+
+  // keep bits: bit i of `keep` <-> J = lane + 32 i
+  uint32_t keep = 0u;
+  const double target = 1.0 - thr;
+  double total = 0.0;
+#pragma unroll
+  for (int i = 0; i < kMaxJ; ++i) total += a[i];
+  total = warp_sum(total);
+  if (thr == 0.0 || total < target) {
+    // thr == 0 keeps every block; so does a row whose whole mass rounds below 1 - thr.
+#pragma unroll
+    for (int i = 0; i < kMaxJ; ++i)
+      if (lane + 32 * i < nb) keep |= 1u << i;
+  } else {
+    // Largest key v (bit pattern of a non-negative double, monotone in value)
+    // with mass(A >= v) >= target: the probability of the last kept block.
+    unsigned long long lo = 0ull, hi = ~0ull;
+    int cnt_lo = nb, cnt_hi = 0;
+    bool unique = false;
+    for (int bit = 62; bit >= 0; --bit) {
+      const unsigned long long cand = lo | (1ull << bit);
+      double m = 0.0;
+      int c = 0;
+#pragma unroll
+      for (int i = 0; i < kMaxJ; ++i) {
+        const bool ge = (lane + 32 * i < nb) && (unsigned long long)__double_as_longlong(a[i]) >= cand;
+        m += ge ? a[i] : 0.0;
+        c += ge ? 1 : 0;
+      }
+      m = warp_sum(m);
+      c = warp_sum(c);
+      if (m >= target) {
+        lo = cand;
+        cnt_lo = c;
+      } else {
+        hi = cand;
+        cnt_hi = c;
+      }
+      if (cnt_lo - cnt_hi == 1) {
+        unique = true;
+        break;
+      }
+    }
+    unsigned long long vb = lo;
+    if (unique) {  // the single block with lo <= key < hi
+      unsigned long long best = 0ull;
+#pragma unroll
+      for (int i = 0; i < kMaxJ; ++i) {
+        const unsigned long long key = (unsigned long long)__double_as_longlong(a[i]);
+        if (lane + 32 * i < nb && key < hi && key > best) best = key;
+      }
+      vb = warp_max(best);
+    }
+    // Every block above the boundary value is kept; blocks equal to it are
+    // added in ascending index order until the mass reaches the target.
+    double run = 0.0;
+#pragma unroll
+    for (int i = 0; i < kMaxJ; ++i) {
+      const unsigned long long key = (unsigned long long)__double_as_longlong(a[i]);
+      if (lane + 32 * i < nb && key > vb) {
+        keep |= 1u << i;
+        run += a[i];
+      }
+    }
+    run = warp_sum(run);
+    const double vval = __longlong_as_double((long long)vb);
+#pragma unroll
+    for (int i = 0; i < kMaxJ; ++i) {
+      if (run >= target) break;
+      const unsigned long long key = (unsigned long long)__double_as_longlong(a[i]);
+      uint32_t ties = __ballot_sync(0xffffffffu, (lane + 32 * i < nb) && key == vb);
+      while (ties != 0u && run < target) {
+        const int src = __ffs(ties) - 1;
+        ties &= ties - 1u;
+        if (lane == src) keep |= 1u << i;
+        run += vval;
+      }
+    }
+  }
+
+  if (sta_t >= 0) {
+    int ti, hi_, wi;
+    block_tile(I, g, ti, hi_, wi);
+#pragma unroll 1
+    for (int i = 0; i < kMaxJ; ++i) {
+      const int J = lane + 32 * i;
+      if (J >= nb) break;
+      int tj, hj, wj;
+      block_tile(J, g, tj, hj, wj);
+      if (abs(ti - tj) <= sta_t && abs(hi_ - hj) <= sta_h && abs(wi - wj) <= sta_w) keep |= 1u << i;
+    }
+  }
+
+  const size_t row = bh * nb + I;
+  int base = 0;
+  const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int i = 0; i < kMaxJ; ++i) {
+    const int J = lane + 32 * i;
+    const bool k = (keep >> i) & 1u;
+    const uint32_t bal = __ballot_sync(0xffffffffu, k);
+    if (k) kv_idx[row * nb + base + __popc(bal & lt)] = J;
+    if (mask != nullptr && J < nb) mask[row * nb + J] = k ? 1 : 0;
+    base += __popc(bal);
+  }
+  if (lane == 0) kv_count[row] = base;
+}
+
+}  // namespace
+
+cudaError_t launch_pool(const Dims& g, const void* q, const void* k, double* qbar, double* kbar, cudaStream_t st) {
+  dim3 grid(g.nb, g.heads, 2 * g.B);
+  const uint4* q4 = (const uint4*)q;
+  const uint4* k4 = (const uint4*)k;
+  if (g.d == 128 && g.bs == 64) pool_kernel<128, 64><<<grid, kPoolThreads, 0, st>>>(q4, k4, qbar, kbar, g);
+  else if (g.d == 128 && g.bs == 128) pool_kernel<128, 128><<<grid, kPoolThreads, 0, st>>>(q4, k4, qbar, kbar, g);
+  else if (g.d == 64 && g.bs == 64) pool_kernel<64, 64><<<grid, kPoolThreads, 0, st>>>(q4, k4, qbar, kbar, g);
+  else pool_kernel<64, 128><<<grid, kPoolThreads, 0, st>>>(q4, k4, qbar, kbar, g);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mask(const Dims& g, const double* qbar, const double* kbar, double thr, int sta_t, int sta_h,
+                        int sta_w, int32_t* kv_count, int32_t* kv_idx, uint8_t* mask, cudaStream_t st) {
+  dim3 grid((g.nb + kMaskRows - 1) / kMaskRows, g.heads, g.B);
+  const size_t smem = (size_t)kMaskRows * (g.d + g.nb) * sizeof(double);
+  const double scale = 1.0 / std::sqrt((double)g.d);
+  cudaError_t e;
+  if (g.d == 128) {
+    e = cudaFuncSetAttribute(mask_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    mask_kernel<128><<<grid, kMaskThreads, smem, st>>>(qbar, kbar, g, thr, scale, sta_t, sta_h, sta_w, kv_count,
+                                                       kv_idx, mask);
+  } else {
+    e = cudaFuncSetAttribute(mask_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    mask_kernel<64><<<grid, kMaskThreads, smem, st>>>(qbar, kbar, g, thr, scale, sta_t, sta_h, sta_w, kv_count,
+                                                      kv_idx, mask);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace bsa

@@ -1,0 +1,163 @@
+/*
+ * bsa.h -- C ABI of the B200 block-sparse video attention library (libbsa.so).
+ *
+ * The library implements NABLA-style content-adaptive block-sparse
+ * self-attention as described in the NABLA technical summary
+ * ("NABLA - Atencion de Bloque Adaptativa al Vecindario para la Generacion
+ * Eficiente de Video", gist.science/es/paper/2507.13546), section
+ * "Metodologia":
+ *   1. fractal P x P token reorder           -> bsa_reorder / bsa_inverse_reorder
+ *   2. block mean-pooling of Q and K,
+ *      reduced attention map, per-row CDF
+ *      threshold (optionally united with a
+ *      static sliding-tile window, item 3)  -> bsa_build_block_mask
+ *   3. attention restricted to the kept
+ *      N x N tiles ("Expansion")             -> bsa_attn_fwd
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Device pointers refer to memory of the current CUDA device; every call is
+ *    asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream)
+ *    and never synchronises, except bsa_check_device_status.
+ *  - The caller owns every buffer.  The library never allocates or frees
+ *    memory.  Buffers must be contiguous and 16-byte aligned.
+ *  - Tensors are bf16 (IEEE-754 binary16 "brain float", __nv_bfloat16).
+ *  - Layouts:  model order  [B, N, heads, d]     (token n = t*H*W + h*W + w)
+ *              kernel order [B, heads, Npad, d]  (fractal order, zero tail)
+ *    with N = T*H*W, Npad = ceil(N / block) * block, nb = Npad / block.
+ *  - Argument errors are reported synchronously by the return value and
+ *    launch nothing.  Errors found on the device (an out-of-range KV index or
+ *    count, a bounded wait that expired) never trap: they set bits of an error
+ *    word held in the workspace, which bsa_check_device_status reports.
+ */
+#ifndef BSA_H
+#define BSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define BSA_API __attribute__((visibility("default")))
+#else
+#define BSA_API
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st* bsa_stream_t;
+
+typedef enum bsa_status {
+  BSA_OK = 0,
+  BSA_ERR_INVALID_ARG = 1,   /* bad shape, pointer, alignment, threshold or workspace size   */
+  BSA_ERR_UNSUPPORTED = 2,   /* valid but outside what the kernels implement (e.g. nb > max) */
+  BSA_ERR_CUDA = 3,          /* a CUDA runtime call or kernel launch failed                   */
+  BSA_ERR_DEVICE_INDEX = 4,  /* device saw a KV index outside [0, nb) or a count outside [1, nb] */
+  BSA_ERR_TIMEOUT = 5        /* a bounded device-side wait expired                           */
+} bsa_status;
+
+/* Problem shape.  d in {64, 128}; block in {64, 128}; patch >= 1. */
+typedef struct bsa_shape {
+  int32_t B;      /* batch                                  */
+  int32_t T;      /* latent frames                          */
+  int32_t H;      /* latent height                          */
+  int32_t W;      /* latent width                           */
+  int32_t heads;  /* attention heads                        */
+  int32_t d;      /* head dimension                         */
+  int32_t block;  /* block size (tokens per mask block)     */
+  int32_t patch;  /* P of the fractal P x P reorder         */
+} bsa_shape;
+
+/* Largest nb (= Npad / block) that bsa_build_block_mask and bsa_attn_fwd accept. */
+#define BSA_MAX_BLOCKS 1024
+
+/* BSA_OK when the shape is one the kernels implement, else the reason. */
+BSA_API bsa_status bsa_validate_shape(const bsa_shape* s);
+
+/* N = T*H*W, Npad and nb of a shape (-1 for a NULL or invalid shape). */
+BSA_API int64_t bsa_seq_len(const bsa_shape* s);
+BSA_API int64_t bsa_padded_len(const bsa_shape* s);
+BSA_API int64_t bsa_num_blocks(const bsa_shape* s);
+
+/* Bytes of device workspace that bsa_build_block_mask and bsa_attn_fwd need
+ * for this shape: a control block (device error word) followed by the pooled
+ * block means of Q and K (2 * B*heads*nb*d doubles).  0 for an invalid shape. */
+BSA_API size_t bsa_workspace_bytes(const bsa_shape* s);
+
+/* Clears the control block of a freshly allocated workspace (async memset).
+ * Call once after allocation; bsa_check_device_status clears it again. */
+BSA_API bsa_status bsa_workspace_init(void* workspace, size_t ws_bytes, bsa_stream_t stream);
+
+/* Fractal reorder plus layout change, NABLA summary, Metodologia 1
+ * ("Reordenamiento de Tokens"): y[b, h, p, :] = x[b, pi(p), h, :] for p < N and
+ * 0 for N <= p < Npad, where pi lists, frame by frame, the P x P spatial patches
+ * in row-major order and the tokens of each patch in row-major order (edge
+ * patches clipped to H and W).  Bit-exact data movement.
+ *   x_bnhd: device, [B, N, heads, d] bf16, read only.
+ *   y_bhnd: device, [B, heads, Npad, d] bf16, written; must not overlap x. */
+BSA_API bsa_status bsa_reorder(const bsa_shape* s, const void* x_bnhd, void* y_bhnd, bsa_stream_t stream);
+
+/* Inverse of bsa_reorder (the output returns to the model's token order):
+ * x[b, pi(p), h, :] = y[b, h, p, :] for p < N; the padded tail is dropped.
+ *   y_bhnd: device, [B, heads, Npad, d] bf16, read only.
+ *   x_bnhd: device, [B, N, heads, d] bf16, written; must not overlap y. */
+BSA_API bsa_status bsa_inverse_reorder(const bsa_shape* s, const void* y_bhnd, void* x_bnhd, bsa_stream_t stream);
+
+/* Adaptive block mask, NABLA summary, Metodologia 2 (pooling, reduced
+ * attention, CDF thresholding, expansion) and 3 (union with STA).
+ *   q_bhnd, k_bhnd: device, [B, heads, Npad, d] bf16 in kernel order (output of
+ *       bsa_reorder; the padded tail is ignored).
+ *   thr: in [0, 1).  Per row I of softmax(qbar kbar^T / sqrt(d)) over blocks,
+ *       the blocks taken in decreasing probability (ties: lower index first)
+ *       up to and including the first whose cumulative mass reaches 1 - thr
+ *       are kept; thr == 0 keeps every block.  Means, dot products and masses
+ *       are computed in double precision.
+ *   sta_t, sta_h, sta_w: half-widths of the static 3D window in block-tile
+ *       units; block I sits at the tile (t, h / P, w / P) of its first token in
+ *       fractal order.  Any negative value disables the union.
+ *   kv_count: device, [B, heads, nb] int32, written: kept blocks per row.
+ *   kv_idx:   device, [B, heads, nb, nb] int32, written: row (b, h, I) holds its
+ *       kept block indices in ascending order in its first kv_count entries;
+ *       later entries are left untouched.
+ *   mask_or_null: device, [B, heads, nb, nb] uint8 (1 = kept) or NULL.
+ *   workspace / ws_bytes: at least bsa_workspace_bytes(s), initialised once by
+ *       bsa_workspace_init; the pooled means are scratch. */
+BSA_API bsa_status bsa_build_block_mask(const bsa_shape* s, const void* q_bhnd, const void* k_bhnd, float thr,
+                                int32_t sta_t, int32_t sta_h, int32_t sta_w,
+                                int32_t* kv_count, int32_t* kv_idx, uint8_t* mask_or_null,
+                                void* workspace, size_t ws_bytes, bsa_stream_t stream);
+
+/* Block-sparse attention forward, NABLA summary, Metodologia 2 "Expansion":
+ * for every valid query row q of block I,
+ *   O[q] = sum_k softmax_k(scale * Q[q] . K[k]) V[k],
+ * with k over the valid keys (k < N) of the blocks listed for I.  fp32
+ * accumulation and softmax, bf16 output (round to nearest even).  Any valid
+ * lists are accepted (e.g. an externally computed mask).
+ *   q, k, v: device, [B, heads, Npad, d] bf16 in kernel order.
+ *   kv_count, kv_idx: as written by bsa_build_block_mask.  Indices outside
+ *       [0, nb) are skipped and counts outside [1, nb] clamped; both set the
+ *       device error word (BSA_ERR_DEVICE_INDEX).
+ *   scale: softmax scale; 0 selects 1/sqrt(d).
+ *   o: device, [B, heads, Npad, d] bf16, written (padded rows are 0).
+ *   lse_or_null: device, [B, heads, Npad] float32 natural-log sum-exp of the
+ *       scaled scores per row (0 for padded rows), or NULL.
+ *   workspace / ws_bytes: as for bsa_build_block_mask. */
+BSA_API bsa_status bsa_attn_fwd(const bsa_shape* s, const void* q, const void* k, const void* v,
+                        const int32_t* kv_count, const int32_t* kv_idx, float scale,
+                        void* o, float* lse_or_null,
+                        void* workspace, size_t ws_bytes, bsa_stream_t stream);
+
+/* Synchronises `stream`, reads and clears the device error word of
+ * `workspace`: BSA_OK, BSA_ERR_DEVICE_INDEX, BSA_ERR_TIMEOUT or BSA_ERR_CUDA
+ * (a pending asynchronous CUDA error). */
+BSA_API bsa_status bsa_check_device_status(void* workspace, bsa_stream_t stream);
+
+/* Static string naming a status. */
+BSA_API const char* bsa_status_string(bsa_status st);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BSA_H */

@@ -1,0 +1,162 @@
+"""GPU parity: every C-ABI call against the fp64 oracle on the same seeded inputs.
+
+* reorder / inverse reorder: bit-exact;
+* block mask: bit-exact except blocks the oracle flags as ambiguous (prefix
+  mass within 1e-6 of 1 - thr, or a near-tie with the boundary block), which
+  are counted;
+* attention, with the oracle's mask fed to the kernel: max-abs <= 2e-2 and
+  mean-abs <= 2e-3 on the valid rows, LSE within 2e-3.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_attention_fractal_b200 import synth
+
+from _util import LSE_ABS, MAX_ABS, MEAN_ABS, compare_outputs, lists_to_keep, small, to64
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [
+    synth.WORKLOADS["tiny"],
+    small("ragged64", 1, 3, 20, 28, 2, 128, 64, 8, 0.15),
+    small("ragged128_d64", 1, 2, 13, 37, 3, 64, 128, 4, 0.3),
+    small("batch2_d64", 2, 2, 16, 24, 2, 64, 64, 8, 0.25),
+    small("hybrid_small", 1, 4, 24, 24, 2, 128, 64, 8, 0.2, sta=(1, 1, 1)),
+    small("dense_thr0", 1, 2, 12, 20, 2, 128, 128, 4, 0.0),
+    small("one_block", 1, 1, 5, 7, 2, 64, 64, 8, 0.1),
+    small("sharp", 1, 3, 16, 16, 2, 128, 64, 8, 0.05, alpha=3.0),
+]
+
+
+@pytest.fixture(scope="module")
+def bsa():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import block_sparse_attention_fractal_b200 as m
+    return m
+
+
+def _shape(bsa, w):
+    return bsa.make_shape(w.B, w.T, w.H, w.W, w.heads, w.d, w.block, w.patch)
+
+
+def _run_mask(bsa, w, plan, q, k):
+    bsa.reorder(plan.shape, q, plan.q)
+    bsa.reorder(plan.shape, k, plan.k)
+    plan.mask_step(w.thr, w.sta)
+    torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_reorder_bit_exact(bsa, w):
+    q, _, _ = synth.make_qkv(w)
+    s = _shape(bsa, w)
+    Npad = bsa.padded_len(s)
+    qd = q.cuda()
+    y = torch.full((w.B, w.heads, Npad, w.d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    bsa.reorder(s, qd, y)
+    want = oracle.reorder(to64(q), w.T, w.H, w.W, w.patch, w.block)
+    assert np.array_equal(to64(y), want)
+    back = torch.full_like(qd, float("nan"))
+    bsa.inverse_reorder(s, y, back)
+    assert torch.equal(back, qd)
+    assert np.array_equal(to64(back), oracle.inverse_reorder(want, w.T, w.H, w.W, w.patch))
+
+
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_block_mask_matches_oracle(bsa, w):
+    q, k, _ = synth.make_qkv(w)
+    plan = bsa.NablaAttention(_shape(bsa, w), with_mask=True)
+    _run_mask(bsa, w, plan, q.cuda(), k.cuda())
+    assert plan.status() == 0
+    keep_ref, amb = oracle.block_mask(to64(plan.q), to64(plan.k), w.T, w.H, w.W, w.patch, w.block, w.thr, w.sta)
+    keep = lists_to_keep(plan.kv_count, plan.kv_idx, plan.nb)
+    assert np.array_equal(keep, plan.mask.cpu().numpy().astype(bool))
+    mismatch = (keep != keep_ref) & ~amb
+    assert not mismatch.any(), f"{int(mismatch.sum())} unambiguous blocks differ"
+    assert amb.sum() <= max(2, 0.01 * amb.size)
+
+
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_attention_matches_oracle_with_oracle_mask(bsa, w):
+    q, k, v = synth.make_qkv(w)
+    plan = bsa.NablaAttention(_shape(bsa, w), with_lse=True)
+    for src, dst in ((q, plan.q), (k, plan.k), (v, plan.v)):
+        bsa.reorder(plan.shape, src.cuda(), dst)
+    q64, k64, v64 = to64(plan.q), to64(plan.k), to64(plan.v)
+    keep, _ = oracle.block_mask(q64, k64, w.T, w.H, w.W, w.patch, w.block, w.thr, w.sta)
+    cnt, idx = oracle.mask_to_lists(keep)
+    plan.kv_count.copy_(torch.from_numpy(cnt))
+    plan.kv_idx.copy_(torch.from_numpy(idx))
+    plan.attention_step()
+    torch.cuda.synchronize()
+    assert plan.status() == 0
+    O_ref, lse_ref = oracle.masked_attention(q64, k64, v64, keep, w.N, w.block)
+    O = to64(plan.o)
+    mx, mean = compare_outputs(O[:, :, :w.N], O_ref[:, :, :w.N])
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean)
+    assert np.all(O[:, :, w.N:] == 0)
+    lse = to64(plan.lse)
+    assert np.abs(lse[:, :, :w.N] - lse_ref[:, :, :w.N]).max() <= LSE_ABS
+    assert np.all(lse[:, :, w.N:] == 0)
+
+
+@pytest.mark.parametrize("w", [SMALL[0], SMALL[1], SMALL[4]], ids=lambda w: w.name)
+def test_whole_path_matches_oracle(bsa, w):
+    q, k, v = synth.make_qkv(w)
+    plan = bsa.NablaAttention(_shape(bsa, w))
+    out = plan(q.cuda(), k.cuda(), v.cuda(), w.thr, w.sta)
+    torch.cuda.synchronize()
+    assert plan.status() == 0
+    O_ref, keep_ref, amb = oracle.nabla_attention(to64(q), to64(k), to64(v), w.T, w.H, w.W, w.patch, w.block,
+                                                  w.thr, w.sta)
+    assert not amb.any()
+    mx, mean = compare_outputs(to64(out), O_ref)
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean)
+
+
+def test_random_lists_any_density(bsa):
+    """Arbitrary (seeded random) lists, as an external mask would give them."""
+    w = small("random_lists", 1, 2, 16, 40, 3, 128, 64, 8, 0.0, iid=True)
+    q, k, v = synth.make_qkv(w)
+    plan = bsa.NablaAttention(_shape(bsa, w))
+    for src, dst in ((q, plan.q), (k, plan.k), (v, plan.v)):
+        bsa.reorder(plan.shape, src.cuda(), dst)
+    q64, k64, v64 = to64(plan.q), to64(plan.k), to64(plan.v)
+    for dens in (0.05, 0.3, 1.0):
+        cnt, idx = synth.random_block_lists(w.B, w.heads, plan.nb, dens, seed=7)
+        plan.kv_count.copy_(cnt)
+        plan.kv_idx.copy_(idx)
+        plan.attention_step()
+        torch.cuda.synchronize()
+        keep = lists_to_keep(cnt, idx, plan.nb)
+        O_ref, _ = oracle.masked_attention(q64, k64, v64, keep, w.N, w.block)
+        mx, mean = compare_outputs(to64(plan.o)[:, :, :w.N], O_ref[:, :, :w.N])
+        assert mx <= MAX_ABS and mean <= MEAN_ABS, (dens, mx, mean)
+
+
+def test_bad_lists_set_the_device_error_word(bsa):
+    w = small("bad_lists", 1, 1, 16, 16, 2, 64, 64, 8, 0.0)
+    q, k, v = synth.make_qkv(w)
+    plan = bsa.NablaAttention(_shape(bsa, w))
+    for src, dst in ((q, plan.q), (k, plan.k), (v, plan.v)):
+        bsa.reorder(plan.shape, src.cuda(), dst)
+    nb = plan.nb
+    plan.kv_count.fill_(1)
+    plan.kv_idx.zero_()
+    plan.kv_idx[0, 1, 2, 0] = nb + 5            # out of range: skipped, flagged
+    plan.attention_step()
+    assert plan.status() == 4
+    assert plan.status() == 0                    # cleared on read
+    plan.kv_idx[0, 1, 2, 0] = 0
+    plan.kv_count[0, 0, 1] = nb + 1              # count out of range: clamped, flagged
+    plan.attention_step()
+    assert plan.status() == 4
+    plan.kv_count[0, 0, 1] = 0
+    plan.attention_step()
+    assert plan.status() == 4
+    assert torch.all(plan.o[0, 0, w.block:2 * w.block] == 0)   # empty row -> zero output
