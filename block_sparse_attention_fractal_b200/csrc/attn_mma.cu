@@ -71,6 +71,10 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+__device__ __forceinline__ float2 unpack_bf16(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
 // Copies a [64][D] tile starting at global row `row0` of a [rows][D] matrix.
 template <int D>
 __device__ __forceinline__ void load_tile(__nv_bfloat16* s, const __nv_bfloat16* gsrc, size_t row0) {
@@ -214,10 +218,16 @@ __global__ void __launch_bounds__(kThreads) attn_mma_kernel(const __nv_bfloat16*
       const float p1 = ex2(sacc[j][1] - msafe[0]);
       const float p2 = ex2(sacc[j][2] - msafe[1]);
       const float p3 = ex2(sacc[j][3] - msafe[1]);
-      rs[0] += p0 + p1;
-      rs[1] += p2 + p3;
-      pf[j >> 1][(j & 1) * 2 + 0] = pack_bf16(p0, p1);
-      pf[j >> 1][(j & 1) * 2 + 1] = pack_bf16(p2, p3);
+      const uint32_t w01 = pack_bf16(p0, p1);
+      const uint32_t w23 = pack_bf16(p2, p3);
+      pf[j >> 1][(j & 1) * 2 + 0] = w01;
+      pf[j >> 1][(j & 1) * 2 + 1] = w23;
+      // the row sums use the rounded weights the P.V product sees, so O is an
+      // exact convex combination of V rows up to accumulation rounding
+      const float2 r01 = unpack_bf16(w01);
+      const float2 r23 = unpack_bf16(w23);
+      rs[0] += r01.x + r01.y;
+      rs[1] += r23.x + r23.y;
     }
     l[0] = l[0] * alpha[0] + rs[0];
     l[1] = l[1] * alpha[1] + rs[1];

@@ -28,8 +28,18 @@ SMALL = [
     small("hybrid_small", 1, 4, 24, 24, 2, 128, 64, 8, 0.2, sta=(1, 1, 1)),
     small("dense_thr0", 1, 2, 12, 20, 2, 128, 128, 4, 0.0),
     small("one_block", 1, 1, 5, 7, 2, 64, 64, 8, 0.1),
-    small("sharp", 1, 3, 16, 16, 2, 128, 64, 8, 0.05, alpha=3.0),
+    small("sharp", 1, 3, 16, 16, 2, 128, 64, 8, 0.05, alpha=2.0),
 ]
+
+# Larger values than the pages' workloads: |O| reaches 8 and more, where one
+# bf16 ulp (1/16) already exceeds the absolute bound.  Checked against the
+# bound plus half a bf16 ulp of the reference value.
+HOT = small("hot", 1, 3, 16, 16, 2, 128, 64, 8, 0.05, alpha=3.0)
+
+
+def _half_ulp_bf16(x):
+    ax = np.maximum(np.abs(x), 2.0 ** -126)
+    return 0.5 * 2.0 ** (np.floor(np.log2(ax)) - 7)
 
 
 @pytest.fixture(scope="module")
@@ -160,3 +170,22 @@ def test_bad_lists_set_the_device_error_word(bsa):
     plan.attention_step()
     assert plan.status() == 4
     assert torch.all(plan.o[0, 0, w.block:2 * w.block] == 0)   # empty row -> zero output
+
+
+def test_attention_large_values_within_bf16_resolution(bsa):
+    w = HOT
+    q, k, v = synth.make_qkv(w)
+    plan = bsa.NablaAttention(_shape(bsa, w))
+    for src, dst in ((q, plan.q), (k, plan.k), (v, plan.v)):
+        bsa.reorder(plan.shape, src.cuda(), dst)
+    q64, k64, v64 = to64(plan.q), to64(plan.k), to64(plan.v)
+    keep, _ = oracle.block_mask(q64, k64, w.T, w.H, w.W, w.patch, w.block, w.thr, w.sta)
+    cnt, idx = oracle.mask_to_lists(keep)
+    plan.kv_count.copy_(torch.from_numpy(cnt))
+    plan.kv_idx.copy_(torch.from_numpy(idx))
+    plan.attention_step()
+    torch.cuda.synchronize()
+    O_ref, _ = oracle.masked_attention(q64, k64, v64, keep, w.N, w.block)
+    got, want = to64(plan.o)[:, :, :w.N], O_ref[:, :, :w.N]
+    assert np.abs(want).max() > 8.0
+    assert np.all(np.abs(got - want) <= MAX_ABS + _half_ulp_bf16(want))
