@@ -17,12 +17,12 @@ from typing import Optional, Tuple
 
 import torch
 
-from ._lib import (BsaError, Shape, attn_fwd, build_block_mask, check_device_status, inverse_reorder,  # noqa: F401
+from ._lib import (BsaError, Shape, attn_fwd, attn_fwd_baseline, build_block_mask, check_device_status, inverse_reorder,  # noqa: F401
                    lib, make_shape, num_blocks, padded_len, reorder, seq_len, validate_shape, workspace_bytes,
                    workspace_init, LIB_PATH)
 
 __all__ = ["BsaError", "Shape", "make_shape", "NablaAttention", "reorder", "inverse_reorder", "build_block_mask",
-           "attn_fwd", "check_device_status", "workspace_bytes", "workspace_init", "padded_len", "num_blocks",
+           "attn_fwd", "attn_fwd_baseline", "check_device_status", "workspace_bytes", "workspace_init", "padded_len", "num_blocks",
            "seq_len", "validate_shape", "LIB_PATH"]
 
 
@@ -56,8 +56,9 @@ class NablaAttention:
     def mask_step(self, thr: float, sta: Optional[Tuple[int, int, int]] = None) -> None:
         build_block_mask(self.shape, self.q, self.k, thr, sta, self.kv_count, self.kv_idx, self.mask, self.ws)
 
-    def attention_step(self, scale: float = 0.0) -> None:
-        attn_fwd(self.shape, self.q, self.k, self.v, self.kv_count, self.kv_idx, scale, self.o, self.lse, self.ws)
+    def attention_step(self, scale: float = 0.0, baseline: bool = False) -> None:
+        fn = attn_fwd_baseline if baseline else attn_fwd
+        fn(self.shape, self.q, self.k, self.v, self.kv_count, self.kv_idx, scale, self.o, self.lse, self.ws)
 
     def __call__(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, thr: float,
                  sta: Optional[Tuple[int, int, int]] = None, scale: float = 0.0,

@@ -54,6 +54,7 @@ def _load() -> ctypes.CDLL:
         "bsa_build_block_mask": (st, [S, P, P, ctypes.c_float, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                       P, P, P, P, ctypes.c_size_t, P]),
         "bsa_attn_fwd": (st, [S, P, P, P, P, P, ctypes.c_float, P, P, P, ctypes.c_size_t, P]),
+        "bsa_attn_fwd_baseline": (st, [S, P, P, P, P, P, ctypes.c_float, P, P, P, ctypes.c_size_t, P]),
         "bsa_check_device_status": (st, [P, P]),
         "bsa_status_string": (ctypes.c_char_p, [st]),
     }
@@ -139,6 +140,16 @@ def attn_fwd(s: Shape, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, kv_cou
                             float(scale), _ptr(o), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(),
                             _stream(q.device)),
            "bsa_attn_fwd")
+
+
+def attn_fwd_baseline(s: Shape, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, kv_count: torch.Tensor,
+                      kv_idx: torch.Tensor, scale: float, o: torch.Tensor, lse: Optional[torch.Tensor],
+                      ws: torch.Tensor) -> None:
+    """The legacy mma.sync kernel with the same contract (the measured baseline)."""
+    _check(lib.bsa_attn_fwd_baseline(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(kv_count), _ptr(kv_idx),
+                                     float(scale), _ptr(o), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(),
+                                     _stream(q.device)),
+           "bsa_attn_fwd_baseline")
 
 
 def check_device_status(ws: torch.Tensor) -> int:

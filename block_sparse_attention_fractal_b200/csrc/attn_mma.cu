@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(kThreads) attn_mma_kernel(const __nv_bfloat16*
   cp_async_commit();
 
   float m[2] = {-INFINITY, -INFINITY};
-  float l[2] = {0.f, 0.f};
+  float l[2] = {0.f, 0.f}, lx[2] = {0.f, 0.f};
   float oacc[D / 8][4];
 #pragma unroll
   for (int i = 0; i < D / 8; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
@@ -210,7 +210,7 @@ __global__ void __launch_bounds__(kThreads) attn_mma_kernel(const __nv_bfloat16*
       alpha[h] = ex2(m[h] - msafe[h]);
       m[h] = mn;
     }
-    float rs[2] = {0.f, 0.f};
+    float rs[2] = {0.f, 0.f}, rx[2] = {0.f, 0.f};
     uint32_t pf[4][4];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -228,9 +228,13 @@ __global__ void __launch_bounds__(kThreads) attn_mma_kernel(const __nv_bfloat16*
       const float2 r23 = unpack_bf16(w23);
       rs[0] += r01.x + r01.y;
       rs[1] += r23.x + r23.y;
+      rx[0] += p0 + p1;   // exact weights, for the log-sum-exp
+      rx[1] += p2 + p3;
     }
     l[0] = l[0] * alpha[0] + rs[0];
     l[1] = l[1] * alpha[1] + rs[1];
+    lx[0] = lx[0] * alpha[0] + rx[0];
+    lx[1] = lx[1] * alpha[1] + rx[1];
 #pragma unroll
     for (int i = 0; i < D / 8; ++i) {
       oacc[i][0] *= alpha[0];
@@ -261,6 +265,8 @@ __global__ void __launch_bounds__(kThreads) attn_mma_kernel(const __nv_bfloat16*
   for (int h = 0; h < 2; ++h) {
     l[h] += __shfl_xor_sync(0xffffffffu, l[h], 1);
     l[h] += __shfl_xor_sync(0xffffffffu, l[h], 2);
+    lx[h] += __shfl_xor_sync(0xffffffffu, lx[h], 1);
+    lx[h] += __shfl_xor_sync(0xffffffffu, lx[h], 2);
   }
   const float kLn2 = 0.69314718055994531f;
 #pragma unroll
@@ -274,7 +280,7 @@ __global__ void __launch_bounds__(kThreads) attn_mma_kernel(const __nv_bfloat16*
       const int col = i * 8 + 2 * (lane & 3);
       *reinterpret_cast<uint32_t*>(orow + col) = pack_bf16(oacc[i][2 * h] * inv, oacc[i][2 * h + 1] * inv);
     }
-    if (lse != nullptr && (lane & 3) == 0) lse[rowbase + row] = real ? (m[h] + log2f(l[h])) * kLn2 : 0.f;
+    if (lse != nullptr && (lane & 3) == 0) lse[rowbase + row] = real ? (m[h] + log2f(lx[h])) * kLn2 : 0.f;
   }
 }
 

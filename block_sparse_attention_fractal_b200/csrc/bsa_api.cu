@@ -128,9 +128,13 @@ bsa_status bsa_build_block_mask(const bsa_shape* s, const void* q_bhnd, const vo
   return from_cuda(e);
 }
 
-bsa_status bsa_attn_fwd(const bsa_shape* s, const void* q, const void* k, const void* v, const int32_t* kv_count,
-                        const int32_t* kv_idx, float scale, void* o, float* lse_or_null, void* workspace,
-                        size_t ws_bytes, bsa_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+bsa_status attn_common(const bsa_shape* s, const void* q, const void* k, const void* v, const int32_t* kv_count,
+                       const int32_t* kv_idx, float scale, void* o, float* lse_or_null, void* workspace,
+                       size_t ws_bytes, bsa_stream_t stream, bool baseline) {
   Dims g;
   bsa_status st = check_shape(s, &g);
   if (st != BSA_OK) return st;
@@ -145,8 +149,27 @@ bsa_status bsa_attn_fwd(const bsa_shape* s, const void* q, const void* k, const 
   if (!std::isfinite(scale)) return BSA_ERR_INVALID_ARG;
   if (scale == 0.0f) scale = (float)(1.0 / std::sqrt((double)g.d));
   Ctrl* ctrl = (Ctrl*)workspace;
-  return from_cuda(bsa::launch_attn_mma(g, q, k, v, kv_count, kv_idx, scale, o, lse_or_null, ctrl,
-                                        (cudaStream_t)stream));
+  if (baseline)
+    return from_cuda(bsa::launch_attn_mma(g, q, k, v, kv_count, kv_idx, scale, o, lse_or_null, ctrl,
+                                          (cudaStream_t)stream));
+  return from_cuda(bsa::launch_attn_tc(g, q, k, v, kv_count, kv_idx, scale, o, lse_or_null, ctrl,
+                                       (cudaStream_t)stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+bsa_status bsa_attn_fwd(const bsa_shape* s, const void* q, const void* k, const void* v, const int32_t* kv_count,
+                        const int32_t* kv_idx, float scale, void* o, float* lse_or_null, void* workspace,
+                        size_t ws_bytes, bsa_stream_t stream) {
+  return attn_common(s, q, k, v, kv_count, kv_idx, scale, o, lse_or_null, workspace, ws_bytes, stream, false);
+}
+
+bsa_status bsa_attn_fwd_baseline(const bsa_shape* s, const void* q, const void* k, const void* v,
+                                 const int32_t* kv_count, const int32_t* kv_idx, float scale, void* o,
+                                 float* lse_or_null, void* workspace, size_t ws_bytes, bsa_stream_t stream) {
+  return attn_common(s, q, k, v, kv_count, kv_idx, scale, o, lse_or_null, workspace, ws_bytes, stream, true);
 }
 
 bsa_status bsa_check_device_status(void* workspace, bsa_stream_t stream) {

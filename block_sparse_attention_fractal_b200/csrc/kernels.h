@@ -22,4 +22,9 @@ cudaError_t launch_mask(const Dims& g, const double* qbar, const double* kbar, d
 cudaError_t launch_attn_mma(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
                             const int32_t* kv_idx, float scale, void* o, float* lse, Ctrl* ctrl, cudaStream_t st);
 
+// Block-sparse attention on the tcgen05 tensor cores (TMEM accumulators,
+// TMA-staged tiles).
+cudaError_t launch_attn_tc(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
+                           const int32_t* kv_idx, float scale, void* o, float* lse, Ctrl* ctrl, cudaStream_t st);
+
 }  // namespace bsa

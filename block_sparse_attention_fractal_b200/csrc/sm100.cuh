@@ -58,6 +58,28 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
   return false;
 }
 
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;\n" : "=l"(t));
+  return t;
+}
+
+// Waits until the phase with the given parity has completed.  Gives up and
+// returns false after `limit_ns` nanoseconds, or as soon as `abort_word`
+// (a global flag other CTAs set when they give up) has any of `abort_bits`.
+__device__ __forceinline__ bool mbar_wait_ns(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                             const volatile uint32_t* abort_word, uint32_t abort_bits) {
+  if (mbar_test(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_test(bar, parity)) return true;
+    if (global_ns() - t0 > limit_ns) return false;
+    if (*abort_word & abort_bits) return false;
+  }
+}
+
 // ----------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

@@ -149,6 +149,14 @@ BSA_API bsa_status bsa_attn_fwd(const bsa_shape* s, const void* q, const void* k
                         void* o, float* lse_or_null,
                         void* workspace, size_t ws_bytes, bsa_stream_t stream);
 
+/* Same contract as bsa_attn_fwd, computed by the legacy warp-level
+ * mma.sync tensor-core kernel instead of the tcgen05 one.  Kept as the measured
+ * baseline the tcgen05 kernel is compared with. */
+BSA_API bsa_status bsa_attn_fwd_baseline(const bsa_shape* s, const void* q, const void* k, const void* v,
+                                         const int32_t* kv_count, const int32_t* kv_idx, float scale,
+                                         void* o, float* lse_or_null,
+                                         void* workspace, size_t ws_bytes, bsa_stream_t stream);
+
 /* Synchronises `stream`, reads and clears the device error word of
  * `workspace`: BSA_OK, BSA_ERR_DEVICE_INDEX, BSA_ERR_TIMEOUT or BSA_ERR_CUDA
  * (a pending asynchronous CUDA error). */

@@ -91,8 +91,9 @@ def test_block_mask_matches_oracle(bsa, w):
     assert amb.sum() <= max(2, 0.01 * amb.size)
 
 
+@pytest.mark.parametrize("baseline", [False, True], ids=["tcgen05", "mma_sync"])
 @pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
-def test_attention_matches_oracle_with_oracle_mask(bsa, w):
+def test_attention_matches_oracle_with_oracle_mask(bsa, w, baseline):
     q, k, v = synth.make_qkv(w)
     plan = bsa.NablaAttention(_shape(bsa, w), with_lse=True)
     for src, dst in ((q, plan.q), (k, plan.k), (v, plan.v)):
@@ -102,7 +103,7 @@ def test_attention_matches_oracle_with_oracle_mask(bsa, w):
     cnt, idx = oracle.mask_to_lists(keep)
     plan.kv_count.copy_(torch.from_numpy(cnt))
     plan.kv_idx.copy_(torch.from_numpy(idx))
-    plan.attention_step()
+    plan.attention_step(baseline=baseline)
     torch.cuda.synchronize()
     assert plan.status() == 0
     O_ref, lse_ref = oracle.masked_attention(q64, k64, v64, keep, w.N, w.block)
