@@ -38,7 +38,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "block-sparse attn fwd ms & effective TFLOPS (% bf16 peak), Wan-480p shape"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_LAUNCHES_PER_STEP = 7   # reorder x3, pool, mask, attention, inverse reorder
+KERNEL_LAUNCHES_PER_STEP = 8   # reorder x3, pool, mask, plan, attention, inverse reorder
 
 
 # ------------------------------------------------------------------ helpers
@@ -367,7 +367,7 @@ def run_ours(args, w, rank, world, dist):
                      "kernel": "attention", "peak_source": f"{src} bf16 burst",
                      "frac_of_sustained": attn_tf / peak_tf_sus},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": KERNEL_LAUNCHES_PER_STEP * args.steps if not w.iid else 5 * args.steps,
+        "gpu_launches": KERNEL_LAUNCHES_PER_STEP * args.steps if not w.iid else 6 * args.steps,
         "clocks": clk,
     }
     if cpu is not None:

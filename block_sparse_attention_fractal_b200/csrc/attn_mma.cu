@@ -71,9 +71,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-__device__ __forceinline__ float2 unpack_bf16(uint32_t w) {
-  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
-}
 
 // Copies a [64][D] tile starting at global row `row0` of a [rows][D] matrix.
 template <int D>
@@ -222,13 +219,11 @@ __global__ void __launch_bounds__(kThreads) attn_mma_kernel(const __nv_bfloat16*
       const uint32_t w23 = pack_bf16(p2, p3);
       pf[j >> 1][(j & 1) * 2 + 0] = w01;
       pf[j >> 1][(j & 1) * 2 + 1] = w23;
-      // the row sums use the rounded weights the P.V product sees, so O is an
-      // exact convex combination of V rows up to accumulation rounding
-      const float2 r01 = unpack_bf16(w01);
-      const float2 r23 = unpack_bf16(w23);
-      rs[0] += r01.x + r01.y;
-      rs[1] += r23.x + r23.y;
-      rx[0] += p0 + p1;   // exact weights, for the log-sum-exp
+      // O is normalised by the sum of the rounded weights the P.V product
+      // uses; the LSE by the sum of the unrounded ones
+      rs[0] += __uint_as_float(w01 << 16) + __uint_as_float(w01 & 0xFFFF0000u);
+      rs[1] += __uint_as_float(w23 << 16) + __uint_as_float(w23 & 0xFFFF0000u);
+      rx[0] += p0 + p1;
       rx[1] += p2 + p3;
     }
     l[0] = l[0] * alpha[0] + rs[0];

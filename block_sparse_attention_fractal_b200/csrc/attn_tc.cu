@@ -11,7 +11,8 @@
 //                 the keys its query block does not keep (and padding), keeps
 //                 a running base-2 max (rescaling O only when the max grows
 //                 by more than 8) and writes P = 2^(s - m) as bf16 back into
-//                 the S columns of TMEM
+//                 the S columns of TMEM; O is normalised by the sum of the
+//                 rounded weights, the LSE uses the unrounded ones
 //   O += P V      tcgen05.mma with A = P from TMEM and B = V (MN-major) from
 //                 shared memory, O in TMEM
 // Roles: warp 0 issues TMA loads, warp 1 issues MMAs (one elected thread),
@@ -57,10 +58,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-__device__ __forceinline__ float2 unpack_bf16(uint32_t w) {
-  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
-}
-
 __device__ __forceinline__ void timeout(Ctrl* ctrl, uint32_t site) {
   report_error(ctrl, kErrTimeout, blockIdx.x, threadIdx.x, site);
 }
@@ -77,12 +74,13 @@ __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, Ctrl* 
   return __all_sync(0xffffffffu, ok);
 }
 
-template <int D, int BS>
+template <int D, int BS, bool WITH_LSE>
 __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_constant__ CUtensorMap mq,
                                                               const __grid_constant__ CUtensorMap mk,
                                                               const __grid_constant__ CUtensorMap mv,
                                                               const int32_t* __restrict__ kv_count,
-                                                              const int32_t* __restrict__ kv_idx, float scale_log2,
+                                                              const int32_t* __restrict__ kv_idx,
+                                                              const int2* __restrict__ items, float scale_log2,
                                                               __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
                                                               Ctrl* ctrl, Dims g, int items_per_bh) {
   constexpr int QB = 128 / BS;          // query blocks per tile
@@ -106,12 +104,18 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
   const int nb = g.nb;
   const int nw = (nb + 31) >> 5;
 
+  // the tile's query blocks, from the plan (second block -1 when single)
+  const int2 it = items[(size_t)bh * items_per_bh + item];
   int qblk[QB];
   bool qval[QB];
-#pragma unroll
-  for (int h = 0; h < QB; ++h) {
-    qblk[h] = item * QB + h;
-    qval[h] = qblk[h] < nb;
+  qblk[0] = it.x;
+  qval[0] = it.x >= 0 && it.x < nb;
+  if (QB == 2) {
+    qblk[QB - 1] = it.y;
+    qval[QB - 1] = it.y >= 0 && it.y < nb;
+  }
+  if (!qval[0]) {  // a corrupt plan: compute nothing for this tile
+    qblk[0] = 0;
   }
 
   if (tid == 0) {
@@ -198,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           int row0;
-          if (QB == 2) row0 = (qval[h] ? qblk[h] : qblk[0]) * 64;
+          if (QB == 2) row0 = (qval[h & (QB - 1)] ? qblk[h & (QB - 1)] : qblk[0]) * 64;
           else row0 = qblk[0] * 128 + 64 * h;
           tma_load_3d(sQ + ch * kChunk + h * (kChunk / 2), &mq, &c.q_full, ch * 64, row0, bh);
         }
@@ -292,25 +296,21 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
       tmem_ld32(trow + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
       tmem_ld32(trow + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
       tmem_wait_ld();
-      float* x = reinterpret_cast<float*>(sr);
+      const float* x = reinterpret_cast<const float*>(sr);
+      // Row max of the raw scores over the kept, real keys (scale > 0 keeps
+      // the order), then in the base-2 domain.
       float mx = -INFINITY;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         if (lim[h] == 64) {
 #pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            x[h * 64 + i] *= scale_log2;
-            mx = fmaxf(mx, x[h * 64 + i]);
-          }
-        } else {
+          for (int i = 0; i < 64; ++i) mx = fmaxf(mx, x[h * 64 + i]);
+        } else if (lim[h] > 0) {
 #pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            x[h * 64 + i] = (i < lim[h]) ? x[h * 64 + i] * scale_log2 : -INFINITY;
-            mx = fmaxf(mx, x[h * 64 + i]);
-          }
+          for (int i = 0; i < 64; ++i) mx = (i < lim[h]) ? fmaxf(mx, x[h * 64 + i]) : mx;
         }
       }
-      const float mnew = fmaxf(m, mx);
+      const float mnew = fmaxf(m, mx * scale_log2);
       // The running max moves only when it grows by more than 8 (a factor 256
       // in p), or when it is set for the first time.  The O rescale that goes
       // with it uses warp-collective TMEM accesses, so the whole warp takes it
@@ -333,22 +333,44 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
         lx *= alpha;
       }
       if (grow) m = mnew;
-      const float msub = (m == -INFINITY) ? 0.f : m;
-      uint32_t pk[64];
+      const float nm = (m == -INFINITY) ? 0.f : -m;
+      // p = 2^(s * scale_log2 - m): one FFMA and one MUFU op per score.
+      // Halves the row's query block does not keep cost nothing.
       float rs = 0.f, rx = 0.f;
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const float p0 = ex2f(x[2 * i] - msub), p1 = ex2f(x[2 * i + 1] - msub);
-        const uint32_t w = pack_bf16(p0, p1);
-        pk[i] = w;
-        const float2 f = unpack_bf16(w);
-        rs += f.x + f.y;   // the weights the P.V product sees: normalises O
-        rx += p0 + p1;     // the exact weights: the log-sum-exp
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int qq = 0; qq < 2; ++qq) {   // 32 keys -> 16 packed columns at a time
+          uint32_t pk[16];
+          if (lim[h] > 0) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int c = qq * 32 + 2 * i;  // key within the half
+              float p0 = ex2f(fmaf(x[h * 64 + c], scale_log2, nm));
+              float p1 = ex2f(fmaf(x[h * 64 + c + 1], scale_log2, nm));
+              if (lim[h] < 64) {
+                p0 = (c < lim[h]) ? p0 : 0.f;
+                p1 = (c + 1 < lim[h]) ? p1 : 0.f;
+              }
+              const uint32_t w = pack_bf16(p0, p1);
+              pk[i] = w;
+              // O is normalised by the sum of the rounded weights the P.V
+              // product uses (an exact convex combination of V rows); the LSE,
+              // when asked for, by the fp32 sum of the unrounded weights.
+              rs += __uint_as_float(w << 16) + __uint_as_float(w & 0xFFFF0000u);
+              if (WITH_LSE) rx += p0 + p1;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[i] = 0u;
+          }
+          // keys [64h + 32qq, +32) -> bf16 pairs in TMEM columns [32h + 16qq, +16)
+          // (those S columns are already in registers)
+          tmem_st16(trow + 32 * h + 16 * qq, pk);
+        }
       }
       l += rs;
-      lx += rx;
-      tmem_st32(trow + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(trow + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      if (WITH_LSE) lx += rx;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&c.p_full);
@@ -361,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
     }
     int grow;
     if (QB == 2) grow = qval[half] ? qblk[half] * 64 + (r & 63) : -1;
-    else grow = qblk[0] * 128 + r;
+    else grow = qval[0] ? qblk[0] * 128 + r : -1;
     if (grow >= 0 && grow < g.Npad) {
       const bool real = ok && n_tiles > 0 && grow < g.N && l > 0.f;
       const float inv = real ? 1.f / l : 0.f;
@@ -380,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
 #pragma unroll
         for (int i = 0; i < 4; ++i) orow[cc / 8 + i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
       }
-      if (lse != nullptr)
+      if (WITH_LSE)
         lse[(size_t)bh * g.Npad + grow] = real ? (m + __log2f(lx)) * 0.69314718055994531f : 0.f;
     }
   }
@@ -394,32 +416,47 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
   }
 }
 
-template <int D, int BS>
+template <int D, int BS, bool WITH_LSE>
 cudaError_t launch_tc(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
-                      const int32_t* kv_idx, float scale, void* o, float* lse, Ctrl* ctrl, cudaStream_t st) {
+                      const int32_t* kv_idx, const int2* items, float scale, void* o, float* lse, Ctrl* ctrl,
+                      cudaStream_t st) {
   CUtensorMap mq, mk, mv;
   const uint64_t rows = (uint64_t)g.Npad, bhs = (uint64_t)g.B * g.heads;
   if (!make_map_bf16_3d(&mq, q, D, rows, bhs, 64, 64) || !make_map_bf16_3d(&mk, k, D, rows, bhs, 64, 64) ||
       !make_map_bf16_3d(&mv, v, D, rows, bhs, 64, 64))
     return cudaErrorInvalidValue;
-  const int items = (BS == 64) ? (g.nb + 1) / 2 : g.nb;
+  const int n_items = (BS == 64) ? (g.nb + 1) / 2 : g.nb;
   const size_t smem = 3u * 128u * D * 2u + sizeof(Ctl) + 1024u;
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D, BS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e =
+      cudaFuncSetAttribute(attn_tc_kernel<D, BS, WITH_LSE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const dim3 grid((unsigned)(bhs * items));
-  attn_tc_kernel<D, BS><<<grid, kThreads, smem, st>>>(mq, mk, mv, kv_count, kv_idx, scale * 1.4426950408889634f,
-                                                      (__nv_bfloat16*)o, lse, ctrl, g, items);
+  const dim3 grid((unsigned)(bhs * n_items));
+  attn_tc_kernel<D, BS, WITH_LSE><<<grid, kThreads, smem, st>>>(mq, mk, mv, kv_count, kv_idx, items,
+                                                      scale * 1.4426950408889634f, (__nv_bfloat16*)o, lse, ctrl, g,
+                                                      n_items);
   return cudaGetLastError();
+}
+
+template <int D, int BS>
+cudaError_t launch_tc_lse(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
+                          const int32_t* kv_idx, const int2* items, float scale, void* o, float* lse, Ctrl* ctrl,
+                          cudaStream_t st) {
+  if (lse != nullptr) return launch_tc<D, BS, true>(g, q, k, v, kv_count, kv_idx, items, scale, o, lse, ctrl, st);
+  return launch_tc<D, BS, false>(g, q, k, v, kv_count, kv_idx, items, scale, o, lse, ctrl, st);
 }
 
 }  // namespace
 
 cudaError_t launch_attn_tc(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
-                           const int32_t* kv_idx, float scale, void* o, float* lse, Ctrl* ctrl, cudaStream_t st) {
-  if (g.d == 128 && g.bs == 64) return launch_tc<128, 64>(g, q, k, v, kv_count, kv_idx, scale, o, lse, ctrl, st);
-  if (g.d == 128 && g.bs == 128) return launch_tc<128, 128>(g, q, k, v, kv_count, kv_idx, scale, o, lse, ctrl, st);
-  if (g.d == 64 && g.bs == 64) return launch_tc<64, 64>(g, q, k, v, kv_count, kv_idx, scale, o, lse, ctrl, st);
-  return launch_tc<64, 128>(g, q, k, v, kv_count, kv_idx, scale, o, lse, ctrl, st);
+                           const int32_t* kv_idx, const int2* items, float scale, void* o, float* lse, Ctrl* ctrl,
+                           cudaStream_t st) {
+  if (g.d == 128 && g.bs == 64)
+    return launch_tc_lse<128, 64>(g, q, k, v, kv_count, kv_idx, items, scale, o, lse, ctrl, st);
+  if (g.d == 128 && g.bs == 128)
+    return launch_tc_lse<128, 128>(g, q, k, v, kv_count, kv_idx, items, scale, o, lse, ctrl, st);
+  if (g.d == 64 && g.bs == 64)
+    return launch_tc_lse<64, 64>(g, q, k, v, kv_count, kv_idx, items, scale, o, lse, ctrl, st);
+  return launch_tc_lse<64, 128>(g, q, k, v, kv_count, kv_idx, items, scale, o, lse, ctrl, st);
 }
 
 }  // namespace bsa

@@ -44,7 +44,12 @@ bsa_status check_shape(const bsa_shape* s, Dims* out) {
 
 size_t pooled_bytes(const Dims& g) { return (size_t)g.B * g.heads * g.nb * g.d * sizeof(double); }
 
-size_t workspace_bytes(const Dims& g) { return sizeof(Ctrl) + 2 * pooled_bytes(g); }
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Workspace: control block | qbar | kbar | attention plan items.
+size_t plan_offset(const Dims& g) { return sizeof(Ctrl) + align256(2 * pooled_bytes(g)); }
+
+size_t workspace_bytes(const Dims& g) { return plan_offset(g) + align256(bsa::plan_items_bytes(g)); }
 
 bsa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_CUDA; }
 
@@ -146,13 +151,16 @@ bsa_status attn_common(const bsa_shape* s, const void* q, const void* k, const v
       !aligned16(kv_idx) || !aligned16(workspace) || (lse_or_null != nullptr && !aligned16(lse_or_null)))
     return BSA_ERR_INVALID_ARG;
   if (ws_bytes < workspace_bytes(g)) return BSA_ERR_INVALID_ARG;
-  if (!std::isfinite(scale)) return BSA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || scale < 0.0f) return BSA_ERR_INVALID_ARG;
   if (scale == 0.0f) scale = (float)(1.0 / std::sqrt((double)g.d));
   Ctrl* ctrl = (Ctrl*)workspace;
   if (baseline)
     return from_cuda(bsa::launch_attn_mma(g, q, k, v, kv_count, kv_idx, scale, o, lse_or_null, ctrl,
                                           (cudaStream_t)stream));
-  return from_cuda(bsa::launch_attn_tc(g, q, k, v, kv_count, kv_idx, scale, o, lse_or_null, ctrl,
+  int2* items = (int2*)((char*)workspace + plan_offset(g));
+  cudaError_t e = bsa::launch_plan(g, kv_count, kv_idx, items, (cudaStream_t)stream);
+  if (e != cudaSuccess) return BSA_ERR_CUDA;
+  return from_cuda(bsa::launch_attn_tc(g, q, k, v, kv_count, kv_idx, items, scale, o, lse_or_null, ctrl,
                                        (cudaStream_t)stream));
 }
 

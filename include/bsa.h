@@ -82,8 +82,9 @@ BSA_API int64_t bsa_padded_len(const bsa_shape* s);
 BSA_API int64_t bsa_num_blocks(const bsa_shape* s);
 
 /* Bytes of device workspace that bsa_build_block_mask and bsa_attn_fwd need
- * for this shape: a control block (device error word) followed by the pooled
- * block means of Q and K (2 * B*heads*nb*d doubles).  0 for an invalid shape. */
+ * for this shape: a control block (device error word), the pooled block means
+ * of Q and K (2 * B*heads*nb*d doubles) and the attention work plan (one int2
+ * per 128-row query tile).  0 for an invalid shape. */
 BSA_API size_t bsa_workspace_bytes(const bsa_shape* s);
 
 /* Clears the control block of a freshly allocated workspace (async memset).
@@ -139,7 +140,7 @@ BSA_API bsa_status bsa_build_block_mask(const bsa_shape* s, const void* q_bhnd, 
  *   kv_count, kv_idx: as written by bsa_build_block_mask.  Indices outside
  *       [0, nb) are skipped and counts outside [1, nb] clamped; both set the
  *       device error word (BSA_ERR_DEVICE_INDEX).
- *   scale: softmax scale; 0 selects 1/sqrt(d).
+ *   scale: softmax scale, >= 0; 0 selects 1/sqrt(d).
  *   o: device, [B, heads, Npad, d] bf16, written (padded rows are 0).
  *   lse_or_null: device, [B, heads, Npad] float32 natural-log sum-exp of the
  *       scaled scores per row (0 for padded rows), or NULL.
