@@ -16,3 +16,14 @@ def pytest_configure(config):
 @pytest.fixture(scope="session")
 def golden_dir():
     return os.path.join(ROOT, "tests", "golden")
+
+
+def pytest_sessionstart(session):
+    """Builds libbsa.so (sm_100a, in-tree) when it is missing or stale, so
+    test modules that import the package find it."""
+    import importlib.util
+    path = os.path.join(ROOT, "block_sparse_attention_fractal_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("_bsa_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
