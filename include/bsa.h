@@ -158,6 +158,48 @@ BSA_API bsa_status bsa_attn_fwd_baseline(const bsa_shape* s, const void* q, cons
                                          void* o, float* lse_or_null,
                                          void* workspace, size_t ws_bytes, bsa_stream_t stream);
 
+/* Size in bytes of the device array that bsa_attn_fwd_noalloc uses as its
+ * scratch (4 MiB, reserved on every GPU that loads the library). */
+#define BSA_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/* bsa_attn_fwd for callers that cannot allocate device memory.  The NABLA
+ * summary has no counterpart: this is a library convenience.
+ *
+ * Some callers cannot call cudaMalloc or any other allocator where they run
+ * attention: code given a fixed memory budget up front, a plug-in inside a host
+ * program that owns every allocation, or a path that must not take the
+ * allocator's locks.  This entry point needs no workspace.  Its scratch (the
+ * device error word and the work plan of the tensor-core kernel) lives in one
+ * static device array of BSA_NOALLOC_SCRATCH_BYTES that the library holds on
+ * every GPU until the process exits.  The entry point calls no cudaMalloc,
+ * cudaFree or other allocating routine.
+ *
+ * Arguments, layouts and results are those of bsa_attn_fwd.  There is no
+ * workspace argument.  Instead:
+ *   error_word_or_null: device, one uint32 (4-byte aligned), written at the end
+ *       of the call with the device error bits of this call (0 = none,
+ *       1 = a KV index outside [0, nb), 2 = a KV count outside [1, nb],
+ *       4 = a bounded wait expired), or NULL to ignore them.
+ *
+ * Limits and errors: a shape whose scratch (256 bytes plus 8 bytes per
+ * 128-row query tile, i.e. per B*heads*ceil(nb / (128 / block)) tiles, rounded
+ * up to 256) exceeds BSA_NOALLOC_SCRATCH_BYTES is refused with
+ * BSA_ERR_UNSUPPORTED before anything is launched.  Argument errors are those
+ * of bsa_attn_fwd.
+ *
+ * Set-up: the first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current).  Make that first call
+ * before any stream capture.
+ *
+ * Sharing: every call on a device uses the same array.  The call clears the
+ * error word at its start and rewrites the plan, so nothing carries over from
+ * one call to the next.  Calls whose GPU work overlaps (other streams, other
+ * host threads) race on the array: serialise them. */
+BSA_API bsa_status bsa_attn_fwd_noalloc(const bsa_shape* s, const void* q, const void* k, const void* v,
+                                        const int32_t* kv_count, const int32_t* kv_idx, float scale,
+                                        void* o, float* lse_or_null, uint32_t* error_word_or_null,
+                                        bsa_stream_t stream);
+
 /* Synchronises `stream`, reads and clears the device error word of
  * `workspace`: BSA_OK, BSA_ERR_DEVICE_INDEX, BSA_ERR_TIMEOUT or BSA_ERR_CUDA
  * (a pending asynchronous CUDA error). */
