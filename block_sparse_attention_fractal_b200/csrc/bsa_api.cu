@@ -46,10 +46,10 @@ size_t pooled_bytes(const Dims& g) { return (size_t)g.B * g.heads * g.nb * g.d *
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// Workspace: control block | qbar | kbar | attention plan items.
+// Workspace: control block | qbar | kbar | attention plan region.
 size_t plan_offset(const Dims& g) { return sizeof(Ctrl) + align256(2 * pooled_bytes(g)); }
 
-size_t workspace_bytes(const Dims& g) { return plan_offset(g) + align256(bsa::plan_items_bytes(g)); }
+size_t workspace_bytes(const Dims& g) { return plan_offset(g) + align256(bsa::plan_region_bytes(g)); }
 
 bsa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_CUDA; }
 

@@ -23,9 +23,10 @@ cudaError_t launch_attn_mma(const Dims& g, const void* q, const void* k, const v
                             const int32_t* kv_idx, float scale, void* o, float* lse, Ctrl* ctrl, cudaStream_t st);
 
 // Work plan of the tcgen05 attention kernel: one int2 (first block, second
-// block or -1) per 128-row tile of every (batch, head), in launch order.
-size_t plan_items_bytes(const Dims& g);
-size_t plan_smem_bytes(const Dims& g);
+// block or -1) per 128-row tile of every (batch, head), in launch order, at
+// the start of a plan region of plan_region_bytes(g) bytes (the rest is the
+// matching scratch of 64-token blocks).
+size_t plan_region_bytes(const Dims& g);
 cudaError_t launch_plan(const Dims& g, const int32_t* kv_count, const int32_t* kv_idx, int2* items, cudaStream_t st);
 
 // Block-sparse attention on the tcgen05 tensor cores (TMEM accumulators,

@@ -86,7 +86,7 @@ bsa_status bsa_attn_fwd_noalloc(const bsa_shape* s, const void* q, const void* k
   if (scale == 0.0f) scale = (float)(1.0 / std::sqrt((double)g.d));
   // Scratch this shape needs: control block + work plan.  Larger shapes are
   // refused before anything is launched.
-  const size_t need = sizeof(Ctrl) + align256(bsa::plan_items_bytes(g));
+  const size_t need = sizeof(Ctrl) + align256(bsa::plan_region_bytes(g));
   if (need > (size_t)BSA_NOALLOC_SCRATCH_BYTES) return BSA_ERR_UNSUPPORTED;
 
   void* scratch = nullptr;

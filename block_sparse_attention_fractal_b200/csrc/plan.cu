@@ -14,6 +14,15 @@
 // Tiles of each (batch, head) are then ordered by decreasing union size, so the
 // longest tiles start first and short ones fill the tail of the grid.
 // Pairing and order change only the schedule, never the result.
+//
+// Two kernels (64-token blocks):
+//   overlap_kernel  many CTAs: each builds the kept-block bitmaps of 64 rows
+//                   from the lists (coalesced reads) and writes, for its 32
+//                   rows, the overlap with each of the next kWindow rows and
+//                   the row's own distinct-block count;
+//   match_kernel    one CTA per (batch, head): matching rounds over those
+//                   weights, then the ordered tile list.
+// With 128-token blocks only match_kernel runs, keyed by the list counts.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -21,95 +30,151 @@ namespace bsa {
 
 namespace {
 
-constexpr int kPlanThreads = 1024;
-constexpr int kWindow = 32;
+constexpr int kWindow = 32;          // partner candidates: rows r - kWindow .. r + kWindow
 constexpr int kRounds = 6;
+constexpr int kOverlapRows = 32;     // rows whose weights one overlap CTA writes
+constexpr int kOverlapThreads = kOverlapRows * kWindow;  // 1024
+constexpr int kMatchThreads = 1024;
 
-__device__ __forceinline__ int overlap(const uint32_t* a, const uint32_t* b, int nw) {
-  int s = 0;
-  for (int w = 0; w < nw; ++w) s += __popc(a[w] & b[w]);
-  return s;
-}
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-struct PlanLayout {
-  int nw, stride, n_items, pow2;
-  size_t off_partner, off_choice, off_key;  // in 32-bit words
-  size_t bytes;
+// Plan region of the workspace: items | weights | counts (the last two only
+// with 64-token blocks).
+struct PlanRegion {
+  size_t items, weights, counts, total;
 };
 
-__host__ __device__ inline PlanLayout plan_layout(int nb, int qb) {
-  PlanLayout L;
-  L.nw = (nb + 31) >> 5;
-  L.stride = L.nw + 1;  // padded rows: conflict-free access by row
-  L.n_items = (nb + qb - 1) / qb;
-  L.pow2 = 1;
-  while (L.pow2 < L.n_items) L.pow2 <<= 1;
-  L.off_partner = (size_t)nb * L.stride;
-  L.off_choice = L.off_partner + nb;
-  L.off_key = (L.off_choice + nb + 1) & ~(size_t)1;  // 8-byte aligned
-  L.bytes = L.off_key * 4 + (size_t)L.pow2 * 8;
-  return L;
+PlanRegion plan_region(const Dims& g) {
+  const size_t bh = (size_t)g.B * g.heads;
+  const int qb = 128 / g.bs;
+  PlanRegion R;
+  R.items = 0;
+  const size_t items_bytes = bh * ((g.nb + qb - 1) / qb) * sizeof(int2);
+  R.weights = align256(items_bytes);
+  const size_t w_bytes = (qb == 2) ? bh * g.nb * kWindow * sizeof(uint16_t) : 0;
+  R.counts = R.weights + align256(w_bytes);
+  const size_t c_bytes = (qb == 2) ? bh * g.nb * sizeof(int32_t) : 0;
+  R.total = R.counts + align256(c_bytes);
+  return R;
 }
 
-// grid: B*heads CTAs.  Shared memory (PlanLayout): kept bitmaps [nb][nw + 1]
-// words, partner [nb], choice [nb], item keys [pow2] (64-bit).
-template <int QB>
-__global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __restrict__ kv_count,
-                                                            const int32_t* __restrict__ kv_idx, Dims g,
-                                                            int2* __restrict__ items) {
-  extern __shared__ __align__(16) uint32_t psm[];
-  __shared__ int n_keys;
+// grid (ceil(nb / 32), B*heads), 1024 threads.  Shared memory: bitmaps of
+// rows [r0, r0 + 64) with a padded stride (conflict-free by row).
+__global__ void __launch_bounds__(kOverlapThreads) overlap_kernel(const int32_t* __restrict__ kv_count,
+                                                                  const int32_t* __restrict__ kv_idx, Dims g,
+                                                                  uint16_t* __restrict__ weights,
+                                                                  int32_t* __restrict__ counts) {
+  constexpr int kRowsHeld = kOverlapRows + kWindow;
+  constexpr int kStride = BSA_MAX_BLOCKS / 32 + 1;
+  __shared__ uint32_t bm[kRowsHeld * kStride];
   const int nb = g.nb;
-  const PlanLayout L = plan_layout(nb, QB);
-  const int nw = L.nw, stride = L.stride;
-  uint32_t* bm = psm;
-  int* partner = reinterpret_cast<int*>(psm + L.off_partner);
-  int* choice = reinterpret_cast<int*>(psm + L.off_choice);
-  unsigned long long* key = reinterpret_cast<unsigned long long*>(psm + L.off_key);
-  const size_t bh = blockIdx.x;
+  const int nw = (nb + 31) >> 5;
+  const size_t bh = blockIdx.y;
+  const int r0 = blockIdx.x * kOverlapRows;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  for (int i = threadIdx.x; i < nb * stride; i += blockDim.x) bm[i] = 0u;
-  if (threadIdx.x == 0) n_keys = 0;
+  for (int i = threadIdx.x; i < kRowsHeld * kStride; i += kOverlapThreads) bm[i] = 0u;
   __syncthreads();
-  for (int r = threadIdx.x; r < nb; r += blockDim.x) {
+  for (int lr = warp; lr < kRowsHeld; lr += kOverlapThreads / 32) {
+    const int r = r0 + lr;
+    if (r >= nb) break;
     const size_t row = bh * nb + r;
     int cnt = kv_count[row];
     cnt = cnt < 0 ? 0 : (cnt > nb ? nb : cnt);
     const int32_t* list = kv_idx + row * nb;
-    for (int i = 0; i < cnt; ++i) {
-      const int J = list[i];
-      if (J >= 0 && J < nb) bm[r * stride + (J >> 5)] |= 1u << (J & 31);
+    for (int e = lane; e < cnt; e += 32) {
+      const int J = list[e];
+      if (J >= 0 && J < nb) atomicOr(&bm[lr * kStride + (J >> 5)], 1u << (J & 31));
     }
+  }
+  __syncthreads();
+
+  const int lr = threadIdx.x / kWindow;
+  const int off = threadIdx.x % kWindow + 1;
+  const int r = r0 + lr;
+  if (r >= nb) return;
+  int w = 0;
+  if (r + off < nb) {
+    const uint32_t* a = bm + lr * kStride;
+    const uint32_t* b = bm + (lr + off) * kStride;
+    for (int i = 0; i < nw; ++i) w += __popc(a[i] & b[i]);
+  }
+  weights[(bh * nb + r) * kWindow + (off - 1)] = (uint16_t)w;
+  if (off == 1) {
+    int c = 0;
+    for (int i = 0; i < nw; ++i) c += __popc(bm[lr * kStride + i]);
+    counts[bh * nb + r] = c;
+  }
+}
+
+// grid B*heads, 1024 threads.  QB = 2: pairs rows by the weights; QB = 1:
+// every row is its own tile.  Both then sort the tiles by decreasing size.
+template <int QB>
+__global__ void __launch_bounds__(kMatchThreads) match_kernel(const int32_t* __restrict__ kv_count,
+                                                              const uint16_t* __restrict__ weights,
+                                                              const int32_t* __restrict__ counts, Dims g,
+                                                              int2* __restrict__ items) {
+  __shared__ int partner[BSA_MAX_BLOCKS];
+  __shared__ int choice[BSA_MAX_BLOCKS];
+  __shared__ int cnt_s[BSA_MAX_BLOCKS];
+  __shared__ unsigned long long key[BSA_MAX_BLOCKS];
+  __shared__ int n_keys;
+  extern __shared__ uint16_t wts[];   // [nb][kWindow] (QB == 2 only)
+  const int nb = g.nb;
+  const size_t bh = blockIdx.x;
+  const int n_items = (nb + QB - 1) / QB;
+  int pow2 = 1;
+  while (pow2 < n_items) pow2 <<= 1;
+
+  if (threadIdx.x == 0) n_keys = 0;
+  for (int r = threadIdx.x; r < nb; r += kMatchThreads) {
+    int c;
+    if (QB == 2) {
+      c = counts[bh * nb + r];
+    } else {
+      c = kv_count[bh * nb + r];
+      c = c < 0 ? 0 : (c > nb ? nb : c);
+    }
+    cnt_s[r] = c;
     partner[r] = (QB == 2) ? -1 : r;
+  }
+  if (QB == 2) {
+    const uint4* src = reinterpret_cast<const uint4*>(weights + bh * nb * kWindow);
+    uint4* dst = reinterpret_cast<uint4*>(wts);
+    for (int i = threadIdx.x; i < nb * kWindow * 2 / 16; i += kMatchThreads) dst[i] = src[i];
   }
   __syncthreads();
 
   if (QB == 2) {
     for (int round = 0; round < kRounds; ++round) {
-      for (int r = threadIdx.x; r < nb; r += blockDim.x) {
+      for (int r = threadIdx.x; r < nb; r += kMatchThreads) {
         int best = -1, bestw = -1;
         if (partner[r] < 0) {
           for (int off = 1; off <= kWindow; ++off) {
-#pragma unroll
-            for (int sgn = 0; sgn < 2; ++sgn) {
-              const int J = sgn ? r + off : r - off;
-              if (J < 0 || J >= nb || partner[J] >= 0) continue;
-              const int w = overlap(bm + r * stride, bm + J * stride, nw);
-              if (w > bestw) {  // ties keep the nearer, then the lower, index
-                bestw = w;
-                best = J;
-              }
+            const int lo = r - off, hi = r + off;
+            // ties keep the nearer, then the lower, index
+            if (lo >= 0 && partner[lo] < 0) {
+              const int w = wts[lo * kWindow + off - 1];
+              if (w > bestw) { bestw = w; best = lo; }
+            }
+            if (hi < nb && partner[hi] < 0) {
+              const int w = wts[r * kWindow + off - 1];
+              if (w > bestw) { bestw = w; best = hi; }
             }
           }
         }
         choice[r] = best;
       }
       __syncthreads();
-      for (int r = threadIdx.x; r < nb; r += blockDim.x) {
+      int formed = 0;
+      for (int r = threadIdx.x; r < nb; r += kMatchThreads) {
         const int J = choice[r];
-        if (partner[r] < 0 && J >= 0 && choice[J] == r) partner[r] = J;  // mutual: both sides set it
+        if (partner[r] < 0 && J >= 0 && choice[J] == r) {  // mutual: both sides set it
+          partner[r] = J;
+          formed = 1;
+        }
       }
-      __syncthreads();
+      if (!__syncthreads_or(formed)) break;
     }
     if (threadIdx.x == 0) {  // the rest, in index order
       int pending = -1;
@@ -128,24 +193,28 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
     __syncthreads();
   }
 
-  // One key per tile (the lower block of each pair): descending union size,
-  // then ascending block index.
-  for (int r = threadIdx.x; r < nb; r += blockDim.x) {
+  // One key per tile (the lower block of each pair): descending union size
+  // (for pairs beyond the window, the sum of both counts), then ascending block.
+  for (int r = threadIdx.x; r < nb; r += kMatchThreads) {
     const int p = partner[r];
     if (p < r) continue;
-    int u = 0;
-    for (int w = 0; w < nw; ++w) u += __popc(bm[r * stride + w] | bm[p * stride + w]);
+    int u = cnt_s[r];
+    if (QB == 2 && p != r) {
+      u += cnt_s[p];
+      if (p - r <= kWindow) u -= wts[r * kWindow + (p - r) - 1];
+    }
+    u = min(u, 0xFFFF);
     const int slot = atomicAdd(&n_keys, 1);
     key[slot] = ((unsigned long long)(0xFFFFu - (unsigned)u) << 32) | ((unsigned long long)r << 16) |
                 (unsigned long long)(p & 0xFFFF);
   }
   __syncthreads();
-  for (int i = n_keys + threadIdx.x; i < L.pow2; i += blockDim.x) key[i] = ~0ull;
+  for (int i = n_keys + threadIdx.x; i < pow2; i += kMatchThreads) key[i] = ~0ull;
   __syncthreads();
   // bitonic sort of the keys, ascending
-  for (int k = 2; k <= L.pow2; k <<= 1) {
+  for (int k = 2; k <= pow2; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = threadIdx.x; i < L.pow2; i += blockDim.x) {
+      for (int i = threadIdx.x; i < pow2; i += kMatchThreads) {
         const int ixj = i ^ j;
         if (ixj > i) {
           const unsigned long long a = key[i], b = key[ixj];
@@ -159,35 +228,36 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
       __syncthreads();
     }
   }
-  for (int i = threadIdx.x; i < L.n_items; i += blockDim.x) {
+  for (int i = threadIdx.x; i < n_items; i += kMatchThreads) {
     const unsigned long long kk = key[i];
     const int r = (int)((kk >> 16) & 0xFFFFu);
     const int p = (int)(kk & 0xFFFFu);
-    items[bh * L.n_items + i] = make_int2(r, (QB == 2 && p != r) ? p : -1);
+    items[bh * n_items + i] = make_int2(r, (QB == 2 && p != r) ? p : -1);
   }
 }
 
 }  // namespace
 
-size_t plan_smem_bytes(const Dims& g) { return plan_layout(g.nb, 128 / g.bs).bytes; }
-
-size_t plan_items_bytes(const Dims& g) {
-  const int qb = 128 / g.bs;
-  return (size_t)g.B * g.heads * ((g.nb + qb - 1) / qb) * sizeof(int2);
-}
+size_t plan_region_bytes(const Dims& g) { return plan_region(g).total; }
 
 cudaError_t launch_plan(const Dims& g, const int32_t* kv_count, const int32_t* kv_idx, int2* items,
                         cudaStream_t st) {
-  const size_t smem = plan_smem_bytes(g);
+  const PlanRegion R = plan_region(g);
+  const int bh = g.B * g.heads;
   cudaError_t e;
   if (g.bs == 64) {
-    e = cudaFuncSetAttribute(plan_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    uint16_t* weights = (uint16_t*)((char*)items + R.weights);
+    int32_t* counts = (int32_t*)((char*)items + R.counts);
+    const dim3 grid((g.nb + kOverlapRows - 1) / kOverlapRows, bh);
+    overlap_kernel<<<grid, kOverlapThreads, 0, st>>>(kv_count, kv_idx, g, weights, counts);
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    plan_kernel<2><<<g.B * g.heads, kPlanThreads, smem, st>>>(kv_count, kv_idx, g, items);
+    const size_t smem = (size_t)g.nb * kWindow * sizeof(uint16_t);
+    e = cudaFuncSetAttribute(match_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    match_kernel<2><<<bh, kMatchThreads, smem, st>>>(kv_count, weights, counts, g, items);
   } else {
-    e = cudaFuncSetAttribute(plan_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    plan_kernel<1><<<g.B * g.heads, kPlanThreads, smem, st>>>(kv_count, kv_idx, g, items);
+    match_kernel<1><<<bh, kMatchThreads, 0, st>>>(kv_count, nullptr, nullptr, g, items);
   }
   return cudaGetLastError();
 }

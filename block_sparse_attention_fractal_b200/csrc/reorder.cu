@@ -20,10 +20,12 @@ __global__ void __launch_bounds__(kThreads) reorder_kernel(const uint4* __restri
                                                            Dims g) {
   const int vec = g.d / 8;                    // 16-byte vectors per row
   const int rows_per_pass = kThreads / vec;
-  const int head = blockIdx.y;
-  const int b = blockIdx.z;
+  // heads fastest: CTAs that run together move the same positions of every
+  // head, i.e. adjacent rows of the same model-order tokens
+  const int head = blockIdx.x % g.heads;
+  const int b = blockIdx.y;
   const int c = threadIdx.x % vec;
-  const int p0 = blockIdx.x * kRows;
+  const int p0 = (blockIdx.x / g.heads) * kRows;
   const size_t bh = (size_t)b * g.heads + head;
 #pragma unroll 4
   for (int r = threadIdx.x / vec; r < kRows; r += rows_per_pass) {
@@ -47,13 +49,13 @@ __global__ void __launch_bounds__(kThreads) reorder_kernel(const uint4* __restri
 }  // namespace
 
 cudaError_t launch_reorder(const Dims& g, const void* x_bnhd, void* y_bhnd, cudaStream_t st) {
-  dim3 grid((g.Npad + kRows - 1) / kRows, g.heads, g.B);
+  dim3 grid((unsigned)(g.heads * ((g.Npad + kRows - 1) / kRows)), g.B);
   reorder_kernel<false><<<grid, kThreads, 0, st>>>((const uint4*)x_bnhd, (uint4*)y_bhnd, g);
   return cudaGetLastError();
 }
 
 cudaError_t launch_inverse_reorder(const Dims& g, const void* y_bhnd, void* x_bnhd, cudaStream_t st) {
-  dim3 grid((g.Npad + kRows - 1) / kRows, g.heads, g.B);
+  dim3 grid((unsigned)(g.heads * ((g.Npad + kRows - 1) / kRows)), g.B);
   reorder_kernel<true><<<grid, kThreads, 0, st>>>((const uint4*)y_bhnd, (uint4*)x_bnhd, g);
   return cudaGetLastError();
 }

@@ -84,7 +84,8 @@ BSA_API int64_t bsa_num_blocks(const bsa_shape* s);
 /* Bytes of device workspace that bsa_build_block_mask and bsa_attn_fwd need
  * for this shape: a control block (device error word), the pooled block means
  * of Q and K (2 * B*heads*nb*d doubles) and the attention work plan (one int2
- * per 128-row query tile).  0 for an invalid shape. */
+ * per 128-row query tile; with 64-token blocks also 64 bytes of pairing
+ * weights and 4 bytes of counts per block row).  0 for an invalid shape. */
 BSA_API size_t bsa_workspace_bytes(const bsa_shape* s);
 
 /* Clears the control block of a freshly allocated workspace (async memset).
@@ -181,11 +182,13 @@ BSA_API bsa_status bsa_attn_fwd_baseline(const bsa_shape* s, const void* q, cons
  *       1 = a KV index outside [0, nb), 2 = a KV count outside [1, nb],
  *       4 = a bounded wait expired), or NULL to ignore them.
  *
- * Limits and errors: a shape whose scratch (256 bytes plus 8 bytes per
- * 128-row query tile, i.e. per B*heads*ceil(nb / (128 / block)) tiles, rounded
- * up to 256) exceeds BSA_NOALLOC_SCRATCH_BYTES is refused with
- * BSA_ERR_UNSUPPORTED before anything is launched.  Argument errors are those
- * of bsa_attn_fwd.
+ * Limits and errors: a shape whose scratch exceeds BSA_NOALLOC_SCRATCH_BYTES
+ * is refused with
+ * BSA_ERR_UNSUPPORTED before anything is launched.  The scratch is 256 bytes
+ * plus the work plan: 8 bytes per 128-row query tile (B*heads*ceil(nb /
+ * (128 / block)) tiles), and with 64-token blocks 68 bytes per block row
+ * (B*heads*nb rows), each part rounded up to 256 bytes.  Argument errors are
+ * those of bsa_attn_fwd.
  *
  * Set-up: the first call on each device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current).  Make that first call
