@@ -25,6 +25,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
+#include "softmax_math.cuh"
 #include "tma_host.h"
 
 namespace bsa {
@@ -32,10 +33,13 @@ namespace bsa {
 namespace {
 
 using namespace sm100;
+using namespace smx;
 
 constexpr int kThreads = 192;
 constexpr uint64_t kWaitNs = 250ull * 1000ull * 1000ull;  // 250 ms: far beyond any legitimate wait
 constexpr uint32_t kTmemCols = 256;
+// One pair of scores in kPolyEvery takes the software exp2 (0 = none).
+constexpr int kPolyEvery = 0;
 
 struct Ctl {
   uint64_t q_full, k_full, k_empty, v_full, v_empty, s_full, p_full, pv_done;
@@ -46,17 +50,6 @@ struct Ctl {
   uint16_t ent[BSA_MAX_BLOCKS];         // union of the lists, ascending
   uint8_t mem[BSA_MAX_BLOCKS];          // bit h: entry kept by query block h
 };
-
-__device__ __forceinline__ float ex2f(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
-  return y;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
 
 __device__ __forceinline__ void timeout(Ctrl* ctrl, uint32_t site) {
   report_error(ctrl, kErrTimeout, blockIdx.x, threadIdx.x, site);
@@ -304,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
       for (int h = 0; h < 2; ++h) {
         if (lim[h] == 64) {
 #pragma unroll
-          for (int i = 0; i < 64; ++i) mx = fmaxf(mx, x[h * 64 + i]);
+          for (int i = 0; i < 64; i += 2) mx = fmax3(mx, x[h * 64 + i], x[h * 64 + i + 1]);
         } else if (lim[h] > 0) {
 #pragma unroll
           for (int i = 0; i < 64; ++i) mx = (i < lim[h]) ? fmaxf(mx, x[h * 64 + i]) : mx;
@@ -334,9 +327,16 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
       }
       if (grow) m = mnew;
       const float nm = (m == -INFINITY) ? 0.f : -m;
-      // p = 2^(s * scale_log2 - m): one FFMA and one MUFU op per score.
-      // Halves the row's query block does not keep cost nothing.
-      float rs = 0.f, rx = 0.f;
+      // p = 2^(s * scale_log2 - m): one packed FFMA per two scores, then the
+      // MUFU ex2 for most pairs and the FMA-pipe polynomial for one pair in
+      // kPolyEvery.  O is normalised by the sum of the bf16-rounded weights
+      // the P.V product uses (an exact convex combination of V rows up to
+      // accumulation rounding); the LSE, when asked for, uses the fp32 sum of
+      // the unrounded ones.  Halves the row's query block does not keep cost
+      // nothing.
+      const float2 sl2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(nm, nm);
+      float rs[2] = {0.f, 0.f};
+      float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
 #pragma unroll
@@ -346,19 +346,21 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int c = qq * 32 + 2 * i;  // key within the half
-              float p0 = ex2f(fmaf(x[h * 64 + c], scale_log2, nm));
-              float p1 = ex2f(fmaf(x[h * 64 + c + 1], scale_log2, nm));
-              if (lim[h] < 64) {
-                p0 = (c < lim[h]) ? p0 : 0.f;
-                p1 = (c + 1 < lim[h]) ? p1 : 0.f;
+              const float2 y = ffma2(make_float2(x[h * 64 + c], x[h * 64 + c + 1]), sl2, nm2);
+              float2 p;
+              if (kPolyEvery > 0 && (i % kPolyEvery) == kPolyEvery - 1) {
+                p = exp2_poly2(y);
+              } else {
+                p.x = ex2f(y.x);
+                p.y = ex2f(y.y);
               }
-              const uint32_t w = pack_bf16(p0, p1);
-              pk[i] = w;
-              // O is normalised by the sum of the rounded weights the P.V
-              // product uses (an exact convex combination of V rows); the LSE,
-              // when asked for, by the fp32 sum of the unrounded weights.
-              rs += __uint_as_float(w << 16) + __uint_as_float(w & 0xFFFF0000u);
-              if (WITH_LSE) rx += p0 + p1;
+              if (lim[h] < 64) {
+                p.x = (c < lim[h]) ? p.x : 0.f;
+                p.y = (c + 1 < lim[h]) ? p.y : 0.f;
+              }
+              pk[i] = pack_bf16(p.x, p.y);
+              rs[i & 1] = add_bf16x2(rs[i & 1], pk[i]);
+              if (WITH_LSE) acc = fadd2(acc, p);
             }
           } else {
 #pragma unroll
@@ -369,8 +371,8 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
           tmem_st16(trow + 32 * h + 16 * qq, pk);
         }
       }
-      l += rs;
-      if (WITH_LSE) lx += rx;
+      l += rs[0] + rs[1];
+      if (WITH_LSE) lx += acc.x + acc.y;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&c.p_full);

@@ -1,0 +1,567 @@
+// Block-sparse attention forward on the sm_100a tensor cores: persistent,
+// one CTA per SM.  NABLA summary, Metodologia 2 "Expansion": only the listed
+// N x N tiles are computed.
+//
+// Work: the plan's 128-row query tiles (one block of 128, or two blocks of 64,
+// rows 0-63 and 64-127), fetched one at a time from a work counter in the
+// plan's order (longest first within each head).  A tile walks the union of
+// its KV lists in KV tiles of 128 keys (one entry of 128, or two of 64):
+//   S = Q K^T      tcgen05.mma (M=128, N=128), A = Q and B = K from shared
+//                  memory, S in TMEM
+//   softmax        two threads per query row, each on 64 keys of the KV tile:
+//                  masks keys its row's block does not keep (and padding),
+//                  shares the tile max with its partner through shared memory,
+//                  keeps a running base-2 max (O rescaled only when it grows
+//                  by more than 8) and writes P = 2^(s - m) as bf16 over its
+//                  S columns in TMEM
+//   O += P V       tcgen05.mma with A = P from TMEM and B = V (MN-major) from
+//                  shared memory, O in TMEM
+// TMEM holds three S buffers and O (4 x 128 columns), so the S product of
+// KV tile j+2 is queued right behind the P.V product of tile j and the tensor
+// pipe never waits for the softmax of the tile in between; K and V are double
+// buffered in shared memory.  O is normalised by the sum of the bf16-rounded
+// weights the P.V product uses (an exact convex combination of V rows up to
+// accumulation rounding); the LSE uses the fp32 sum of the unrounded ones.
+//
+// Roles: warp 0 issues TMA loads, warp 1 issues MMAs (one elected thread),
+// warps 4-11 run the softmax and the epilogue (warp w reads TMEM lanes
+// 32 (w mod 4) .. +31, keys 64 ((w - 4) div 4) .. +63 of each KV tile).
+// Every mbarrier wait is bounded; on expiry the CTA records BSA_ERR_TIMEOUT in
+// the workspace error word and leaves.
+#include <cmath>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+#include "softmax_math.cuh"
+#include "tma_host.h"
+
+namespace bsa {
+
+namespace {
+
+using namespace sm100;
+using namespace smx;
+
+constexpr int kThreads = 384;
+constexpr int kSoftmaxWarp0 = 4;
+constexpr uint32_t kSoftmaxThreads = 256;
+constexpr uint64_t kWaitNs = 250ull * 1000ull * 1000ull;  // 250 ms: far beyond any legitimate wait
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemO = 384;     // O columns; S buffers at 0, 128, 256
+// One pair of scores in kPolyEvery takes the software exp2 (0 = none).
+constexpr int kPolyEvery = 0;
+
+struct Ctl {
+  uint64_t q_full;
+  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
+  uint64_t s_full[3], p_full[3], pv_done[3];
+  uint32_t tmem_base;
+  int n_ent;
+  int item;
+  int abort;
+  float xmax[2][2][128];   // [tile parity][key half][row]: tile max of each half
+  float xsum[2][2][128];   // [sum kind][key half][row]: row sums at the epilogue
+  uint32_t bm[2][BSA_MAX_BLOCKS / 32];  // kept blocks of each query block of the tile
+  uint16_t ent[BSA_MAX_BLOCKS];         // union of the lists, ascending
+  uint8_t mem[BSA_MAX_BLOCKS];          // bit h: entry kept by query block h
+};
+
+__device__ __forceinline__ void timeout(Ctrl* ctrl, Ctl& c, uint32_t site) {
+  report_error(ctrl, kErrTimeout, blockIdx.x, threadIdx.x, site);
+  c.abort = 1;
+}
+
+// Bounded wait; gives up early once any CTA of the launch has timed out.
+__device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity, Ctrl* ctrl) {
+  return mbar_wait_ns(bar, parity, kWaitNs, &ctrl->error, kErrTimeout);
+}
+
+// Same, with one verdict for the whole warp (the tcgen05.ld/st that follow
+// are warp-collective and must not run in a partial warp).
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, Ctrl* ctrl) {
+  const bool ok = wait(bar, parity, ctrl);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Barrier of the two softmax warps that share TMEM lane quarter q4; returns
+// the AND of `ok` over both warps, so the pair leaves its loop together (a
+// named barrier has no time limit: both warps must always reach it).
+__device__ __forceinline__ bool pair_sync(int q4, bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n"
+      ".reg .pred p, q;\n"
+      "setp.ne.u32 q, %1, 0;\n"
+      "bar.red.and.pred p, %2, 64, q;\n"
+      "selp.u32 %0, 1, 0, p;\n"
+      "}\n"
+      : "=r"(r)
+      : "r"((uint32_t)ok), "r"(1 + q4)
+      : "memory");
+  return r != 0u;
+}
+
+template <int D, int BS, bool WITH_LSE>
+__global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_constant__ CUtensorMap mq,
+                                                               const __grid_constant__ CUtensorMap mk,
+                                                               const __grid_constant__ CUtensorMap mv,
+                                                               const int32_t* __restrict__ kv_count,
+                                                               const int32_t* __restrict__ kv_idx,
+                                                               const int2* __restrict__ items, int* work,
+                                                               float scale_log2, __nv_bfloat16* __restrict__ o,
+                                                               float* __restrict__ lse, Ctrl* ctrl, Dims g,
+                                                               int items_per_bh, int n_items) {
+  constexpr int QB = 128 / BS;          // query blocks per tile
+  constexpr int E = 128 / BS;           // list entries per KV tile
+  constexpr int CH = D / 64;            // 64-column (128-byte) chunks of a row
+  constexpr uint32_t kTile = 128u * D * 2u;
+  constexpr uint32_t kChunk = 128u * 128u;  // bytes of one chunk of a 128-row tile
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = base;
+  uint8_t* sK = base + kTile;          // two stages
+  uint8_t* sV = base + 3 * kTile;      // two stages
+  Ctl& c = *reinterpret_cast<Ctl*>(base + 5 * kTile);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int nb = g.nb;
+  const int nw = (nb + 31) >> 5;
+
+  if (tid == 0) {
+    mbar_init(&c.q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&c.k_full[s], 1);
+      mbar_init(&c.k_empty[s], 1);
+      mbar_init(&c.v_full[s], 1);
+      mbar_init(&c.v_empty[s], 1);
+    }
+    for (int b = 0; b < 3; ++b) {
+      mbar_init(&c.s_full[b], 1);
+      mbar_init(&c.p_full[b], kSoftmaxThreads);
+      mbar_init(&c.pv_done[b], 1);
+    }
+    c.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&c.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&mq);
+    tma_prefetch_desc(&mk);
+    tma_prefetch_desc(&mv);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = c.tmem_base;
+
+  uint32_t jbase = 0;  // KV tiles this CTA has run so far (phase counter of the pipeline)
+  uint32_t nq = 0;     // Q loads so far (phase of q_full)
+
+  for (;;) {
+    if (tid == 0) c.item = atomicAdd(work, 1);
+    for (int i = tid; i < 2 * (BSA_MAX_BLOCKS / 32); i += kThreads) (&c.bm[0][0])[i] = 0u;
+    __syncthreads();
+    const int item = c.item;
+    if (item >= n_items || c.abort) break;
+    const int bh = item / items_per_bh;
+
+    // the tile's query blocks, from the plan (second block -1 when single)
+    const int2 it = items[item];
+    int qblk[QB];
+    bool qval[QB];
+    qblk[0] = it.x;
+    qval[0] = it.x >= 0 && it.x < nb;
+    if (QB == 2) {
+      qblk[QB - 1] = it.y;
+      qval[QB - 1] = it.y >= 0 && it.y < nb;
+    }
+    if (!qval[0]) qblk[0] = 0;  // a corrupt plan: compute nothing for this tile
+
+    // Kept-block bitmaps of the tile's query blocks (duplicates collapse).
+#pragma unroll
+    for (int h = 0; h < QB; ++h) {
+      if (!qval[h]) continue;
+      const size_t row = (size_t)bh * nb + qblk[h];
+      int cnt = kv_count[row];
+      if (cnt < 1 || cnt > nb) {
+        if (tid == 0) report_error(ctrl, kErrCount, (uint32_t)row, (uint32_t)cnt, 3u);
+        cnt = cnt < 0 ? 0 : (cnt > nb ? nb : cnt);
+      }
+      const int32_t* list = kv_idx + row * nb;
+      for (int i = tid; i < cnt; i += kThreads) {
+        const int J = list[i];
+        if (J >= 0 && J < nb) atomicOr(&c.bm[h][J >> 5], 1u << (J & 31));
+        else report_error(ctrl, kErrIndex, (uint32_t)row, (uint32_t)J, 4u);
+      }
+    }
+    __syncthreads();
+
+    // Union list in ascending order (warp 0).
+    if (warp == 0) {
+      int off = 0;
+      for (int w0 = 0; w0 < nw; w0 += 32) {
+        const int wi = w0 + lane;
+        const uint32_t b0 = (wi < nw) ? c.bm[0][wi] : 0u;
+        const uint32_t b1 = (QB > 1 && wi < nw) ? c.bm[1][wi] : 0u;
+        uint32_t u = b0 | b1;
+        const int n = __popc(u);
+        int incl = n;
+#pragma unroll
+        for (int s = 1; s < 32; s <<= 1) {
+          const int t = __shfl_up_sync(0xffffffffu, incl, s);
+          if (lane >= s) incl += t;
+        }
+        int pos = off + incl - n;
+        while (u != 0u) {
+          const int bit = __ffs(u) - 1;
+          u &= u - 1u;
+          c.ent[pos] = (uint16_t)(wi * 32 + bit);
+          c.mem[pos] = (uint8_t)(((b0 >> bit) & 1u) | (((b1 >> bit) & 1u) << 1));
+          ++pos;
+        }
+        off += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (lane == 0) c.n_ent = off;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const int n_ent = c.n_ent;
+    const int n_tiles = (n_ent + E - 1) / E;
+
+    if (warp == 0) {
+      // ---------------------------------------------------------- TMA producer
+      if (lane == 0 && n_tiles > 0) {
+        mbar_arrive_expect_tx(&c.q_full, kTile);
+#pragma unroll
+        for (int ch = 0; ch < CH; ++ch) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            int row0;
+            if (QB == 2) row0 = (qval[h & (QB - 1)] ? qblk[h & (QB - 1)] : qblk[0]) * 64;
+            else row0 = qblk[0] * 128 + 64 * h;
+            tma_load_3d(sQ + ch * kChunk + h * (kChunk / 2), &mq, &c.q_full, ch * 64, row0, bh);
+          }
+        }
+        for (int j = 0; j < n_tiles; ++j) {
+          const uint32_t jg = jbase + j;
+          const int s = jg & 1;
+          int krow[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if (E == 2) {
+              const int idx = (2 * j + h < n_ent) ? 2 * j + h : 2 * j;
+              krow[h] = (int)c.ent[idx] * 64;
+            } else {
+              krow[h] = (int)c.ent[j] * 128 + 64 * h;
+            }
+          }
+          if (jg >= 2 && !wait(&c.k_empty[s], ((jg - 2) >> 1) & 1, ctrl)) { timeout(ctrl, c, 10); break; }
+          mbar_arrive_expect_tx(&c.k_full[s], kTile);
+          uint8_t* dk = sK + s * kTile;
+#pragma unroll
+          for (int ch = 0; ch < CH; ++ch)
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              tma_load_3d(dk + ch * kChunk + h * (kChunk / 2), &mk, &c.k_full[s], ch * 64, krow[h], bh);
+          if (jg >= 2 && !wait(&c.v_empty[s], ((jg - 2) >> 1) & 1, ctrl)) { timeout(ctrl, c, 11); break; }
+          mbar_arrive_expect_tx(&c.v_full[s], kTile);
+          uint8_t* dv = sV + s * kTile;
+#pragma unroll
+          for (int ch = 0; ch < CH; ++ch)
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              tma_load_3d(dv + ch * kChunk + h * (kChunk / 2), &mv, &c.v_full[s], ch * 64, krow[h], bh);
+        }
+      }
+    } else if (warp == 1) {
+      // ---------------------------------------------------------- MMA issuer
+      if (lane == 0 && n_tiles > 0) {
+        constexpr uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);
+        constexpr uint32_t idO = idesc_bf16_f32(128, D, 0, 1);
+        const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV);
+        bool ok = wait(&c.q_full, nq & 1, ctrl);
+        if (!ok) timeout(ctrl, c, 20);
+        // S of global KV tile jg into S buffer jg mod 3 (free once the P.V
+        // product of tile jg - 3 has completed).
+        auto issue_s = [&](uint32_t jg) -> bool {
+          const uint32_t b = jg % 3, s = jg & 1;
+          if (!wait(&c.k_full[s], (jg >> 1) & 1, ctrl)) { timeout(ctrl, c, 21); return false; }
+          if (jg >= 3 && !wait(&c.pv_done[b], ((jg - 3) / 3) & 1, ctrl)) { timeout(ctrl, c, 22); return false; }
+          tc_fence_after();
+          const uint32_t kbase = aK + s * kTile;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
+            mma_ss(tmem + 128 * b, smem_desc_sw128(aQ + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024), idS,
+                   kk > 0);
+          }
+          mma_commit(&c.s_full[b]);
+          mma_commit(&c.k_empty[s]);
+          return true;
+        };
+        if (ok) ok = issue_s(jbase);
+        if (ok && n_tiles > 1) ok = issue_s(jbase + 1);
+        for (int j = 0; ok && j < n_tiles; ++j) {
+          const uint32_t jg = jbase + j;
+          const uint32_t b = jg % 3, s = jg & 1;
+          if (!wait(&c.p_full[b], (jg / 3) & 1, ctrl)) { timeout(ctrl, c, 23); break; }
+          if (!wait(&c.v_full[s], (jg >> 1) & 1, ctrl)) { timeout(ctrl, c, 24); break; }
+          tc_fence_after();
+          const uint32_t vbase = aV + s * kTile;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + kTmemO, tmem + 128 * b + kk * 8, smem_desc_sw128(vbase + kk * 2048, kChunk, 1024), idO,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&c.pv_done[b]);
+          mma_commit(&c.v_empty[s]);
+          if (j + 2 < n_tiles) ok = issue_s(jg + 2);
+        }
+      }
+    } else if (warp >= kSoftmaxWarp0) {
+      // ---------------------------------------------------------- softmax + epilogue
+      const int q4 = warp & 3;                         // TMEM lane quarter of this warp
+      const int hf = (warp - kSoftmaxWarp0) >> 2;      // which 64 keys of each KV tile
+      const int r = q4 * 32 + lane;                    // query row of the tile
+      const int half = (QB == 2) ? (r >> 6) : 0;       // query block of the row
+      const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16);
+      float m = -INFINITY;
+      float l = 0.f, lx = 0.f;
+      bool ok = true;
+      for (int j = 0; j < n_tiles; ++j) {
+        const uint32_t jg = jbase + j;
+        const uint32_t b = jg % 3;
+        int key0, kept;
+        if (E == 2) {
+          const int idx = 2 * j + hf;
+          kept = (idx < n_ent) ? ((c.mem[idx] >> half) & 1) : 0;
+          key0 = (idx < n_ent) ? (int)c.ent[idx] * 64 : 0;
+        } else {
+          kept = 1;
+          key0 = (int)c.ent[j] * 128 + 64 * hf;
+        }
+        const int lim = kept ? max(0, min(64, g.N - key0)) : 0;
+        const bool got = wait_warp(&c.s_full[b], (jg / 3) & 1, ctrl);
+        tc_fence_after();
+        const uint32_t tS = trow + 128 * b;
+        uint32_t sr[64];
+        if (got) {
+          tmem_ld32(tS + 64 * hf, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+          tmem_ld32(tS + 64 * hf + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+          tmem_wait_ld();
+        }
+        const float* x = reinterpret_cast<const float*>(sr);
+        // Max of the raw scores over this half's kept, real keys (scale > 0
+        // keeps the order), four independent chains.
+        float mx;
+        if (!got) {
+          mx = -INFINITY;
+        } else if (lim == 64) {
+          float m0 = x[0], m1 = x[1], m2 = x[2], m3 = x[3];
+#pragma unroll
+          for (int i = 4; i < 64; i += 8) {
+            m0 = fmax3(m0, x[i], x[i + 1]);
+            m1 = fmax3(m1, x[i + 2], x[i + 3]);
+            m2 = fmax3(m2, x[i + 4], x[i + 5]);
+            m3 = fmax3(m3, x[i + 6], x[i + 7]);
+          }
+          mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+        } else {
+          mx = -INFINITY;
+          if (lim > 0) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) mx = (i < lim) ? fmaxf(mx, x[i]) : mx;
+          }
+        }
+        c.xmax[j & 1][hf][r] = mx;
+        if (!pair_sync(q4, got)) { timeout(ctrl, c, 30); ok = false; break; }
+        mx = fmaxf(mx, c.xmax[j & 1][hf ^ 1][r]);
+        const float mnew = fmaxf(m, mx * scale_log2);
+        // The running max moves only when it grows by more than 8 (a factor
+        // 256 in p), or when it is set for the first time.  Both threads of a
+        // row see the same maxima and take the same decisions.  The O rescale
+        // uses warp-collective TMEM accesses, so the whole warp takes it when
+        // any lane needs it (lanes whose max did not move use alpha = 1); it
+        // waits for the P.V product of the previous KV tile first.
+        const bool grow = mnew > m + 8.0f;
+        if (__any_sync(0xffffffffu, grow && m != -INFINITY)) {
+          const uint32_t jp = jg - 1;   // j > 0 here: m is set
+          const bool done = wait_warp(&c.pv_done[jp % 3], (jp / 3) & 1, ctrl);
+          if (!pair_sync(q4, done)) { timeout(ctrl, c, 32); ok = false; break; }
+          tc_fence_after();
+          const float alpha = (grow && m != -INFINITY) ? ex2f(m - mnew) : 1.0f;
+#pragma unroll 1
+          for (int cc = 0; cc < D / 2; cc += 32) {
+            uint32_t ov[32];
+            const uint32_t tO = trow + kTmemO + hf * (D / 2) + cc;
+            tmem_ld32(tO, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+            tmem_st32(tO, ov);
+          }
+          tmem_wait_st();
+          l *= alpha;
+          lx *= alpha;
+        }
+        if (grow) m = mnew;
+        const float nm = (m == -INFINITY) ? 0.f : -m;
+        // p = 2^(s * scale_log2 - m): one packed FFMA per two scores, then the
+        // MUFU ex2 (or, for one pair in kPolyEvery, the FMA-pipe polynomial).
+        const float2 sl2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(nm, nm);
+        float rs[2] = {0.f, 0.f};
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int qq = 0; qq < 2; ++qq) {   // 32 keys -> 16 packed columns at a time
+          uint32_t pk[16];
+          if (lim > 0) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int cidx = qq * 32 + 2 * i;  // key within the half
+              const float2 y = ffma2(make_float2(x[cidx], x[cidx + 1]), sl2, nm2);
+              float2 p;
+              if (kPolyEvery > 0 && (i % kPolyEvery) == kPolyEvery - 1) {
+                p = exp2_poly2(y);
+              } else {
+                p.x = ex2f(y.x);
+                p.y = ex2f(y.y);
+              }
+              if (lim < 64) {
+                p.x = (cidx < lim) ? p.x : 0.f;
+                p.y = (cidx + 1 < lim) ? p.y : 0.f;
+              }
+              pk[i] = pack_bf16(p.x, p.y);
+              rs[i & 1] = add_bf16x2(rs[i & 1], pk[i]);
+              if (WITH_LSE) acc = fadd2(acc, p);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[i] = 0u;
+          }
+          // keys [64 hf + 32 qq, +32) -> bf16 pairs in TMEM columns [32 hf + 16 qq, +16)
+          // of the S buffer (the partner's S columns there were read before pair_sync)
+          tmem_st16(tS + 32 * hf + 16 * qq, pk);
+        }
+        l += rs[0] + rs[1];
+        if (WITH_LSE) lx += acc.x + acc.y;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&c.p_full[b]);
+      }
+
+      // epilogue: O / l -> bf16 rows (this thread: D / 2 columns), LSE
+      const bool have = ok && n_tiles > 0;
+      if (have) {
+        const uint32_t jl = jbase + n_tiles - 1;
+        if (!wait_warp(&c.pv_done[jl % 3], (jl / 3) & 1, ctrl)) { timeout(ctrl, c, 31); ok = false; }
+        tc_fence_after();
+      }
+      c.xsum[0][hf][r] = l;
+      c.xsum[1][hf][r] = lx;
+      ok = pair_sync(q4, ok);
+      const float lt = l + c.xsum[0][hf ^ 1][r];
+      const float lxt = lx + c.xsum[1][hf ^ 1][r];
+      int grow;
+      if (QB == 2) grow = qval[half] ? qblk[half] * 64 + (r & 63) : -1;
+      else grow = qval[0] ? qblk[0] * 128 + r : -1;
+      if (grow >= 0 && grow < g.Npad) {
+        const bool real = ok && have && grow < g.N && lt > 0.f;
+        const float inv = real ? 1.f / lt : 0.f;
+        uint4* orow = reinterpret_cast<uint4*>(o + ((size_t)bh * g.Npad + grow) * D + hf * (D / 2));
+#pragma unroll 1
+        for (int cc = 0; cc < D / 2; cc += 32) {
+          uint32_t ov[32];
+          if (ok && have) {
+            tmem_ld32(trow + kTmemO + hf * (D / 2) + cc, ov);
+            tmem_wait_ld();
+          }
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            w[i] = real ? pack_bf16(__uint_as_float(ov[2 * i]) * inv, __uint_as_float(ov[2 * i + 1]) * inv) : 0u;
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            orow[cc / 8 + i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
+        if (WITH_LSE && hf == 0)
+          lse[(size_t)bh * g.Npad + grow] = real ? (m + __log2f(lxt)) * 0.69314718055994531f : 0.f;
+      }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    jbase += n_tiles;
+    if (n_tiles > 0) ++nq;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+template <int D, int BS, bool WITH_LSE>
+cudaError_t launch_tc2(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
+                       const int32_t* kv_idx, const int2* items, int* work, float scale, void* o, float* lse,
+                       Ctrl* ctrl, cudaStream_t st) {
+  CUtensorMap mq, mk, mv;
+  const uint64_t rows = (uint64_t)g.Npad, bhs = (uint64_t)g.B * g.heads;
+  if (!make_map_bf16_3d(&mq, q, D, rows, bhs, 64, 64) || !make_map_bf16_3d(&mk, k, D, rows, bhs, 64, 64) ||
+      !make_map_bf16_3d(&mv, v, D, rows, bhs, 64, 64))
+    return cudaErrorInvalidValue;
+  const int items_per_bh = (BS == 64) ? (g.nb + 1) / 2 : g.nb;
+  const int n_items = (int)(bhs * items_per_bh);
+  const size_t smem = 5u * 128u * D * 2u + sizeof(Ctl) + 1024u;
+  cudaError_t e =
+      cudaFuncSetAttribute(attn_tc2_kernel<D, BS, WITH_LSE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int grid = n_items < num_sms() ? n_items : num_sms();
+  attn_tc2_kernel<D, BS, WITH_LSE><<<grid, kThreads, smem, st>>>(mq, mk, mv, kv_count, kv_idx, items, work,
+                                                                 scale * 1.4426950408889634f, (__nv_bfloat16*)o, lse,
+                                                                 ctrl, g, items_per_bh, n_items);
+  return cudaGetLastError();
+}
+
+template <int D, int BS>
+cudaError_t launch_tc2_lse(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
+                           const int32_t* kv_idx, const int2* items, int* work, float scale, void* o, float* lse,
+                           Ctrl* ctrl, cudaStream_t st) {
+  if (lse != nullptr)
+    return launch_tc2<D, BS, true>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, st);
+  return launch_tc2<D, BS, false>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, st);
+}
+
+}  // namespace
+
+cudaError_t launch_attn_tc2(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
+                            const int32_t* kv_idx, const int2* items, int* work, float scale, void* o, float* lse,
+                            Ctrl* ctrl, cudaStream_t st) {
+  if (g.d == 128 && g.bs == 64)
+    return launch_tc2_lse<128, 64>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, st);
+  if (g.d == 128 && g.bs == 128)
+    return launch_tc2_lse<128, 128>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, st);
+  if (g.d == 64 && g.bs == 64)
+    return launch_tc2_lse<64, 64>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, st);
+  return launch_tc2_lse<64, 128>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, st);
+}
+
+}  // namespace bsa

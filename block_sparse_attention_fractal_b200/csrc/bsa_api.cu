@@ -160,7 +160,7 @@ bsa_status attn_common(const bsa_shape* s, const void* q, const void* k, const v
   int2* items = (int2*)((char*)workspace + plan_offset(g));
   cudaError_t e = bsa::launch_plan(g, kv_count, kv_idx, items, (cudaStream_t)stream);
   if (e != cudaSuccess) return BSA_ERR_CUDA;
-  return from_cuda(bsa::launch_attn_tc(g, q, k, v, kv_count, kv_idx, items, scale, o, lse_or_null, ctrl,
+  return from_cuda(bsa::launch_attn_tc2(g, q, k, v, kv_count, kv_idx, items, bsa::plan_work_counter(g, items), scale, o, lse_or_null, ctrl,
                                        (cudaStream_t)stream));
 }
 

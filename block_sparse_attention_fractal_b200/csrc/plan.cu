@@ -41,7 +41,7 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 // Plan region of the workspace: items | weights | counts (the last two only
 // with 64-token blocks).
 struct PlanRegion {
-  size_t items, weights, counts, total;
+  size_t items, weights, counts, counter, total;
 };
 
 PlanRegion plan_region(const Dims& g) {
@@ -54,7 +54,8 @@ PlanRegion plan_region(const Dims& g) {
   const size_t w_bytes = (qb == 2) ? bh * g.nb * kWindow * sizeof(uint16_t) : 0;
   R.counts = R.weights + align256(w_bytes);
   const size_t c_bytes = (qb == 2) ? bh * g.nb * sizeof(int32_t) : 0;
-  R.total = R.counts + align256(c_bytes);
+  R.counter = R.counts + align256(c_bytes);  // work counter of the persistent attention kernel
+  R.total = R.counter + 256;
   return R;
 }
 
@@ -113,7 +114,7 @@ template <int QB>
 __global__ void __launch_bounds__(kMatchThreads) match_kernel(const int32_t* __restrict__ kv_count,
                                                               const uint16_t* __restrict__ weights,
                                                               const int32_t* __restrict__ counts, Dims g,
-                                                              int2* __restrict__ items) {
+                                                              int2* __restrict__ items, int* __restrict__ work) {
   __shared__ int partner[BSA_MAX_BLOCKS];
   __shared__ int choice[BSA_MAX_BLOCKS];
   __shared__ int cnt_s[BSA_MAX_BLOCKS];
@@ -127,6 +128,7 @@ __global__ void __launch_bounds__(kMatchThreads) match_kernel(const int32_t* __r
   while (pow2 < n_items) pow2 <<= 1;
 
   if (threadIdx.x == 0) n_keys = 0;
+  if (threadIdx.x == 0 && blockIdx.x == 0) *work = 0;
   for (int r = threadIdx.x; r < nb; r += kMatchThreads) {
     int c;
     if (QB == 2) {
@@ -240,6 +242,8 @@ __global__ void __launch_bounds__(kMatchThreads) match_kernel(const int32_t* __r
 
 size_t plan_region_bytes(const Dims& g) { return plan_region(g).total; }
 
+int* plan_work_counter(const Dims& g, int2* items) { return (int*)((char*)items + plan_region(g).counter); }
+
 cudaError_t launch_plan(const Dims& g, const int32_t* kv_count, const int32_t* kv_idx, int2* items,
                         cudaStream_t st) {
   const PlanRegion R = plan_region(g);
@@ -255,9 +259,10 @@ cudaError_t launch_plan(const Dims& g, const int32_t* kv_count, const int32_t* k
     const size_t smem = (size_t)g.nb * kWindow * sizeof(uint16_t);
     e = cudaFuncSetAttribute(match_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    match_kernel<2><<<bh, kMatchThreads, smem, st>>>(kv_count, weights, counts, g, items);
+    match_kernel<2><<<bh, kMatchThreads, smem, st>>>(kv_count, weights, counts, g, items,
+                                                     plan_work_counter(g, items));
   } else {
-    match_kernel<1><<<bh, kMatchThreads, 0, st>>>(kv_count, nullptr, nullptr, g, items);
+    match_kernel<1><<<bh, kMatchThreads, 0, st>>>(kv_count, nullptr, nullptr, g, items, plan_work_counter(g, items));
   }
   return cudaGetLastError();
 }

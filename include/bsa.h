@@ -85,7 +85,8 @@ BSA_API int64_t bsa_num_blocks(const bsa_shape* s);
  * for this shape: a control block (device error word), the pooled block means
  * of Q and K (2 * B*heads*nb*d doubles) and the attention work plan (one int2
  * per 128-row query tile; with 64-token blocks also 64 bytes of pairing
- * weights and 4 bytes of counts per block row).  0 for an invalid shape. */
+ * weights and 4 bytes of counts per block row; a work counter).  0 for an
+ * invalid shape. */
 BSA_API size_t bsa_workspace_bytes(const bsa_shape* s);
 
 /* Clears the control block of a freshly allocated workspace (async memset).
@@ -186,9 +187,9 @@ BSA_API bsa_status bsa_attn_fwd_baseline(const bsa_shape* s, const void* q, cons
  * is refused with
  * BSA_ERR_UNSUPPORTED before anything is launched.  The scratch is 256 bytes
  * plus the work plan: 8 bytes per 128-row query tile (B*heads*ceil(nb /
- * (128 / block)) tiles), and with 64-token blocks 68 bytes per block row
- * (B*heads*nb rows), each part rounded up to 256 bytes.  Argument errors are
- * those of bsa_attn_fwd.
+ * (128 / block)) tiles), with 64-token blocks 68 bytes per block row
+ * (B*heads*nb rows), and a 256-byte work counter, each part rounded up to 256
+ * bytes.  Argument errors are those of bsa_attn_fwd.
  *
  * Set-up: the first call on each device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current).  Make that first call
