@@ -348,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
               const int c = qq * 32 + 2 * i;  // key within the half
               const float2 y = ffma2(make_float2(x[h * 64 + c], x[h * 64 + c + 1]), sl2, nm2);
               float2 p;
-              if (kPolyEvery > 0 && (i % kPolyEvery) == kPolyEvery - 1) {
+              if (kPolyEvery > 0 && (i % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
                 p = exp2_poly2(y);
               } else {
                 p.x = ex2f(y.x);

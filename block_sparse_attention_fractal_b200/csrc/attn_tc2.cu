@@ -18,12 +18,13 @@
 //                  shared memory, O in TMEM
 // TMEM holds three S buffers and O (4 x 128 columns), so the S product of
 // KV tile j+2 is queued right behind the P.V product of tile j and the tensor
-// pipe never waits for the softmax of the tile in between; K and V are double
-// buffered in shared memory.  O is normalised by the sum of the bf16-rounded
+// pipe never waits for the softmax of the tile in between; K has three and V
+// two stages in shared memory, each loaded by its own producer warp.  O is normalised by the sum of the bf16-rounded
 // weights the P.V product uses (an exact convex combination of V rows up to
 // accumulation rounding); the LSE uses the fp32 sum of the unrounded ones.
 //
-// Roles: warp 0 issues TMA loads, warp 1 issues MMAs (one elected thread),
+// Roles: warps 0 and 2 issue TMA loads (Q and K; V), warp 1 issues MMAs (one
+// elected thread),
 // warps 4-11 run the softmax and the epilogue (warp w reads TMEM lanes
 // 32 (w mod 4) .. +31, keys 64 ((w - 4) div 4) .. +63 of each KV tile).
 // Every mbarrier wait is bounded; on expiry the CTA records BSA_ERR_TIMEOUT in
@@ -45,23 +46,23 @@ using namespace smx;
 
 constexpr int kThreads = 384;
 constexpr int kSoftmaxWarp0 = 4;
-constexpr uint32_t kSoftmaxThreads = 256;
+constexpr uint32_t kGroupThreads = 128;   // threads of one softmax group
 constexpr uint64_t kWaitNs = 250ull * 1000ull * 1000ull;  // 250 ms: far beyond any legitimate wait
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = 384;     // O columns; S buffers at 0, 128, 256
+constexpr uint32_t kTmemO = 256;     // O_0 at 256, O_1 at 384; S_0 at 0, S_1 at 128
 // One pair of scores in kPolyEvery takes the software exp2 (0 = none).
 constexpr int kPolyEvery = 0;
 
 struct Ctl {
   uint64_t q_full;
-  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
-  uint64_t s_full[3], p_full[3], pv_done[3];
+  uint64_t k_full[3], k_empty[3], v_full[2], v_empty[2];
+  uint64_t s_full[2], p_full[2], pv_done[2];   // per softmax group
   uint32_t tmem_base;
   int n_ent;
   int item;
   int abort;
-  float xmax[2][2][128];   // [tile parity][key half][row]: tile max of each half
-  float xsum[2][2][128];   // [sum kind][key half][row]: row sums at the epilogue
+  float xm[2][128];        // [group][row]: running max at the epilogue
+  float xl[2][2][128];     // [group][sum kind][row]: row sums at the epilogue
   uint32_t bm[2][BSA_MAX_BLOCKS / 32];  // kept blocks of each query block of the tile
   uint16_t ent[BSA_MAX_BLOCKS];         // union of the lists, ascending
   uint8_t mem[BSA_MAX_BLOCKS];          // bit h: entry kept by query block h
@@ -121,9 +122,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = base;
-  uint8_t* sK = base + kTile;          // two stages
-  uint8_t* sV = base + 3 * kTile;      // two stages
-  Ctl& c = *reinterpret_cast<Ctl*>(base + 5 * kTile);
+  uint8_t* sK = base + kTile;          // three stages
+  uint8_t* sV = base + 4 * kTile;      // two stages
+  Ctl& c = *reinterpret_cast<Ctl*>(base + 6 * kTile);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -133,16 +134,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
 
   if (tid == 0) {
     mbar_init(&c.q_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < 3; ++s) {
       mbar_init(&c.k_full[s], 1);
       mbar_init(&c.k_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&c.v_full[s], 1);
       mbar_init(&c.v_empty[s], 1);
     }
-    for (int b = 0; b < 3; ++b) {
-      mbar_init(&c.s_full[b], 1);
-      mbar_init(&c.p_full[b], kSoftmaxThreads);
-      mbar_init(&c.pv_done[b], 1);
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&c.s_full[w], 1);
+      mbar_init(&c.p_full[w], kGroupThreads);
+      mbar_init(&c.pv_done[w], 1);
     }
     c.abort = 0;
     fence_mbar_init();
@@ -161,7 +164,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
   tc_fence_after();
   const uint32_t tmem = c.tmem_base;
 
-  uint32_t jbase = 0;  // KV tiles this CTA has run so far (phase counter of the pipeline)
+  uint32_t jbase = 0;  // KV tiles this CTA has run so far (phase counter of the K/V stages)
+  uint32_t gbase[2] = {0u, 0u};  // KV tiles each softmax group has run so far
   uint32_t nq = 0;     // Q loads so far (phase of q_full)
 
   for (;;) {
@@ -237,23 +241,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
     const int n_ent = c.n_ent;
     const int n_tiles = (n_ent + E - 1) / E;
 
-    if (warp == 0) {
-      // ---------------------------------------------------------- TMA producer
+    if (warp == 0 || warp == 2) {
+      // ---------------------------------------------------------- TMA producers
+      // warp 0: Q, then K of every KV tile (three stages); warp 2: V (two
+      // stages), so a V wait never holds back the next K.
+      const bool is_k = warp == 0;
       if (lane == 0 && n_tiles > 0) {
-        mbar_arrive_expect_tx(&c.q_full, kTile);
+        if (is_k) {
+          mbar_arrive_expect_tx(&c.q_full, kTile);
 #pragma unroll
-        for (int ch = 0; ch < CH; ++ch) {
+          for (int ch = 0; ch < CH; ++ch) {
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            int row0;
-            if (QB == 2) row0 = (qval[h & (QB - 1)] ? qblk[h & (QB - 1)] : qblk[0]) * 64;
-            else row0 = qblk[0] * 128 + 64 * h;
-            tma_load_3d(sQ + ch * kChunk + h * (kChunk / 2), &mq, &c.q_full, ch * 64, row0, bh);
+            for (int h = 0; h < 2; ++h) {
+              int row0;
+              if (QB == 2) row0 = (qval[h & (QB - 1)] ? qblk[h & (QB - 1)] : qblk[0]) * 64;
+              else row0 = qblk[0] * 128 + 64 * h;
+              tma_load_3d(sQ + ch * kChunk + h * (kChunk / 2), &mq, &c.q_full, ch * 64, row0, bh);
+            }
           }
         }
         for (int j = 0; j < n_tiles; ++j) {
           const uint32_t jg = jbase + j;
-          const int s = jg & 1;
           int krow[2];
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
@@ -264,149 +272,155 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
               krow[h] = (int)c.ent[j] * 128 + 64 * h;
             }
           }
-          if (jg >= 2 && !wait(&c.k_empty[s], ((jg - 2) >> 1) & 1, ctrl)) { timeout(ctrl, c, 10); break; }
-          mbar_arrive_expect_tx(&c.k_full[s], kTile);
-          uint8_t* dk = sK + s * kTile;
+          if (is_k) {
+            const uint32_t s = jg % 3;
+            if (jg >= 3 && !wait(&c.k_empty[s], ((jg - 3) / 3) & 1, ctrl)) { timeout(ctrl, c, 10); break; }
+            mbar_arrive_expect_tx(&c.k_full[s], kTile);
+            uint8_t* dk = sK + s * kTile;
 #pragma unroll
-          for (int ch = 0; ch < CH; ++ch)
+            for (int ch = 0; ch < CH; ++ch)
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
-              tma_load_3d(dk + ch * kChunk + h * (kChunk / 2), &mk, &c.k_full[s], ch * 64, krow[h], bh);
-          if (jg >= 2 && !wait(&c.v_empty[s], ((jg - 2) >> 1) & 1, ctrl)) { timeout(ctrl, c, 11); break; }
-          mbar_arrive_expect_tx(&c.v_full[s], kTile);
-          uint8_t* dv = sV + s * kTile;
+              for (int h = 0; h < 2; ++h)
+                tma_load_3d(dk + ch * kChunk + h * (kChunk / 2), &mk, &c.k_full[s], ch * 64, krow[h], bh);
+          } else {
+            const uint32_t s = jg & 1;
+            if (jg >= 2 && !wait(&c.v_empty[s], ((jg - 2) >> 1) & 1, ctrl)) { timeout(ctrl, c, 11); break; }
+            mbar_arrive_expect_tx(&c.v_full[s], kTile);
+            uint8_t* dv = sV + s * kTile;
 #pragma unroll
-          for (int ch = 0; ch < CH; ++ch)
+            for (int ch = 0; ch < CH; ++ch)
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
-              tma_load_3d(dv + ch * kChunk + h * (kChunk / 2), &mv, &c.v_full[s], ch * 64, krow[h], bh);
+              for (int h = 0; h < 2; ++h)
+                tma_load_3d(dv + ch * kChunk + h * (kChunk / 2), &mv, &c.v_full[s], ch * 64, krow[h], bh);
+          }
         }
       }
     } else if (warp == 1) {
       // ---------------------------------------------------------- MMA issuer
+      // KV tile j of the item belongs to softmax group w = j mod 2: its S goes
+      // to S buffer w (free once the group's previous P.V product, which read
+      // P from there, has completed) and its P.V product to O_w.
       if (lane == 0 && n_tiles > 0) {
         constexpr uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);
         constexpr uint32_t idO = idesc_bf16_f32(128, D, 0, 1);
         const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV);
         bool ok = wait(&c.q_full, nq & 1, ctrl);
         if (!ok) timeout(ctrl, c, 20);
-        // S of global KV tile jg into S buffer jg mod 3 (free once the P.V
-        // product of tile jg - 3 has completed).
-        auto issue_s = [&](uint32_t jg) -> bool {
-          const uint32_t b = jg % 3, s = jg & 1;
-          if (!wait(&c.k_full[s], (jg >> 1) & 1, ctrl)) { timeout(ctrl, c, 21); return false; }
-          if (jg >= 3 && !wait(&c.pv_done[b], ((jg - 3) / 3) & 1, ctrl)) { timeout(ctrl, c, 22); return false; }
+        auto issue_s = [&](int j) -> bool {
+          const uint32_t jg = jbase + j, ks = jg % 3;
+          const int w = j & 1;
+          const uint32_t gw = gbase[w] + (j >> 1);   // this group's tile count
+          if (!wait(&c.k_full[ks], (jg / 3) & 1, ctrl)) { timeout(ctrl, c, 21); return false; }
+          if (gw >= 1 && !wait(&c.pv_done[w], (gw - 1) & 1, ctrl)) { timeout(ctrl, c, 22); return false; }
           tc_fence_after();
-          const uint32_t kbase = aK + s * kTile;
+          const uint32_t kbase = aK + ks * kTile;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
-            mma_ss(tmem + 128 * b, smem_desc_sw128(aQ + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024), idS,
+            mma_ss(tmem + 128 * w, smem_desc_sw128(aQ + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024), idS,
                    kk > 0);
           }
-          mma_commit(&c.s_full[b]);
-          mma_commit(&c.k_empty[s]);
+          mma_commit(&c.s_full[w]);
+          mma_commit(&c.k_empty[ks]);
           return true;
         };
-        if (ok) ok = issue_s(jbase);
-        if (ok && n_tiles > 1) ok = issue_s(jbase + 1);
+        if (ok) ok = issue_s(0);
+        if (ok && n_tiles > 1) ok = issue_s(1);
         for (int j = 0; ok && j < n_tiles; ++j) {
-          const uint32_t jg = jbase + j;
-          const uint32_t b = jg % 3, s = jg & 1;
-          if (!wait(&c.p_full[b], (jg / 3) & 1, ctrl)) { timeout(ctrl, c, 23); break; }
-          if (!wait(&c.v_full[s], (jg >> 1) & 1, ctrl)) { timeout(ctrl, c, 24); break; }
+          const uint32_t jg = jbase + j, vs = jg & 1;
+          const int w = j & 1;
+          const uint32_t gw = gbase[w] + (j >> 1);
+          // S of tile j + 1 (the other group) as soon as its buffer is free:
+          // the P.V product of tile j - 1 was issued one iteration ago
+          if (j >= 1 && j + 1 < n_tiles && !(ok = issue_s(j + 1))) break;
+          if (!wait(&c.p_full[w], gw & 1, ctrl)) { timeout(ctrl, c, 23); break; }
+          if (!wait(&c.v_full[vs], (jg >> 1) & 1, ctrl)) { timeout(ctrl, c, 24); break; }
           tc_fence_after();
-          const uint32_t vbase = aV + s * kTile;
+          const uint32_t vbase = aV + vs * kTile;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + kTmemO, tmem + 128 * b + kk * 8, smem_desc_sw128(vbase + kk * 2048, kChunk, 1024), idO,
-                   (j > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&c.pv_done[b]);
-          mma_commit(&c.v_empty[s]);
-          if (j + 2 < n_tiles) ok = issue_s(jg + 2);
+            mma_ts(tmem + kTmemO + 128 * w, tmem + 128 * w + kk * 8, smem_desc_sw128(vbase + kk * 2048, kChunk, 1024),
+                   idO, (j >= 2 || kk > 0) ? 1u : 0u);
+          mma_commit(&c.pv_done[w]);
+          mma_commit(&c.v_empty[vs]);
         }
       }
     } else if (warp >= kSoftmaxWarp0) {
       // ---------------------------------------------------------- softmax + epilogue
       const int q4 = warp & 3;                         // TMEM lane quarter of this warp
-      const int hf = (warp - kSoftmaxWarp0) >> 2;      // which 64 keys of each KV tile
+      const int w = (warp - kSoftmaxWarp0) >> 2;       // softmax group: KV tiles j = w mod 2
       const int r = q4 * 32 + lane;                    // query row of the tile
       const int half = (QB == 2) ? (r >> 6) : 0;       // query block of the row
       const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16);
+      const uint32_t tS = trow + 128 * w, tOw = trow + kTmemO + 128 * w;
       float m = -INFINITY;
       float l = 0.f, lx = 0.f;
       bool ok = true;
-      for (int j = 0; j < n_tiles; ++j) {
-        const uint32_t jg = jbase + j;
-        const uint32_t b = jg % 3;
-        int key0, kept;
-        if (E == 2) {
-          const int idx = 2 * j + hf;
-          kept = (idx < n_ent) ? ((c.mem[idx] >> half) & 1) : 0;
-          key0 = (idx < n_ent) ? (int)c.ent[idx] * 64 : 0;
-        } else {
-          kept = 1;
-          key0 = (int)c.ent[j] * 128 + 64 * hf;
+      int mine = 0;   // KV tiles this group ran in this item
+      for (int j = w; j < n_tiles; j += 2, ++mine) {
+        const uint32_t gw = gbase[w] + (j >> 1);
+        int lim[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          int key0, kept;
+          if (E == 2) {
+            const int idx = 2 * j + h;
+            kept = (idx < n_ent) ? ((c.mem[idx] >> half) & 1) : 0;
+            key0 = (idx < n_ent) ? (int)c.ent[idx] * 64 : 0;
+          } else {
+            kept = 1;
+            key0 = (int)c.ent[j] * 128 + 64 * h;
+          }
+          lim[h] = kept ? max(0, min(64, g.N - key0)) : 0;
         }
-        const int lim = kept ? max(0, min(64, g.N - key0)) : 0;
-        const bool got = wait_warp(&c.s_full[b], (jg / 3) & 1, ctrl);
+        if (!wait_warp(&c.s_full[w], gw & 1, ctrl)) { timeout(ctrl, c, 30); ok = false; break; }
         tc_fence_after();
-        const uint32_t tS = trow + 128 * b;
-        uint32_t sr[64];
-        if (got) {
-          tmem_ld32(tS + 64 * hf, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-          tmem_ld32(tS + 64 * hf + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        // Pass 1: row max of the raw scores over the kept, real keys (scale > 0
+        // keeps the order), 64 columns at a time.
+        float mh[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t sr[64];
+          tmem_ld32(tS + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+          tmem_ld32(tS + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
           tmem_wait_ld();
-        }
-        const float* x = reinterpret_cast<const float*>(sr);
-        // Max of the raw scores over this half's kept, real keys (scale > 0
-        // keeps the order), four independent chains.
-        float mx;
-        if (!got) {
-          mx = -INFINITY;
-        } else if (lim == 64) {
-          float m0 = x[0], m1 = x[1], m2 = x[2], m3 = x[3];
+          const float* xh = reinterpret_cast<const float*>(sr);
+          if (lim[h] == 64) {
+            float m0 = xh[0], m1 = xh[1], m2 = xh[2], m3 = xh[3];
 #pragma unroll
-          for (int i = 4; i < 64; i += 8) {
-            m0 = fmax3(m0, x[i], x[i + 1]);
-            m1 = fmax3(m1, x[i + 2], x[i + 3]);
-            m2 = fmax3(m2, x[i + 4], x[i + 5]);
-            m3 = fmax3(m3, x[i + 6], x[i + 7]);
-          }
-          mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
-        } else {
-          mx = -INFINITY;
-          if (lim > 0) {
+            for (int i = 4; i < 64; i += 8) {
+              m0 = fmax3(m0, xh[i], xh[i + 1]);
+              m1 = fmax3(m1, xh[i + 2], xh[i + 3]);
+              m2 = fmax3(m2, xh[i + 4], xh[i + 5]);
+              m3 = fmax3(m3, xh[i + 6], xh[i + 7]);
+            }
+            mh[h] = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+          } else {
+            float mm = -INFINITY;
+            if (lim[h] > 0) {
 #pragma unroll
-            for (int i = 0; i < 64; ++i) mx = (i < lim) ? fmaxf(mx, x[i]) : mx;
+              for (int i = 0; i < 64; ++i) mm = (i < lim[h]) ? fmaxf(mm, xh[i]) : mm;
+            }
+            mh[h] = mm;
           }
         }
-        c.xmax[j & 1][hf][r] = mx;
-        if (!pair_sync(q4, got)) { timeout(ctrl, c, 30); ok = false; break; }
-        mx = fmaxf(mx, c.xmax[j & 1][hf ^ 1][r]);
-        const float mnew = fmaxf(m, mx * scale_log2);
+        const float mnew = fmaxf(m, fmaxf(mh[0], mh[1]) * scale_log2);
         // The running max moves only when it grows by more than 8 (a factor
-        // 256 in p), or when it is set for the first time.  Both threads of a
-        // row see the same maxima and take the same decisions.  The O rescale
-        // uses warp-collective TMEM accesses, so the whole warp takes it when
-        // any lane needs it (lanes whose max did not move use alpha = 1); it
-        // waits for the P.V product of the previous KV tile first.
+        // 256 in p), or when it is set for the first time.  The O rescale uses
+        // warp-collective TMEM accesses, so the whole warp takes it when any
+        // lane needs it (lanes whose max did not move use alpha = 1).  O_w is
+        // stable: its last P.V product completed before this S was issued.
         const bool grow = mnew > m + 8.0f;
         if (__any_sync(0xffffffffu, grow && m != -INFINITY)) {
-          const uint32_t jp = jg - 1;   // j > 0 here: m is set
-          const bool done = wait_warp(&c.pv_done[jp % 3], (jp / 3) & 1, ctrl);
-          if (!pair_sync(q4, done)) { timeout(ctrl, c, 32); ok = false; break; }
-          tc_fence_after();
           const float alpha = (grow && m != -INFINITY) ? ex2f(m - mnew) : 1.0f;
 #pragma unroll 1
-          for (int cc = 0; cc < D / 2; cc += 32) {
+          for (int cc = 0; cc < D; cc += 32) {
             uint32_t ov[32];
-            const uint32_t tO = trow + kTmemO + hf * (D / 2) + cc;
-            tmem_ld32(tO, ov);
+            tmem_ld32(tOw + cc, ov);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-            tmem_st32(tO, ov);
+            tmem_st32(tOw + cc, ov);
           }
           tmem_wait_st();
           l *= alpha;
@@ -414,92 +428,127 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
         }
         if (grow) m = mnew;
         const float nm = (m == -INFINITY) ? 0.f : -m;
-        // p = 2^(s * scale_log2 - m): one packed FFMA per two scores, then the
-        // MUFU ex2 (or, for one pair in kPolyEvery, the FMA-pipe polynomial).
-        const float2 sl2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(nm, nm);
+        // p = 2^(s * scale_log2 - m): one FFMA and one MUFU ex2 per score (or,
+        // for one pair in kPolyEvery, the FMA-pipe polynomial).  O is
+        // normalised by the sum of the bf16-rounded weights the P.V product
+        // uses (an exact convex combination of V rows up to accumulation
+        // rounding); the LSE, when asked for, uses the fp32 sum of the
+        // unrounded ones.  Halves the row's query block does not keep cost
+        // nothing.
+        // Pass 2, 32 keys at a time (the next chunk's load in flight): their
+        // bf16 weights go to TMEM columns [16 c, 16 c + 16) of S buffer w,
+        // whose scores were read in this pass already.
         float rs[2] = {0.f, 0.f};
-        float2 acc = make_float2(0.f, 0.f);
+        float rx = 0.f;
+        uint32_t sc[2][32];
+        tmem_ld32(tS, sc[0]);
 #pragma unroll
-        for (int qq = 0; qq < 2; ++qq) {   // 32 keys -> 16 packed columns at a time
+        for (int cch = 0; cch < 4; ++cch) {
+          const int h = cch >> 1;
+          tmem_wait_ld();
+          if (cch < 3) tmem_ld32(tS + 32 * (cch + 1), sc[(cch + 1) & 1]);
+          const float* x = reinterpret_cast<const float*>(sc[cch & 1]);
           uint32_t pk[16];
-          if (lim > 0) {
+          if (lim[h] > 0) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const int cidx = qq * 32 + 2 * i;  // key within the half
-              const float2 y = ffma2(make_float2(x[cidx], x[cidx + 1]), sl2, nm2);
+              const float y0 = fmaf(x[2 * i], scale_log2, nm), y1 = fmaf(x[2 * i + 1], scale_log2, nm);
               float2 p;
-              if (kPolyEvery > 0 && (i % kPolyEvery) == kPolyEvery - 1) {
-                p = exp2_poly2(y);
+              if (kPolyEvery > 0 && (i % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
+                p = exp2_poly2(make_float2(y0, y1));
               } else {
-                p.x = ex2f(y.x);
-                p.y = ex2f(y.y);
+                p.x = ex2f(y0);
+                p.y = ex2f(y1);
               }
-              if (lim < 64) {
-                p.x = (cidx < lim) ? p.x : 0.f;
-                p.y = (cidx + 1 < lim) ? p.y : 0.f;
+              if (lim[h] < 64) {
+                const int kc = (cch & 1) * 32 + 2 * i;   // key within the half
+                p.x = (kc < lim[h]) ? p.x : 0.f;
+                p.y = (kc + 1 < lim[h]) ? p.y : 0.f;
               }
               pk[i] = pack_bf16(p.x, p.y);
               rs[i & 1] = add_bf16x2(rs[i & 1], pk[i]);
-              if (WITH_LSE) acc = fadd2(acc, p);
+              if (WITH_LSE) rx += p.x + p.y;
             }
           } else {
 #pragma unroll
             for (int i = 0; i < 16; ++i) pk[i] = 0u;
           }
-          // keys [64 hf + 32 qq, +32) -> bf16 pairs in TMEM columns [32 hf + 16 qq, +16)
-          // of the S buffer (the partner's S columns there were read before pair_sync)
-          tmem_st16(tS + 32 * hf + 16 * qq, pk);
+          tmem_st16(tS + 16 * cch, pk);
         }
         l += rs[0] + rs[1];
-        if (WITH_LSE) lx += acc.x + acc.y;
+        if (WITH_LSE) lx += rx;
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&c.p_full[b]);
+        mbar_arrive(&c.p_full[w]);
       }
 
-      // epilogue: O / l -> bf16 rows (this thread: D / 2 columns), LSE
-      const bool have = ok && n_tiles > 0;
-      if (have) {
-        const uint32_t jl = jbase + n_tiles - 1;
-        if (!wait_warp(&c.pv_done[jl % 3], (jl / 3) & 1, ctrl)) { timeout(ctrl, c, 31); ok = false; }
-        tc_fence_after();
-      }
-      c.xsum[0][hf][r] = l;
-      c.xsum[1][hf][r] = lx;
+      // epilogue: the two groups' partial results of row r are merged,
+      // O = (O_0 2^(m_0 - m) + O_1 2^(m_1 - m)) / (l_0 2^(m_0 - m) + l_1 2^(m_1 - m));
+      // group w writes the columns [w D / 2, (w + 1) D / 2) of the row.
+      // This thread reads both groups' O accumulators: wait for the last P.V
+      // product of each group that ran a tile.
+      const int cnt0 = (n_tiles + 1) / 2, cnt1 = n_tiles / 2;
+      const bool has0 = cnt0 > 0, has1 = cnt1 > 0;
+      if (ok && has0 && !wait_warp(&c.pv_done[0], (gbase[0] + cnt0 - 1) & 1, ctrl)) { timeout(ctrl, c, 31); ok = false; }
+      if (ok && has1 && !wait_warp(&c.pv_done[1], (gbase[1] + cnt1 - 1) & 1, ctrl)) { timeout(ctrl, c, 31); ok = false; }
+      tc_fence_after();
+      c.xm[w][r] = (mine > 0) ? m : -INFINITY;
+      c.xl[w][0][r] = l;
+      c.xl[w][1][r] = lx;
       ok = pair_sync(q4, ok);
-      const float lt = l + c.xsum[0][hf ^ 1][r];
-      const float lxt = lx + c.xsum[1][hf ^ 1][r];
+      const float m0 = c.xm[0][r], m1 = c.xm[1][r];
+      const float mt = fmaxf(m0, m1);
+      const float a0 = (has0 && m0 != -INFINITY) ? ex2f(m0 - mt) : 0.f;
+      const float a1 = (has1 && m1 != -INFINITY) ? ex2f(m1 - mt) : 0.f;
+      const float lt = c.xl[0][0][r] * a0 + c.xl[1][0][r] * a1;
+      const float lxt = c.xl[0][1][r] * a0 + c.xl[1][1][r] * a1;
       int grow;
       if (QB == 2) grow = qval[half] ? qblk[half] * 64 + (r & 63) : -1;
       else grow = qval[0] ? qblk[0] * 128 + r : -1;
-      if (grow >= 0 && grow < g.Npad) {
-        const bool real = ok && have && grow < g.N && lt > 0.f;
-        const float inv = real ? 1.f / lt : 0.f;
-        uint4* orow = reinterpret_cast<uint4*>(o + ((size_t)bh * g.Npad + grow) * D + hf * (D / 2));
+      const bool store = grow >= 0 && grow < g.Npad;
+      const bool real = ok && store && grow < g.N && lt > 0.f;
+      const float inv = real ? 1.f / lt : 0.f;
+      const float s0 = a0 * inv, s1 = a1 * inv;
+      uint4* orow = reinterpret_cast<uint4*>(o + ((size_t)bh * g.Npad + (store ? grow : 0)) * D + w * (D / 2));
+      // The TMEM loads are warp-collective: their conditions (ok, has0, has1)
+      // are the same in every lane; only the stores depend on the row.
 #pragma unroll 1
-        for (int cc = 0; cc < D / 2; cc += 32) {
-          uint32_t ov[32];
-          if (ok && have) {
-            tmem_ld32(trow + kTmemO + hf * (D / 2) + cc, ov);
-            tmem_wait_ld();
+      for (int cc = 0; cc < D / 2; cc += 16) {
+        const int col = w * (D / 2) + cc;
+        uint32_t o0[16], o1[16];
+        if (ok && has0) tmem_ld16(trow + kTmemO + col, o0);
+        if (ok && has1) tmem_ld16(trow + kTmemO + 128 + col, o1);
+        if (ok && (has0 || has1)) tmem_wait_ld();
+        uint32_t pw[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float v0 = 0.f, v1 = 0.f;
+          if (has0) {
+            v0 = __uint_as_float(o0[2 * i]) * s0;
+            v1 = __uint_as_float(o0[2 * i + 1]) * s0;
           }
-          uint32_t w[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            w[i] = real ? pack_bf16(__uint_as_float(ov[2 * i]) * inv, __uint_as_float(ov[2 * i + 1]) * inv) : 0u;
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            orow[cc / 8 + i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          if (has1) {
+            v0 = fmaf(__uint_as_float(o1[2 * i]), s1, v0);
+            v1 = fmaf(__uint_as_float(o1[2 * i + 1]), s1, v1);
+          }
+          pw[i] = real ? pack_bf16(v0, v1) : 0u;
         }
-        if (WITH_LSE && hf == 0)
-          lse[(size_t)bh * g.Npad + grow] = real ? (m + __log2f(lxt)) * 0.69314718055994531f : 0.f;
+        if (store) {
+#pragma unroll
+          for (int i = 0; i < 2; ++i)
+            orow[cc / 8 + i] = make_uint4(pw[4 * i], pw[4 * i + 1], pw[4 * i + 2], pw[4 * i + 3]);
+        }
       }
+      if (WITH_LSE && w == 0 && store)
+        lse[(size_t)bh * g.Npad + grow] = real ? (mt + __log2f(lxt)) * 0.69314718055994531f : 0.f;
     }
 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     jbase += n_tiles;
+    gbase[0] += (n_tiles + 1) / 2;
+    gbase[1] += n_tiles / 2;
     if (n_tiles > 0) ++nq;
   }
 
@@ -530,7 +579,7 @@ cudaError_t launch_tc2(const Dims& g, const void* q, const void* k, const void* 
     return cudaErrorInvalidValue;
   const int items_per_bh = (BS == 64) ? (g.nb + 1) / 2 : g.nb;
   const int n_items = (int)(bhs * items_per_bh);
-  const size_t smem = 5u * 128u * D * 2u + sizeof(Ctl) + 1024u;
+  const size_t smem = 6u * 128u * D * 2u + sizeof(Ctl) + 1024u;
   cudaError_t e =
       cudaFuncSetAttribute(attn_tc2_kernel<D, BS, WITH_LSE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
