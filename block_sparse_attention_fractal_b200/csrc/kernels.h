@@ -10,7 +10,8 @@ namespace bsa {
 cudaError_t launch_reorder(const Dims& g, const void* x_bnhd, void* y_bhnd, cudaStream_t st);
 cudaError_t launch_inverse_reorder(const Dims& g, const void* y_bhnd, void* x_bnhd, cudaStream_t st);
 
-// Block means of Q and K (double) into `qbar`, `kbar` [B, heads, nb, d].
+// Block means of Q and K (double): `qbar` [B, heads, nb, d], `kbar`
+// transposed [B, heads, d, nb].
 cudaError_t launch_pool(const Dims& g, const void* q, const void* k, double* qbar, double* kbar, cudaStream_t st);
 
 // Reduced attention + CDF threshold (+ STA union) -> KV lists.

@@ -10,6 +10,7 @@
 // are double, which keeps every threshold decision within ~1e-15 of the exact
 // one; only rows whose prefix mass sits that close to 1 - thr can differ from
 // an exact evaluation.
+#include <algorithm>
 #include <cfloat>
 #include <cmath>
 
@@ -23,9 +24,14 @@ namespace {
 // ---------------------------------------------------------------- pooling
 
 constexpr int kPoolThreads = 256;
+constexpr int kPoolBlocks = 1;   // blocks of one (b, head, tensor) per CTA
 
-// grid (nb, heads, 2*B): z = 2*b + {0: Q, 1: K}.  Each thread accumulates 8
-// columns of one 16-byte vector over every (256/vec)-th row of the block.
+// grid (ceil(nb / kPoolBlocks), heads, 2*B): z = 2*b + {0: Q, 1: K}.  Every
+// load of the CTA's kPoolBlocks blocks is issued before the first add (16
+// 16-byte vectors in flight per thread); each thread accumulates 8 columns of
+// one vector over every (256/vec)-th row of a block, and the partial sums of a
+// block are reduced through shared memory.  Sums of bf16 values in double are
+// exact, so the means are the exact means rounded once.
 template <int D, int BS>
 __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
                                                             double* __restrict__ qbar, double* __restrict__ kbar,
@@ -33,47 +39,60 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const uint4* __restr
   constexpr int kVec = D / 8;
   constexpr int kRowsPerPass = kPoolThreads / kVec;
   constexpr int kIters = BS / kRowsPerPass;
-  __shared__ double part[kRowsPerPass][D];
+  extern __shared__ double part[];   // [kPoolBlocks][kRowsPerPass][D]
 
-  const int I = blockIdx.x;
+  const int I0 = blockIdx.x * kPoolBlocks;
   const int head = blockIdx.y;
   const int which = blockIdx.z & 1;
   const int b = blockIdx.z >> 1;
   const uint4* src = which ? k : q;
   double* dst = which ? kbar : qbar;
   const size_t bh = (size_t)b * g.heads + head;
-  const int lo = I * BS;
-  const int cnt = min(BS, g.N - lo);
   const int c = threadIdx.x % kVec;
   const int r0 = threadIdx.x / kVec;
 
-  uint4 raw[kIters];
+  uint4 raw[kPoolBlocks][kIters];
 #pragma unroll
-  for (int it = 0; it < kIters; ++it) {
-    const int r = r0 + it * kRowsPerPass;
-    raw[it] = (r < cnt) ? __ldcs(src + (bh * g.Npad + lo + r) * kVec + c) : make_uint4(0u, 0u, 0u, 0u);
-  }
-  double acc[8];
+  for (int blk = 0; blk < kPoolBlocks; ++blk) {
+    const int lo = (I0 + blk) * BS;
+    const int cnt = (I0 + blk < g.nb) ? min(BS, g.N - lo) : 0;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) acc[j] = 0.0;
-#pragma unroll
-  for (int it = 0; it < kIters; ++it) {
-    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[it]);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 f = __bfloat1622float2(h2[j]);
-      acc[2 * j] += (double)f.x;
-      acc[2 * j + 1] += (double)f.y;
+    for (int it = 0; it < kIters; ++it) {
+      const int r = r0 + it * kRowsPerPass;
+      raw[blk][it] = (r < cnt) ? __ldcs(src + (bh * g.Npad + lo + r) * kVec + c) : make_uint4(0u, 0u, 0u, 0u);
     }
   }
 #pragma unroll
-  for (int j = 0; j < 8; ++j) part[r0][c * 8 + j] = acc[j];
+  for (int blk = 0; blk < kPoolBlocks; ++blk) {
+    double acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = 0.0;
+#pragma unroll
+    for (int it = 0; it < kIters; ++it) {
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[blk][it]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(h2[j]);
+        acc[2 * j] += (double)f.x;
+        acc[2 * j + 1] += (double)f.y;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) part[(blk * kRowsPerPass + r0) * D + c * 8 + j] = acc[j];
+  }
   __syncthreads();
-  for (int col = threadIdx.x; col < D; col += kPoolThreads) {
-    double s = 0.0;
+  for (int e = threadIdx.x; e < kPoolBlocks * D; e += kPoolThreads) {
+    const int blk = e / D, col = e % D;
+    const int I = I0 + blk;
+    if (I >= g.nb) continue;
+    const int cnt = min(BS, g.N - I * BS);
+    double sum = 0.0;
 #pragma unroll 8
-    for (int i = 0; i < kRowsPerPass; ++i) s += part[i][col];
-    dst[(bh * g.nb + I) * D + col] = s / (double)cnt;
+    for (int i = 0; i < kRowsPerPass; ++i) sum += part[(blk * kRowsPerPass + i) * D + col];
+    // qbar row-major [bh][I][d]; kbar transposed [bh][d][I] (the mask kernel
+    // reads it one column of d at a time for 32 consecutive blocks)
+    if (which) dst[(bh * D + col) * g.nb + I] = sum / (double)cnt;
+    else dst[(bh * g.nb + I) * D + col] = sum / (double)cnt;
   }
 }
 
@@ -81,7 +100,6 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const uint4* __restr
 
 constexpr int kMaskRows = 16;                 // query-block rows per CTA (one warp each)
 constexpr int kMaskThreads = 32 * kMaskRows;  // 512
-constexpr int kMaxJ = BSA_MAX_BLOCKS / 32;
 
 __device__ __forceinline__ double warp_sum(double v) {
 #pragma unroll
@@ -117,22 +135,26 @@ __device__ __forceinline__ void block_tile(int I, const Dims& g, int& t, int& th
   tw = (rem - h * g.W) / g.P;
 }
 
-// grid (ceil(nb / kMaskRows), heads, B).  Dynamic smem: qbar rows
-// [kMaskRows][D] then scores [kMaskRows][nb], both double.
-template <int D>
+// Persistent grid: CTA c handles the groups of kMaskRows rows c, c + gridDim.x,
+// ... of all (b, head).  Dynamic smem: qbar rows [kMaskRows][D] then scores
+// [kMaskRows][nb], both double.  NJ = ceil(nb / 32) rounded up to a power of
+// two: the values of a row that each lane holds in phase 2.
+template <int D, int NJ>
 __global__ void __launch_bounds__(kMaskThreads) mask_kernel(const double* __restrict__ qbar,
                                                             const double* __restrict__ kbar, Dims g, double thr,
                                                             double scale, int sta_t, int sta_h, int sta_w,
                                                             int32_t* __restrict__ kv_count,
                                                             int32_t* __restrict__ kv_idx, uint8_t* __restrict__ mask) {
+  constexpr int kMaxJ = NJ;
   extern __shared__ __align__(16) double smem[];
   double* qs = smem;                       // [kMaskRows][D]
   double* sc = smem + kMaskRows * D;       // [kMaskRows][nb]
   const int nb = g.nb;
-  const int head = blockIdx.y;
-  const int b = blockIdx.z;
-  const size_t bh = (size_t)b * g.heads + head;
-  const int I0 = blockIdx.x * kMaskRows;
+  const int groups = (nb + kMaskRows - 1) / kMaskRows;
+  const int total = groups * g.B * g.heads;
+  for (int grp = blockIdx.x; grp < total; grp += gridDim.x) {
+  const size_t bh = (size_t)(grp / groups);
+  const int I0 = (grp % groups) * kMaskRows;
   const int rows = min(kMaskRows, nb - I0);
 
   for (int i = threadIdx.x; i < kMaskRows * D; i += kMaskThreads) {
@@ -142,21 +164,24 @@ __global__ void __launch_bounds__(kMaskThreads) mask_kernel(const double* __rest
   __syncthreads();
 
   // Phase 1: scores s[r][J] = scale * qbar_r . kbar_J; each thread owns whole
-  // columns J and reuses every kbar element across the CTA's rows.
+  // columns J and reuses every kbar element across the CTA's rows.  kbar is
+  // stored transposed, so a warp reads one d-column of 32 consecutive blocks
+  // (256 contiguous bytes) per load; qbar comes from shared memory (broadcast).
   const double2* q2 = reinterpret_cast<const double2*>(qs);
+  const double* kt = kbar + bh * D * (size_t)nb;
   for (int J = threadIdx.x; J < nb; J += kMaskThreads) {
-    const double2* k2 = reinterpret_cast<const double2*>(kbar + (bh * nb + J) * D);
     double acc[kMaskRows];
 #pragma unroll
     for (int r = 0; r < kMaskRows; ++r) acc[r] = 0.0;
 #pragma unroll 4
     for (int c = 0; c < D / 2; ++c) {
-      const double2 kv = __ldg(k2 + c);
+      const double k0 = __ldg(kt + (size_t)(2 * c) * nb + J);
+      const double k1 = __ldg(kt + (size_t)(2 * c + 1) * nb + J);
 #pragma unroll
       for (int r = 0; r < kMaskRows; ++r) {
         const double2 qv = q2[r * (D / 2) + c];
-        acc[r] = fma(qv.x, kv.x, acc[r]);
-        acc[r] = fma(qv.y, kv.y, acc[r]);
+        acc[r] = fma(qv.x, k0, acc[r]);
+        acc[r] = fma(qv.y, k1, acc[r]);
       }
     }
 #pragma unroll
@@ -167,7 +192,7 @@ __global__ void __launch_bounds__(kMaskThreads) mask_kernel(const double* __rest
   // Phase 2: one warp per row.  Lane L holds J = L + 32 i.
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  if (warp >= rows) return;
+  if (warp < rows) {
   const int I = I0 + warp;
   const double* srow = sc + warp * nb;
 
@@ -188,8 +213,9 @@ __global__ void __launch_bounds__(kMaskThreads) mask_kernel(const double* __rest
     z += a[i];
   }
   z = warp_sum(z);
+  const double rz = 1.0 / z;
 #pragma unroll
-  for (int i = 0; i < kMaxJ; ++i) a[i] = a[i] / z;  // A = e / sum(e), a true division
+  for (int i = 0; i < kMaxJ; ++i) a[i] *= rz;  // A = e / sum(e)
 
   // keep bits: bit i of `keep` <-> J = lane + 32 i
   uint32_t keep = 0u;
@@ -296,39 +322,63 @@ __global__ void __launch_bounds__(kMaskThreads) mask_kernel(const double* __rest
     base += __popc(bal);
   }
   if (lane == 0) kv_count[row] = base;
+  }  // warp < rows
+  __syncthreads();   // qs and sc are rewritten by the next group
+  }  // groups
 }
 
 }  // namespace
 
-cudaError_t launch_pool(const Dims& g, const void* q, const void* k, double* qbar, double* kbar, cudaStream_t st) {
-  dim3 grid(g.nb, g.heads, 2 * g.B);
-  const uint4* q4 = (const uint4*)q;
-  const uint4* k4 = (const uint4*)k;
-  if (g.d == 128 && g.bs == 64) pool_kernel<128, 64><<<grid, kPoolThreads, 0, st>>>(q4, k4, qbar, kbar, g);
-  else if (g.d == 128 && g.bs == 128) pool_kernel<128, 128><<<grid, kPoolThreads, 0, st>>>(q4, k4, qbar, kbar, g);
-  else if (g.d == 64 && g.bs == 64) pool_kernel<64, 64><<<grid, kPoolThreads, 0, st>>>(q4, k4, qbar, kbar, g);
-  else pool_kernel<64, 128><<<grid, kPoolThreads, 0, st>>>(q4, k4, qbar, kbar, g);
+template <int D, int BS>
+cudaError_t launch_pool_t(const Dims& g, const void* q, const void* k, double* qbar, double* kbar, cudaStream_t st) {
+  const dim3 grid((g.nb + kPoolBlocks - 1) / kPoolBlocks, g.heads, 2 * g.B);
+  const size_t smem = (size_t)kPoolBlocks * (kPoolThreads / (D / 8)) * D * sizeof(double);
+  cudaError_t e = cudaFuncSetAttribute(pool_kernel<D, BS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  pool_kernel<D, BS><<<grid, kPoolThreads, smem, st>>>((const uint4*)q, (const uint4*)k, qbar, kbar, g);
   return cudaGetLastError();
+}
+
+cudaError_t launch_pool(const Dims& g, const void* q, const void* k, double* qbar, double* kbar, cudaStream_t st) {
+  if (g.d == 128 && g.bs == 64) return launch_pool_t<128, 64>(g, q, k, qbar, kbar, st);
+  if (g.d == 128 && g.bs == 128) return launch_pool_t<128, 128>(g, q, k, qbar, kbar, st);
+  if (g.d == 64 && g.bs == 64) return launch_pool_t<64, 64>(g, q, k, qbar, kbar, st);
+  return launch_pool_t<64, 128>(g, q, k, qbar, kbar, st);
+}
+
+template <int D, int NJ>
+cudaError_t launch_mask_t(const Dims& g, const double* qbar, const double* kbar, double thr, int sta_t, int sta_h,
+                          int sta_w, int32_t* kv_count, int32_t* kv_idx, uint8_t* mask, cudaStream_t st) {
+  const size_t smem = (size_t)kMaskRows * (g.d + g.nb) * sizeof(double);
+  const double scale = 1.0 / std::sqrt((double)g.d);
+  cudaError_t e = cudaFuncSetAttribute(mask_kernel<D, NJ>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0, per_sm = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, mask_kernel<D, NJ>, kMaskThreads, smem)) !=
+      cudaSuccess)
+    return e;
+  const int total = (g.nb + kMaskRows - 1) / kMaskRows * g.B * g.heads;
+  const int grid = std::max(1, std::min(total, sms * std::max(1, per_sm)));
+  mask_kernel<D, NJ><<<grid, kMaskThreads, smem, st>>>(qbar, kbar, g, thr, scale, sta_t, sta_h, sta_w, kv_count,
+                                                       kv_idx, mask);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_mask_d(const Dims& g, const double* qbar, const double* kbar, double thr, int sta_t, int sta_h,
+                          int sta_w, int32_t* kv_count, int32_t* kv_idx, uint8_t* mask, cudaStream_t st) {
+  if (g.nb <= 128) return launch_mask_t<D, 4>(g, qbar, kbar, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask, st);
+  if (g.nb <= 256) return launch_mask_t<D, 8>(g, qbar, kbar, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask, st);
+  if (g.nb <= 512) return launch_mask_t<D, 16>(g, qbar, kbar, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask, st);
+  return launch_mask_t<D, 32>(g, qbar, kbar, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask, st);
 }
 
 cudaError_t launch_mask(const Dims& g, const double* qbar, const double* kbar, double thr, int sta_t, int sta_h,
                         int sta_w, int32_t* kv_count, int32_t* kv_idx, uint8_t* mask, cudaStream_t st) {
-  dim3 grid((g.nb + kMaskRows - 1) / kMaskRows, g.heads, g.B);
-  const size_t smem = (size_t)kMaskRows * (g.d + g.nb) * sizeof(double);
-  const double scale = 1.0 / std::sqrt((double)g.d);
-  cudaError_t e;
-  if (g.d == 128) {
-    e = cudaFuncSetAttribute(mask_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    mask_kernel<128><<<grid, kMaskThreads, smem, st>>>(qbar, kbar, g, thr, scale, sta_t, sta_h, sta_w, kv_count,
-                                                       kv_idx, mask);
-  } else {
-    e = cudaFuncSetAttribute(mask_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    mask_kernel<64><<<grid, kMaskThreads, smem, st>>>(qbar, kbar, g, thr, scale, sta_t, sta_h, sta_w, kv_count,
-                                                      kv_idx, mask);
-  }
-  return cudaGetLastError();
+  if (g.d == 128) return launch_mask_d<128>(g, qbar, kbar, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask, st);
+  return launch_mask_d<64>(g, qbar, kbar, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask, st);
 }
 
 }  // namespace bsa
