@@ -38,7 +38,13 @@ sys.path.insert(0, ROOT)
 
 METRIC = "block-sparse attn fwd ms & effective TFLOPS (% bf16 peak), Wan-480p shape"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_LAUNCHES_PER_STEP = 8   # reorder x3, pool, mask, plan, attention, inverse reorder
+
+
+def kernel_launches_per_step(w) -> int:
+    """Our kernels in one step: reorder x3, pool + mask (adaptive workloads),
+    plan (overlap + matching with 64-token blocks, one kernel with 128),
+    attention, inverse reorder."""
+    return 3 + (0 if w.iid else 2) + (2 if w.block == 64 else 1) + 1 + 1
 
 
 # ------------------------------------------------------------------ helpers
@@ -61,16 +67,16 @@ def attn_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel: str):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, if the
-    kernel sources have not changed since it was taken (else None)."""
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu
+    summary, if the kernel sources have not changed since it was taken (else None)."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         rec = json.load(f)
     ent = rec.get(kernel)
-    if not ent or ent.get("source_hash") != attn_source_hash():
+    if not ent or ent.get("source_hash") != attn_source_hash() or ent.get("workload") != workload:
         return None
     return ent.get("bytes_per_launch")
 
@@ -90,7 +96,7 @@ class ClockSampler:
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -130,6 +136,15 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """The largest `value` over all ranks (the value itself without a process group)."""
+    if dist is None:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 def aggregate(per_rank_ms, per_rank_flops):
@@ -291,10 +306,7 @@ def run_ours(args, w, rank, world, dist):
         dist.barrier()
     parts = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in events])  # ms
     step_ms = float(parts.sum(axis=1).sum())   # total over K steps
-    per_rank = torch.tensor([step_ms], dtype=torch.float64, device=dev)
-    if dist is not None:
-        dist.all_reduce(per_rank, op=dist.ReduceOp.MAX)
-    t_max = float(per_rank.item())
+    t_max = max_over_ranks(step_ms, dist, dev)
     total_flops = flops_step * args.steps * world
     value = total_flops / (t_max * 1e-3) / 1e12
     ms_per_step = t_max / args.steps
@@ -317,11 +329,10 @@ def run_ours(args, w, rank, world, dist):
         out_pin.copy_(out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_t = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
     if dist is not None:
-        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
         dist.barrier()
-    e2e_value = total_flops / (float(e2e_t.item()) * 1e-3) / 1e12
+    e2e_value = total_flops / (e2e_ms * 1e-3) / 1e12
     if plan.status() != 0:
         raise RuntimeError("device status not OK after the timed steps")
 
@@ -332,7 +343,7 @@ def run_ours(args, w, rank, world, dist):
     peak_tf_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     attn_tf = flops_step / (attn_ms * 1e-3) / 1e12
-    traffic = recorded_traffic("attn")
+    traffic = recorded_traffic("attn", w.name)
     qk_bytes = 2 * w.B * w.heads * w.N * w.d * 2
     kept = float(plan.kv_count.sum().item())
     mask_bytes = qk_bytes + 2 * 2 * w.B * w.heads * plan.nb * w.d * 8 + 4 * (kept + w.B * w.heads * plan.nb)
@@ -367,7 +378,7 @@ def run_ours(args, w, rank, world, dist):
                      "kernel": "attention", "peak_source": f"{src} bf16 burst",
                      "frac_of_sustained": attn_tf / peak_tf_sus},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": KERNEL_LAUNCHES_PER_STEP * args.steps if not w.iid else 6 * args.steps,
+        "gpu_launches": kernel_launches_per_step(w) * args.steps,
         "clocks": clk,
     }
     if cpu is not None:
@@ -378,7 +389,7 @@ def run_ours(args, w, rank, world, dist):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="wan480p")

@@ -34,15 +34,10 @@ int* plan_work_counter(const Dims& g, int2* items);
 cudaError_t launch_plan(const Dims& g, const int32_t* kv_count, const int32_t* kv_idx, int2* items, cudaStream_t st);
 
 // Block-sparse attention on the tcgen05 tensor cores (TMEM accumulators,
-// TMA-staged tiles), tiles as listed by the plan.
-// Persistent version (one CTA per SM, three S buffers in TMEM), fetching
-// tiles from the plan's work counter.
+// TMA-staged tiles): persistent, one CTA per SM, two softmax groups on
+// alternating KV tiles, query tiles fetched from the plan's work counter.
 cudaError_t launch_attn_tc2(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
                             const int32_t* kv_idx, const int2* items, int* work, float scale, void* o, float* lse,
                             Ctrl* ctrl, cudaStream_t st);
-
-cudaError_t launch_attn_tc(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
-                           const int32_t* kv_idx, const int2* items, float scale, void* o, float* lse, Ctrl* ctrl,
-                           cudaStream_t st);
 
 }  // namespace bsa
