@@ -35,6 +35,7 @@ constexpr int kRounds = 6;
 constexpr int kOverlapRows = 32;     // rows whose weights one overlap CTA writes
 constexpr int kOverlapThreads = kOverlapRows * kWindow;  // 1024
 constexpr int kMatchThreads = 1024;
+static_assert(kMatchThreads >= BSA_MAX_BLOCKS, "match_kernel handles one block row per thread");
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -118,16 +119,15 @@ __global__ void __launch_bounds__(kMatchThreads) match_kernel(const int32_t* __r
   __shared__ int partner[BSA_MAX_BLOCKS];
   __shared__ int choice[BSA_MAX_BLOCKS];
   __shared__ int cnt_s[BSA_MAX_BLOCKS];
-  __shared__ unsigned long long key[BSA_MAX_BLOCKS];
-  __shared__ int n_keys;
+  __shared__ int unm[BSA_MAX_BLOCKS];     // unmatched rows, ascending
+  __shared__ int bin[BSA_MAX_BLOCKS];      // tiles per union size (bin nb - size), then their first slot
+  __shared__ int wsum[32];
+  __shared__ int n_unm;
   extern __shared__ uint16_t wts[];   // [nb][kWindow] (QB == 2 only)
   const int nb = g.nb;
   const size_t bh = blockIdx.x;
   const int n_items = (nb + QB - 1) / QB;
-  int pow2 = 1;
-  while (pow2 < n_items) pow2 <<= 1;
 
-  if (threadIdx.x == 0) n_keys = 0;
   if (threadIdx.x == 0 && blockIdx.x == 0) *work = 0;
   for (int r = threadIdx.x; r < nb; r += kMatchThreads) {
     int c;
@@ -178,63 +178,92 @@ __global__ void __launch_bounds__(kMatchThreads) match_kernel(const int32_t* __r
       }
       if (!__syncthreads_or(formed)) break;
     }
-    if (threadIdx.x == 0) {  // the rest, in index order
-      int pending = -1;
-      for (int r = 0; r < nb; ++r) {
-        if (partner[r] >= 0) continue;
-        if (pending < 0) {
-          pending = r;
-        } else {
-          partner[pending] = r;
-          partner[r] = pending;
-          pending = -1;
+    // The rest, paired in index order: rank of each unmatched row by a
+    // block-wide prefix count, then pairs (rank 2k, rank 2k + 1).
+    {
+      const int r = threadIdx.x;   // nb <= kMatchThreads: one row per thread
+      const bool un = r < nb && partner[r] < 0;
+      const int lane = r & 31, wid = r >> 5;
+      const uint32_t bal = __ballot_sync(0xffffffffu, un);
+      if (lane == 0) wsum[wid] = __popc(bal);
+      __syncthreads();
+      if (wid == 0) {
+        const int v = wsum[lane];
+        int incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int t = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += t;
         }
+        wsum[lane] = incl - v;                       // exclusive prefix of warp totals
+        if (lane == 31) n_unm = incl;
       }
-      if (pending >= 0) partner[pending] = pending;  // a single block
+      __syncthreads();
+      if (un) unm[wsum[wid] + __popc(bal & ((1u << lane) - 1u))] = r;
+      __syncthreads();
+      const int n = n_unm;
+      for (int k = threadIdx.x; 2 * k < n; k += kMatchThreads) {
+        const int a = unm[2 * k];
+        const int b2 = (2 * k + 1 < n) ? unm[2 * k + 1] : a;   // an odd one out is a single block
+        partner[a] = b2;
+        partner[b2] = a;
+      }
     }
     __syncthreads();
   }
 
-  // One key per tile (the lower block of each pair): descending union size
-  // (for pairs beyond the window, the sum of both counts), then ascending block.
-  for (int r = threadIdx.x; r < nb; r += kMatchThreads) {
-    const int p = partner[r];
-    if (p < r) continue;
-    int u = cnt_s[r];
-    if (QB == 2 && p != r) {
-      u += cnt_s[p];
-      if (p - r <= kWindow) u -= wts[r * kWindow + (p - r) - 1];
-    }
-    u = min(u, 0xFFFF);
-    const int slot = atomicAdd(&n_keys, 1);
-    key[slot] = ((unsigned long long)(0xFFFFu - (unsigned)u) << 32) | ((unsigned long long)r << 16) |
-                (unsigned long long)(p & 0xFFFF);
-  }
+  // Tiles (the lower block of each pair) in decreasing union size: a counting
+  // sort on the size (at most nb), ties in any order (only the launch order of
+  // equal tiles depends on it, never the result).
+  for (int i = threadIdx.x; i < nb; i += kMatchThreads) bin[i] = 0;
   __syncthreads();
-  for (int i = n_keys + threadIdx.x; i < pow2; i += kMatchThreads) key[i] = ~0ull;
-  __syncthreads();
-  // bitonic sort of the keys, ascending
-  for (int k = 2; k <= pow2; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = threadIdx.x; i < pow2; i += kMatchThreads) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const unsigned long long a = key[i], b = key[ixj];
-          const bool up = (i & k) == 0;
-          if ((a > b) == up) {
-            key[i] = b;
-            key[ixj] = a;
-          }
+  int usz = -1, ur = -1, up = -1;
+  {
+    const int r = threadIdx.x;
+    if (r < nb) {
+      const int p = partner[r];
+      if (p >= r) {
+        int u = cnt_s[r];
+        if (QB == 2 && p != r) {
+          u += cnt_s[p];
+          if (p - r <= kWindow) u -= wts[r * kWindow + (p - r) - 1];
         }
+        usz = min(max(u, 1), nb);
+        ur = r;
+        up = p;
+        atomicAdd(&bin[nb - usz], 1);   // bin 0 = largest size
       }
-      __syncthreads();
     }
   }
-  for (int i = threadIdx.x; i < n_items; i += kMatchThreads) {
-    const unsigned long long kk = key[i];
-    const int r = (int)((kk >> 16) & 0xFFFFu);
-    const int p = (int)(kk & 0xFFFFu);
-    items[bh * n_items + i] = make_int2(r, (QB == 2 && p != r) ? p : -1);
+  __syncthreads();
+  {  // exclusive prefix over the nb bins (one per thread)
+    const int t = threadIdx.x, lane = t & 31, wid = t >> 5;
+    const int v = (t < nb) ? bin[t] : 0;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += x;
+    }
+    if (lane == 31) wsum[wid] = incl;
+    __syncthreads();
+    if (wid == 0) {
+      const int wv = wsum[lane];
+      int wi = wv;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int x = __shfl_up_sync(0xffffffffu, wi, o);
+        if (lane >= o) wi += x;
+      }
+      wsum[lane] = wi - wv;
+    }
+    __syncthreads();
+    if (t < nb) bin[t] = wsum[wid] + incl - v;
+  }
+  __syncthreads();
+  if (usz >= 0) {
+    const int slot = atomicAdd(&bin[nb - usz], 1);
+    if (slot < n_items) items[bh * n_items + slot] = make_int2(ur, (QB == 2 && up != ur) ? up : -1);
   }
 }
 
