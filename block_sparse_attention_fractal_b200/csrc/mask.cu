@@ -163,29 +163,49 @@ __global__ void __launch_bounds__(kMaskThreads) mask_kernel(const double* __rest
   }
   __syncthreads();
 
-  // Phase 1: scores s[r][J] = scale * qbar_r . kbar_J; each thread owns whole
-  // columns J and reuses every kbar element across the CTA's rows.  kbar is
-  // stored transposed, so a warp reads one d-column of 32 consecutive blocks
-  // (256 contiguous bytes) per load; qbar comes from shared memory (broadcast).
-  const double2* q2 = reinterpret_cast<const double2*>(qs);
-  const double* kt = kbar + bh * D * (size_t)nb;
-  for (int J = threadIdx.x; J < nb; J += kMaskThreads) {
-    double acc[kMaskRows];
+  // Phase 1: scores s[r][J] = scale * qbar_r . kbar_J on the fp64 tensor
+  // cores (mma.sync m8n8k4, fp64 multiply-add): warp w computes both 8-row
+  // halves of the CTA's rows against the 8-column tiles w, w + 16, ... of J.
+  // A fragments (qbar rows) come from shared memory, B fragments from the
+  // transposed kbar [bh][d][nb] in global memory (64 contiguous bytes per
+  // fragment row).
+  {
+    constexpr int kWarps = kMaskThreads / 32;
+    constexpr int NT = (NJ * 32 / 8 + kWarps - 1) / kWarps;   // 8-column tiles per warp
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int gq = lane >> 2, tq = lane & 3;                   // fragment row / column group
+    const double* kt = kbar + bh * D * (size_t)nb;
+    double acc[2][NT][2];
 #pragma unroll
-    for (int r = 0; r < kMaskRows; ++r) acc[r] = 0.0;
-#pragma unroll 4
-    for (int c = 0; c < D / 2; ++c) {
-      const double k0 = __ldg(kt + (size_t)(2 * c) * nb + J);
-      const double k1 = __ldg(kt + (size_t)(2 * c + 1) * nb + J);
+    for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-      for (int r = 0; r < kMaskRows; ++r) {
-        const double2 qv = q2[r * (D / 2) + c];
-        acc[r] = fma(qv.x, k0, acc[r]);
-        acc[r] = fma(qv.y, k1, acc[r]);
+      for (int n = 0; n < NT; ++n) acc[mt][n][0] = acc[mt][n][1] = 0.0;
+#pragma unroll 2
+    for (int c0 = 0; c0 < D; c0 += 4) {
+      const double a0 = qs[gq * D + c0 + tq];
+      const double a1 = qs[(8 + gq) * D + c0 + tq];
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        const int J = (wid + n * kWarps) * 8 + gq;
+        const double bv = (J < nb) ? __ldg(kt + (size_t)(c0 + tq) * nb + J) : 0.0;
+        asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};\n"
+                     : "+d"(acc[0][n][0]), "+d"(acc[0][n][1])
+                     : "d"(a0), "d"(bv));
+        asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};\n"
+                     : "+d"(acc[1][n][0]), "+d"(acc[1][n][1])
+                     : "d"(a1), "d"(bv));
       }
     }
+    // accumulator element (row gq + 8 mt, column 2 tq + e) of each tile
 #pragma unroll
-    for (int r = 0; r < kMaskRows; ++r) sc[r * nb + J] = acc[r] * scale;
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        const int Jb = (wid + n * kWarps) * 8 + 2 * tq;
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+          if (Jb + e < nb) sc[(mt * 8 + gq) * nb + Jb + e] = acc[mt][n][e] * scale;
+      }
   }
   __syncthreads();
 
