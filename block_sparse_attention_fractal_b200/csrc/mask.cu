@@ -180,20 +180,40 @@ __global__ void __launch_bounds__(kMaskThreads) mask_kernel(const double* __rest
     for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
       for (int n = 0; n < NT; ++n) acc[mt][n][0] = acc[mt][n][1] = 0.0;
-#pragma unroll 2
-    for (int c0 = 0; c0 < D; c0 += 4) {
-      const double a0 = qs[gq * D + c0 + tq];
-      const double a1 = qs[(8 + gq) * D + c0 + tq];
+    // B fragments are loaded PD k-steps ahead of their use (a register ring),
+    // so the L2 latency of kbar overlaps the MMAs of the steps in between.
+    constexpr int PD = (NT <= 4) ? 4 : 2;
+    constexpr int KS = D / 4;                                  // k-steps of 4
+    double bq[PD][NT];
+    auto load_b = [&](int ks, double (&dst)[NT]) {
 #pragma unroll
       for (int n = 0; n < NT; ++n) {
         const int J = (wid + n * kWarps) * 8 + gq;
-        const double bv = (J < nb) ? __ldg(kt + (size_t)(c0 + tq) * nb + J) : 0.0;
-        asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};\n"
-                     : "+d"(acc[0][n][0]), "+d"(acc[0][n][1])
-                     : "d"(a0), "d"(bv));
-        asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};\n"
-                     : "+d"(acc[1][n][0]), "+d"(acc[1][n][1])
-                     : "d"(a1), "d"(bv));
+        dst[n] = (J < nb) ? __ldg(kt + (size_t)(4 * ks + tq) * nb + J) : 0.0;
+      }
+    };
+#pragma unroll
+    for (int p = 0; p < PD; ++p) load_b(p, bq[p]);
+#pragma unroll 1
+    for (int ks0 = 0; ks0 < KS; ks0 += PD) {
+#pragma unroll
+      for (int p = 0; p < PD; ++p) {
+        const int ks = ks0 + p;
+        const double a0 = qs[gq * D + 4 * ks + tq];
+        const double a1 = qs[(8 + gq) * D + 4 * ks + tq];
+        double bv[NT];
+#pragma unroll
+        for (int n = 0; n < NT; ++n) bv[n] = bq[p][n];
+        if (ks + PD < KS) load_b(ks + PD, bq[p]);
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};\n"
+                       : "+d"(acc[0][n][0]), "+d"(acc[0][n][1])
+                       : "d"(a0), "d"(bv[n]));
+          asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};\n"
+                       : "+d"(acc[1][n][0]), "+d"(acc[1][n][1])
+                       : "d"(a1), "d"(bv[n]));
+        }
       }
     }
     // accumulator element (row gq + 8 mt, column 2 tq + e) of each tile
@@ -252,10 +272,20 @@ __global__ void __launch_bounds__(kMaskThreads) mask_kernel(const double* __rest
   } else {
     // Largest key v (bit pattern of a non-negative double, monotone in value)
     // with mass(A >= v) >= target: the probability of the last kept block.
-    unsigned long long lo = 0ull, hi = ~0ull;
+    // Bits above the largest key's highest set bit are 0 in v: the search
+    // starts below them (every key is below hi = 2^(top + 1)).
+    unsigned long long kmax = 0ull;
+#pragma unroll
+    for (int i = 0; i < kMaxJ; ++i) {
+      const unsigned long long key = (unsigned long long)__double_as_longlong(a[i]);
+      kmax = (lane + 32 * i < nb && key > kmax) ? key : kmax;
+    }
+    kmax = warp_max(kmax);
+    const int top = 63 - __clzll((long long)kmax);
+    unsigned long long lo = 0ull, hi = (top >= 63) ? ~0ull : (1ull << (top + 1));
     int cnt_lo = nb, cnt_hi = 0;
     bool unique = false;
-    for (int bit = 62; bit >= 0; --bit) {
+    for (int bit = top; bit >= 0; --bit) {
       const unsigned long long cand = lo | (1ull << bit);
       double m = 0.0;
       int c = 0;
@@ -266,7 +296,7 @@ __global__ void __launch_bounds__(kMaskThreads) mask_kernel(const double* __rest
         c += ge ? 1 : 0;
       }
       m = warp_sum(m);
-      c = warp_sum(c);
+      c = __reduce_add_sync(0xffffffffu, c);
       if (m >= target) {
         lo = cand;
         cnt_lo = c;
