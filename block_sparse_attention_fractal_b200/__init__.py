@@ -27,9 +27,11 @@ __all__ = ["BsaError", "Shape", "make_shape", "NablaAttention", "reorder", "inve
 
 
 class NablaAttention:
-    """Owns the device buffers of one shape and runs the whole path on the
-    current stream: reorder Q, K, V -> block mask -> block-sparse attention ->
-    inverse reorder.  Buffers are allocated once (torch) and reused."""
+    """Owns the device buffers of one shape and runs the whole path: reorder
+    Q, K, V -> block mask -> block-sparse attention -> inverse reorder, ordered
+    on the current stream.  V's reorder runs on a side stream, concurrently
+    with the block mask (which needs only Q and K); the attention waits for
+    both.  Buffers are allocated once (torch) and reused."""
 
     def __init__(self, shape: Shape, device="cuda", with_mask: bool = False, with_lse: bool = False):
         st = validate_shape(shape)
@@ -52,6 +54,20 @@ class NablaAttention:
         ws_bytes = workspace_bytes(shape)
         self.ws = torch.empty((ws_bytes + 15) // 16 * 16, dtype=torch.uint8, **kw)
         workspace_init(self.ws)
+        self.side = torch.cuda.Stream(device=dev)
+
+    def reorder_inputs(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor) -> None:
+        """Q and K on the current stream, V on the side stream (joined by
+        join_side before the attention)."""
+        main = torch.cuda.current_stream(q.device)
+        reorder(self.shape, q, self.q)
+        reorder(self.shape, k, self.k)
+        self.side.wait_stream(main)
+        with torch.cuda.stream(self.side):
+            reorder(self.shape, v, self.v)
+
+    def join_side(self) -> None:
+        torch.cuda.current_stream(self.q.device).wait_stream(self.side)
 
     def mask_step(self, thr: float, sta: Optional[Tuple[int, int, int]] = None) -> None:
         build_block_mask(self.shape, self.q, self.k, thr, sta, self.kv_count, self.kv_idx, self.mask, self.ws)
@@ -63,10 +79,9 @@ class NablaAttention:
     def __call__(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, thr: float,
                  sta: Optional[Tuple[int, int, int]] = None, scale: float = 0.0,
                  out: Optional[torch.Tensor] = None) -> torch.Tensor:
-        reorder(self.shape, q, self.q)
-        reorder(self.shape, k, self.k)
-        reorder(self.shape, v, self.v)
+        self.reorder_inputs(q, k, v)
         self.mask_step(thr, sta)
+        self.join_side()
         self.attention_step(scale)
         if out is None:
             out = torch.empty_like(q)

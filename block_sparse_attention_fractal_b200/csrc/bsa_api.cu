@@ -126,7 +126,7 @@ bsa_status bsa_build_block_mask(const bsa_shape* s, const void* q_bhnd, const vo
   double* qbar = (double*)((char*)workspace + sizeof(Ctrl));
   double* kbar = qbar + pooled_bytes(g) / sizeof(double);
   cudaStream_t cs = (cudaStream_t)stream;
-  cudaError_t e = bsa::launch_pool(g, q_bhnd, k_bhnd, qbar, kbar, cs);
+  cudaError_t e = bsa::launch_pool(g, q_bhnd, k_bhnd, qbar, kbar, (Ctrl*)workspace, cs);
   if (e != cudaSuccess) return BSA_ERR_CUDA;
   e = bsa::launch_mask(g, qbar, kbar, (double)thr, sta ? sta_t : -1, sta ? sta_h : -1, sta ? sta_w : -1, kv_count,
                        kv_idx, mask_or_null, cs);

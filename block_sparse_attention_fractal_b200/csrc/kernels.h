@@ -12,7 +12,8 @@ cudaError_t launch_inverse_reorder(const Dims& g, const void* y_bhnd, void* x_bn
 
 // Block means of Q and K (double): `qbar` [B, heads, nb, d], `kbar`
 // transposed [B, heads, d, nb].
-cudaError_t launch_pool(const Dims& g, const void* q, const void* k, double* qbar, double* kbar, cudaStream_t st);
+cudaError_t launch_pool(const Dims& g, const void* q, const void* k, double* qbar, double* kbar, Ctrl* ctrl,
+                        cudaStream_t st);
 
 // Reduced attention + CDF threshold (+ STA union) -> KV lists.
 cudaError_t launch_mask(const Dims& g, const double* qbar, const double* kbar, double thr, int sta_t, int sta_h,

@@ -16,6 +16,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace bsa {
 
@@ -24,75 +25,104 @@ namespace {
 // ---------------------------------------------------------------- pooling
 
 constexpr int kPoolThreads = 256;
-constexpr int kPoolBlocks = 1;   // blocks of one (b, head, tensor) per CTA
-
-// grid (ceil(nb / kPoolBlocks), heads, 2*B): z = 2*b + {0: Q, 1: K}.  Every
-// load of the CTA's kPoolBlocks blocks is issued before the first add (16
-// 16-byte vectors in flight per thread); each thread accumulates 8 columns of
-// one vector over every (256/vec)-th row of a block, and the partial sums of a
-// block are reduced through shared memory.  Sums of bf16 values in double are
-// exact, so the means are the exact means rounded once.
+// block tiles in flight per CTA (64 KB of stages: several CTAs per SM)
 template <int D, int BS>
-__global__ void __launch_bounds__(kPoolThreads) pool_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
+constexpr int pool_stages() { return (BS * D * 2 <= 16384) ? 4 : 2; }
+constexpr uint64_t kPoolWaitNs = 250ull * 1000ull * 1000ull;
+
+// Persistent: CTA c pools the blocks c, c + gridDim.x, ... of all (tensor, b,
+// head) in that order (item = ((which * B + b) * heads + head) * nb + I,
+// which 0 = Q, 1 = K).  Each block tile (bs rows x d bf16, contiguous in
+// kernel order) arrives by one bulk copy into a ring of kPoolStages shared
+// memory stages, so several tiles per SM are in flight while earlier ones are
+// reduced.  Thread t sums the column pair t mod (d/2) over every
+// (256 / (d/2))-th valid row; the partial sums are combined through shared
+// memory in double.  Sums of bf16 values in double are exact, so the means are
+// the exact means rounded once.  A bulk copy that does not arrive in time sets
+// BSA_ERR_TIMEOUT in the error word and the CTA stops.
+template <int D, int BS>
+__global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __nv_bfloat16* __restrict__ q,
+                                                            const __nv_bfloat16* __restrict__ k,
                                                             double* __restrict__ qbar, double* __restrict__ kbar,
-                                                            Dims g) {
-  constexpr int kVec = D / 8;
-  constexpr int kRowsPerPass = kPoolThreads / kVec;
-  constexpr int kIters = BS / kRowsPerPass;
-  extern __shared__ double part[];   // [kPoolBlocks][kRowsPerPass][D]
+                                                            Ctrl* ctrl, Dims g) {
+  constexpr uint32_t kTileBytes = BS * D * 2;
+  constexpr int kPoolStages = pool_stages<D, BS>();
+  constexpr int kPairs = D / 2;                    // bf16 column pairs of a row
+  constexpr int kRowGroups = kPoolThreads / kPairs;
+  extern __shared__ __align__(128) uint8_t pool_smem[];
+  uint8_t* tiles = pool_smem;                                             // [stages][tile]
+  double* part = reinterpret_cast<double*>(pool_smem + kPoolStages * kTileBytes);  // [row groups][D]
+  __shared__ uint64_t full[4];
+  __shared__ int stop;
 
-  const int I0 = blockIdx.x * kPoolBlocks;
-  const int head = blockIdx.y;
-  const int which = blockIdx.z & 1;
-  const int b = blockIdx.z >> 1;
-  const uint4* src = which ? k : q;
-  double* dst = which ? kbar : qbar;
-  const size_t bh = (size_t)b * g.heads + head;
-  const int c = threadIdx.x % kVec;
-  const int r0 = threadIdx.x / kVec;
-
-  uint4 raw[kPoolBlocks][kIters];
-#pragma unroll
-  for (int blk = 0; blk < kPoolBlocks; ++blk) {
-    const int lo = (I0 + blk) * BS;
-    const int cnt = (I0 + blk < g.nb) ? min(BS, g.N - lo) : 0;
-#pragma unroll
-    for (int it = 0; it < kIters; ++it) {
-      const int r = r0 + it * kRowsPerPass;
-      raw[blk][it] = (r < cnt) ? __ldcs(src + (bh * g.Npad + lo + r) * kVec + c) : make_uint4(0u, 0u, 0u, 0u);
-    }
-  }
-#pragma unroll
-  for (int blk = 0; blk < kPoolBlocks; ++blk) {
-    double acc[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j] = 0.0;
-#pragma unroll
-    for (int it = 0; it < kIters; ++it) {
-      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[blk][it]);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 f = __bfloat1622float2(h2[j]);
-        acc[2 * j] += (double)f.x;
-        acc[2 * j + 1] += (double)f.y;
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) part[(blk * kRowsPerPass + r0) * D + c * 8 + j] = acc[j];
+  const int total = 2 * g.B * g.heads * g.nb;
+  const int G = gridDim.x;
+  auto item_ptr = [&](int it) -> const __nv_bfloat16* {
+    const int I = it % g.nb;
+    const int rest = it / g.nb;                    // (which * B + b) * heads + head
+    const int which = rest / (g.B * g.heads);
+    const size_t bh = rest % (g.B * g.heads);
+    const __nv_bfloat16* src = which ? k : q;
+    return src + (bh * g.Npad + (size_t)I * BS) * D;
+  };
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPoolStages; ++s) sm100::mbar_init(&full[s], 1);
+    stop = 0;
+    sm100::fence_mbar_init();
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < kPoolBlocks * D; e += kPoolThreads) {
-    const int blk = e / D, col = e % D;
-    const int I = I0 + blk;
-    if (I >= g.nb) continue;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPoolStages; ++s) {
+      const int it = blockIdx.x + s * G;
+      if (it >= total) break;
+      sm100::mbar_arrive_expect_tx(&full[s], kTileBytes);
+      sm100::bulk_load(tiles + s * kTileBytes, item_ptr(it), kTileBytes, &full[s]);
+    }
+  }
+  const int cp = threadIdx.x % kPairs;
+  const int rg = threadIdx.x / kPairs;
+  for (int n = 0;; ++n) {
+    const int it = blockIdx.x + n * G;
+    if (it >= total) break;
+    const int s = n % kPoolStages;
+    const bool ok = sm100::mbar_wait_ns(&full[s], (n / kPoolStages) & 1, kPoolWaitNs, &ctrl->error, kErrTimeout);
+    if (!ok) {
+      if (threadIdx.x == 0) report_error(ctrl, kErrTimeout, blockIdx.x, (uint32_t)it, 40u);
+      stop = 1;
+    }
+    __syncthreads();
+    if (stop) break;
+    const int I = it % g.nb;
     const int cnt = min(BS, g.N - I * BS);
-    double sum = 0.0;
-#pragma unroll 8
-    for (int i = 0; i < kRowsPerPass; ++i) sum += part[(blk * kRowsPerPass + i) * D + col];
-    // qbar row-major [bh][I][d]; kbar transposed [bh][d][I] (the mask kernel
-    // reads it one column of d at a time for 32 consecutive blocks)
-    if (which) dst[(bh * D + col) * g.nb + I] = sum / (double)cnt;
-    else dst[(bh * g.nb + I) * D + col] = sum / (double)cnt;
+    const __nv_bfloat162* t2 = reinterpret_cast<const __nv_bfloat162*>(tiles + s * kTileBytes);
+    double a0 = 0.0, a1 = 0.0;
+#pragma unroll 4
+    for (int r = rg; r < cnt; r += kRowGroups) {
+      const float2 f = __bfloat1622float2(t2[r * kPairs + cp]);
+      a0 += (double)f.x;
+      a1 += (double)f.y;
+    }
+    part[rg * D + 2 * cp] = a0;
+    part[rg * D + 2 * cp + 1] = a1;
+    __syncthreads();   // the stage is read and the partial sums are in place
+    if (threadIdx.x == 0 && it + kPoolStages * G < total) {
+      sm100::mbar_arrive_expect_tx(&full[s], kTileBytes);
+      sm100::bulk_load(tiles + s * kTileBytes, item_ptr(it + kPoolStages * G), kTileBytes, &full[s]);
+    }
+    if (threadIdx.x < D) {
+      const int col = threadIdx.x;
+      double sum = 0.0;
+#pragma unroll
+      for (int i = 0; i < kRowGroups; ++i) sum += part[i * D + col];
+      const int rest = it / g.nb;
+      const int which = rest / (g.B * g.heads);
+      const size_t bh = rest % (g.B * g.heads);
+      // qbar row-major [bh][I][d]; kbar transposed [bh][d][I] (the mask kernel
+      // reads it one column of d at a time)
+      if (which) kbar[(bh * D + col) * g.nb + I] = sum / (double)cnt;
+      else qbar[(bh * g.nb + I) * D + col] = sum / (double)cnt;
+    }
+    __syncthreads();   // part is rewritten by the next block
   }
 }
 
@@ -380,20 +410,30 @@ __global__ void __launch_bounds__(kMaskThreads) mask_kernel(const double* __rest
 }  // namespace
 
 template <int D, int BS>
-cudaError_t launch_pool_t(const Dims& g, const void* q, const void* k, double* qbar, double* kbar, cudaStream_t st) {
-  const dim3 grid((g.nb + kPoolBlocks - 1) / kPoolBlocks, g.heads, 2 * g.B);
-  const size_t smem = (size_t)kPoolBlocks * (kPoolThreads / (D / 8)) * D * sizeof(double);
+cudaError_t launch_pool_t(const Dims& g, const void* q, const void* k, double* qbar, double* kbar, Ctrl* ctrl,
+                          cudaStream_t st) {
+  const size_t smem = (size_t)pool_stages<D, BS>() * BS * D * 2 + (size_t)(kPoolThreads / (D / 2)) * D * sizeof(double);
   cudaError_t e = cudaFuncSetAttribute(pool_kernel<D, BS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  pool_kernel<D, BS><<<grid, kPoolThreads, smem, st>>>((const uint4*)q, (const uint4*)k, qbar, kbar, g);
+  int dev = 0, sms = 0, per_sm = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pool_kernel<D, BS>, kPoolThreads, smem)) !=
+      cudaSuccess)
+    return e;
+  const int total = 2 * g.B * g.heads * g.nb;
+  const int grid = std::max(1, std::min(total, sms * std::max(1, per_sm)));
+  pool_kernel<D, BS><<<grid, kPoolThreads, smem, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qbar,
+                                                       kbar, ctrl, g);
   return cudaGetLastError();
 }
 
-cudaError_t launch_pool(const Dims& g, const void* q, const void* k, double* qbar, double* kbar, cudaStream_t st) {
-  if (g.d == 128 && g.bs == 64) return launch_pool_t<128, 64>(g, q, k, qbar, kbar, st);
-  if (g.d == 128 && g.bs == 128) return launch_pool_t<128, 128>(g, q, k, qbar, kbar, st);
-  if (g.d == 64 && g.bs == 64) return launch_pool_t<64, 64>(g, q, k, qbar, kbar, st);
-  return launch_pool_t<64, 128>(g, q, k, qbar, kbar, st);
+cudaError_t launch_pool(const Dims& g, const void* q, const void* k, double* qbar, double* kbar, Ctrl* ctrl,
+                        cudaStream_t st) {
+  if (g.d == 128 && g.bs == 64) return launch_pool_t<128, 64>(g, q, k, qbar, kbar, ctrl, st);
+  if (g.d == 128 && g.bs == 128) return launch_pool_t<128, 128>(g, q, k, qbar, kbar, ctrl, st);
+  if (g.d == 64 && g.bs == 64) return launch_pool_t<64, 64>(g, q, k, qbar, kbar, ctrl, st);
+  return launch_pool_t<64, 128>(g, q, k, qbar, kbar, ctrl, st);
 }
 
 template <int D, int NJ>
