@@ -372,6 +372,10 @@ def run_ours(args, w, rank, world, dist):
             "mask_pct_hbm": 100.0 * mask_bytes / (mask_ms * 1e-3) / 1e9 / hbm if mask_ms > 0 else None,
             "reorder_gbs": reorder_bytes / (float(br[0]) * 1e-3) / 1e9,
             "mask_precision": "f64 pooled means, dots and masses",
+            "step_ms_median": float(np.median(parts.sum(axis=1))),
+            "step_ms_min": float(parts.sum(axis=1).min()),
+            "attn_ms_median": float(np.median(parts[:, 2])),
+            "attn_ms_min": float(parts[:, 2].min()),
         },
         "roofline": {"bound": "tensor", "achieved": attn_tf, "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": attn_tf / peak_tf, "traffic": traffic,
