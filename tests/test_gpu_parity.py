@@ -190,3 +190,47 @@ def test_attention_large_values_within_bf16_resolution(bsa):
     got, want = to64(plan.o)[:, :, :w.N], O_ref[:, :, :w.N]
     assert np.abs(want).max() > 8.0
     assert np.all(np.abs(got - want) <= MAX_ABS + _half_ulp_bf16(want))
+
+
+# Edge cases: the largest nb the kernels accept (1024 blocks of 64 tokens), a
+# threshold close to 1 (about one block per row), batch 2 with 128-token blocks.
+EDGE = [
+    small("max_blocks", 1, 1, 256, 256, 1, 64, 64, 8, 0.3, alpha=2.0, seed=21),
+    small("thr_near_one", 1, 3, 16, 24, 2, 128, 64, 8, 0.995, seed=22),
+    small("batch2_b128", 2, 2, 24, 24, 2, 128, 128, 8, 0.2, seed=23),
+]
+
+
+@pytest.mark.parametrize("w", EDGE, ids=lambda w: w.name)
+def test_edge_shapes_mask_and_attention(bsa, w):
+    q, k, v = synth.make_qkv(w)
+    plan = bsa.NablaAttention(_shape(bsa, w), with_mask=True, with_lse=True)
+    assert plan.nb <= 1024
+    _run_mask(bsa, w, plan, q.cuda(), k.cuda())
+    bsa.reorder(plan.shape, v.cuda(), plan.v)
+    assert plan.status() == 0
+    q64, k64, v64 = to64(plan.q), to64(plan.k), to64(plan.v)
+    keep_ref, amb = oracle.block_mask(q64, k64, w.T, w.H, w.W, w.patch, w.block, w.thr, w.sta)
+    keep = lists_to_keep(plan.kv_count, plan.kv_idx, plan.nb)
+    mismatch = (keep != keep_ref) & ~amb
+    assert not mismatch.any(), f"{int(mismatch.sum())} unambiguous blocks differ"
+    if w.thr > 0.99:
+        assert keep_ref.sum(axis=-1).mean() < 2.0          # about one block per row
+    # attention with the oracle's mask, sampled rows (the largest case has 1024 blocks)
+    cnt, idx = oracle.mask_to_lists(keep_ref)
+    plan.kv_count.copy_(torch.from_numpy(cnt))
+    plan.kv_idx.copy_(torch.from_numpy(idx))
+    plan.attention_step()
+    torch.cuda.synchronize()
+    assert plan.status() == 0
+    rng = np.random.default_rng(5)
+    picks = {(w.B - 1, w.heads - 1, plan.nb - 1), (0, 0, 0)}
+    while len(picks) < min(12, w.B * w.heads * plan.nb):
+        picks.add((int(rng.integers(w.B)), int(rng.integers(w.heads)), int(rng.integers(plan.nb))))
+    O_ref, lse_ref = oracle.masked_attention(q64, k64, v64, keep_ref, w.N, w.block, blocks=sorted(picks))
+    O, lse = to64(plan.o), to64(plan.lse)
+    for (b, h, I) in sorted(picks):
+        lo, hi = I * w.block, min((I + 1) * w.block, w.N)
+        mx, mean = compare_outputs(O[b, h, lo:hi], O_ref[b, h, lo:hi])
+        assert mx <= MAX_ABS and mean <= MEAN_ABS, ((b, h, I), mx, mean)
+        assert np.abs(lse[b, h, lo:hi] - lse_ref[b, h, lo:hi]).max() <= LSE_ABS
