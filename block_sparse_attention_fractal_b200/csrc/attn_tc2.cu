@@ -30,6 +30,7 @@
 // Every mbarrier wait is bounded; on expiry the CTA records BSA_ERR_TIMEOUT in
 // the workspace error word and leaves.
 #include <cmath>
+#include <cstdlib>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -112,7 +113,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
                                                                const int2* __restrict__ items, int* work,
                                                                float scale_log2, __nv_bfloat16* __restrict__ o,
                                                                float* __restrict__ lse, Ctrl* ctrl, Dims g,
-                                                               int items_per_bh, int n_items) {
+                                                               int items_per_bh, int n_items, int force_timeout) {
   constexpr int QB = 128 / BS;          // query blocks per tile
   constexpr int E = 128 / BS;           // list entries per KV tile
   constexpr int CH = D / 64;            // 64-column (128-byte) chunks of a row
@@ -163,6 +164,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = c.tmem_base;
+
+  // Test hook of the failure path: one bounded wait (2 ms) on an mbarrier
+  // that nothing arrives on, before any copy or MMA is issued; it records
+  // BSA_ERR_TIMEOUT and the CTA does no work.
+  if (force_timeout) {
+    if (tid == 0 && !mbar_wait_ns(&c.q_full, 0, 2ull * 1000ull * 1000ull, &ctrl->error, 0u)) timeout(ctrl, c, 1);
+    __syncthreads();
+  }
 
   uint32_t jbase = 0;  // KV tiles this CTA has run so far (phase counter of the K/V stages)
   uint32_t gbase[2] = {0u, 0u};  // KV tiles each softmax group has run so far
@@ -561,6 +570,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
   }
 }
 
+// BSA_TEST_FORCE_TIMEOUT=1 in the environment makes the attention kernel take
+// its bounded-wait failure path (tests of the device error word).
+int force_timeout_requested() {
+  const char* v = std::getenv("BSA_TEST_FORCE_TIMEOUT");
+  return (v != nullptr && v[0] == '1') ? 1 : 0;
+}
+
 int num_sms() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -586,7 +602,7 @@ cudaError_t launch_tc2(const Dims& g, const void* q, const void* k, const void* 
   const int grid = n_items < num_sms() ? n_items : num_sms();
   attn_tc2_kernel<D, BS, WITH_LSE><<<grid, kThreads, smem, st>>>(mq, mk, mv, kv_count, kv_idx, items, work,
                                                                  scale * 1.4426950408889634f, (__nv_bfloat16*)o, lse,
-                                                                 ctrl, g, items_per_bh, n_items);
+                                                                 ctrl, g, items_per_bh, n_items, force_timeout_requested());
   return cudaGetLastError();
 }
 

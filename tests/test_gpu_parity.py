@@ -234,3 +234,26 @@ def test_edge_shapes_mask_and_attention(bsa, w):
         mx, mean = compare_outputs(O[b, h, lo:hi], O_ref[b, h, lo:hi])
         assert mx <= MAX_ABS and mean <= MEAN_ABS, ((b, h, I), mx, mean)
         assert np.abs(lse[b, h, lo:hi] - lse_ref[b, h, lo:hi]).max() <= LSE_ABS
+
+
+def test_forced_timeout_is_reported_and_the_context_stays_usable(bsa, monkeypatch):
+    """The bounded-wait failure path: with the test hook set, the attention
+    kernel's first wait runs out (2 ms, nothing arrives), BSA_ERR_TIMEOUT comes
+    back through the error word, and the next call computes normally."""
+    w = small("forced_timeout", 1, 2, 16, 16, 2, 128, 64, 8, 0.2, seed=31)
+    q, k, v = synth.make_qkv(w)
+    plan = bsa.NablaAttention(_shape(bsa, w))
+    for src, dst in ((q, plan.q), (k, plan.k), (v, plan.v)):
+        bsa.reorder(plan.shape, src.cuda(), dst)
+    plan.mask_step(w.thr, w.sta)
+    monkeypatch.setenv("BSA_TEST_FORCE_TIMEOUT", "1")
+    plan.attention_step()
+    assert plan.status() == 5                     # BSA_ERR_TIMEOUT
+    monkeypatch.delenv("BSA_TEST_FORCE_TIMEOUT")
+    plan.attention_step()
+    torch.cuda.synchronize()
+    assert plan.status() == 0
+    keep = lists_to_keep(plan.kv_count, plan.kv_idx, plan.nb)
+    O_ref, _ = oracle.masked_attention(to64(plan.q), to64(plan.k), to64(plan.v), keep, w.N, w.block)
+    mx, mean = compare_outputs(to64(plan.o)[:, :, :w.N], O_ref[:, :, :w.N])
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean)
