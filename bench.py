@@ -99,17 +99,23 @@ class ClockSampler:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.first = threading.Event()
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            self.first.wait(timeout=5.0)   # sampling is live before the timed region starts
         except (OSError, ValueError):
             self.proc = None
+        self.t0 = time.monotonic()
         return self
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
+            self.first.set()
+        self.first.set()
 
     def __exit__(self, *exc):
+        self.t1 = time.monotonic()
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -121,7 +127,9 @@ class ClockSampler:
     def summary(self):
         sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
+        for t, line in self.lines:
+            if not (self.t0 <= t <= self.t1):      # only samples taken during the timed region
+                continue
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue

@@ -5,28 +5,29 @@
 // Work: the plan's 128-row query tiles (one block of 128, or two blocks of 64,
 // rows 0-63 and 64-127), fetched one at a time from a work counter in the
 // plan's order (longest first within each head).  A tile walks the union of
-// its KV lists in KV tiles of 128 keys (one entry of 128, or two of 64):
+// its KV lists in KV tiles of 128 keys (one entry of 128, or two of 64); KV
+// tile j belongs to softmax group w = j mod 2:
 //   S = Q K^T      tcgen05.mma (M=128, N=128), A = Q and B = K from shared
-//                  memory, S in TMEM
-//   softmax        two threads per query row, each on 64 keys of the KV tile:
+//                  memory, into TMEM S buffer w
+//   softmax        one thread per query row (group w: warps 4 + 4w .. 7 + 4w):
 //                  masks keys its row's block does not keep (and padding),
-//                  shares the tile max with its partner through shared memory,
-//                  keeps a running base-2 max (O rescaled only when it grows
-//                  by more than 8) and writes P = 2^(s - m) as bf16 over its
-//                  S columns in TMEM
-//   O += P V       tcgen05.mma with A = P from TMEM and B = V (MN-major) from
-//                  shared memory, O in TMEM
-// TMEM holds three S buffers and O (4 x 128 columns), so the S product of
-// KV tile j+2 is queued right behind the P.V product of tile j and the tensor
-// pipe never waits for the softmax of the tile in between; K has three and V
-// two stages in shared memory, each loaded by its own producer warp.  O is normalised by the sum of the bf16-rounded
+//                  keeps a running base-2 max (O_w rescaled only when it grows
+//                  by more than 8) and writes P = 2^(s - m) as bf16 into the
+//                  group's P tile in shared memory
+//   O_w += P V     tcgen05.mma with A = P and B = V (MN-major) from shared
+//                  memory, O_w in TMEM
+// TMEM holds S_0, S_1, O_0, O_1 (4 x 128 columns).  Because P does not live in
+// the S buffer, the S of the group's next tile is issued as soon as the group
+// has read its current S, and a softmax waits only for its own S; the P.V
+// products run beside it.  The epilogue merges the two groups' partial results
+// of each row exactly.  K and V have two stages in shared memory, each loaded
+// by its own producer warp.  O is normalised by the sum of the bf16-rounded
 // weights the P.V product uses (an exact convex combination of V rows up to
 // accumulation rounding); the LSE uses the fp32 sum of the unrounded ones.
 //
-// Roles: warps 0 and 2 issue TMA loads (Q and K; V), warp 1 issues MMAs (one
-// elected thread),
-// warps 4-11 run the softmax and the epilogue (warp w reads TMEM lanes
-// 32 (w mod 4) .. +31, keys 64 ((w - 4) div 4) .. +63 of each KV tile).
+// Roles: warps 0 and 2 issue TMA loads (Q and K; V), warp 3 issues the S
+// MMAs and warp 1 the P.V MMAs (one elected thread each), warps 4-11 run the
+// softmax and the epilogue (warp w reads TMEM lanes 32 (w mod 4) .. +31).
 // Every mbarrier wait is bounded; on expiry the CTA records BSA_ERR_TIMEOUT in
 // the workspace error word and leaves.
 #include <cmath>
@@ -51,23 +52,24 @@ constexpr uint32_t kGroupThreads = 128;   // threads of one softmax group
 constexpr uint64_t kWaitNs = 250ull * 1000ull * 1000ull;  // 250 ms: far beyond any legitimate wait
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 256;     // O_0 at 256, O_1 at 384; S_0 at 0, S_1 at 128
+constexpr uint32_t kPTile = 128u * 128u * 2u;  // bf16 P of one 128 x 128 tile in shared memory
 // One pair of scores in kPolyEvery takes the software exp2 (0 = none).
 constexpr int kPolyEvery = 0;
 
 struct Ctl {
   uint64_t q_full;
-  uint64_t k_full[3], k_empty[3], v_full[2], v_empty[2];
-  uint64_t s_full[2], p_full[2], pv_done[2];   // per softmax group
+  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
+  uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];   // per softmax group
   uint32_t tmem_base;
   int n_ent;
   int item;
   int abort;
-  float xm[2][128];        // [group][row]: running max at the epilogue
-  float xl[2][2][128];     // [group][sum kind][row]: row sums at the epilogue
   uint32_t bm[2][BSA_MAX_BLOCKS / 32];  // kept blocks of each query block of the tile
-  uint16_t ent[BSA_MAX_BLOCKS];         // union of the lists, ascending
-  uint8_t mem[BSA_MAX_BLOCKS];          // bit h: entry kept by query block h
+  // union of the lists, ascending: block index in bits 0-11, bit 12 + h set
+  // when query block h of the tile keeps the entry
+  uint16_t ent[BSA_MAX_BLOCKS];
 };
+constexpr uint16_t kEntBlock = 0x0FFFu;
 
 __device__ __forceinline__ void timeout(Ctrl* ctrl, Ctl& c, uint32_t site) {
   report_error(ctrl, kErrTimeout, blockIdx.x, threadIdx.x, site);
@@ -120,12 +122,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
   constexpr uint32_t kTile = 128u * D * 2u;
   constexpr uint32_t kChunk = 128u * 128u;  // bytes of one chunk of a 128-row tile
 
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = base;
-  uint8_t* sK = base + kTile;          // three stages
-  uint8_t* sV = base + 4 * kTile;      // two stages
-  Ctl& c = *reinterpret_cast<Ctl*>(base + 6 * kTile);
+  // 128-byte swizzled tiles need 1024-byte aligned shared memory; the layout
+  // fills the 227 KB of a CTA at D = 128, so there is no room to realign.
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_addr(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) report_error(ctrl, kErrLayout, blockIdx.x, 0u, 2u);
+    return;
+  }
+  uint8_t* sQ = smem_raw;
+  uint8_t* sK = sQ + kTile;            // two stages
+  uint8_t* sV = sQ + 3 * kTile;        // two stages
+  uint8_t* sP = sQ + 5 * kTile;        // P of each softmax group
+  Ctl& c = *reinterpret_cast<Ctl*>(sP + 2 * kPTile);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -135,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
 
   if (tid == 0) {
     mbar_init(&c.q_full, 1);
-    for (int s = 0; s < 3; ++s) {
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&c.k_full[s], 1);
       mbar_init(&c.k_empty[s], 1);
     }
@@ -145,6 +153,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(&c.s_full[w], 1);
+      mbar_init(&c.s_free[w], kGroupThreads);
       mbar_init(&c.p_full[w], kGroupThreads);
       mbar_init(&c.pv_done[w], 1);
     }
@@ -235,8 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
         while (u != 0u) {
           const int bit = __ffs(u) - 1;
           u &= u - 1u;
-          c.ent[pos] = (uint16_t)(wi * 32 + bit);
-          c.mem[pos] = (uint8_t)(((b0 >> bit) & 1u) | (((b1 >> bit) & 1u) << 1));
+          c.ent[pos] = (uint16_t)((wi * 32 + bit) | (((b0 >> bit) & 1u) << 12) | (((b1 >> bit) & 1u) << 13));
           ++pos;
         }
         off += __shfl_sync(0xffffffffu, incl, 31);
@@ -252,8 +260,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
 
     if (warp == 0 || warp == 2) {
       // ---------------------------------------------------------- TMA producers
-      // warp 0: Q, then K of every KV tile (three stages); warp 2: V (two
-      // stages), so a V wait never holds back the next K.
+      // warp 0: Q, then K of every KV tile; warp 2: V (two stages each), so
+      // a V wait never holds back the next K.
       const bool is_k = warp == 0;
       if (lane == 0 && n_tiles > 0) {
         if (is_k) {
@@ -276,14 +284,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
           for (int h = 0; h < 2; ++h) {
             if (E == 2) {
               const int idx = (2 * j + h < n_ent) ? 2 * j + h : 2 * j;
-              krow[h] = (int)c.ent[idx] * 64;
+              krow[h] = (int)(c.ent[idx] & kEntBlock) * 64;
             } else {
-              krow[h] = (int)c.ent[j] * 128 + 64 * h;
+              krow[h] = (int)(c.ent[j] & kEntBlock) * 128 + 64 * h;
             }
           }
           if (is_k) {
-            const uint32_t s = jg % 3;
-            if (jg >= 3 && !wait(&c.k_empty[s], ((jg - 3) / 3) & 1, ctrl)) { timeout(ctrl, c, 10); break; }
+            const uint32_t s = jg & 1;
+            if (jg >= 2 && !wait(&c.k_empty[s], ((jg - 2) >> 1) & 1, ctrl)) { timeout(ctrl, c, 10); break; }
             mbar_arrive_expect_tx(&c.k_full[s], kTile);
             uint8_t* dk = sK + s * kTile;
 #pragma unroll
@@ -304,52 +312,58 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
           }
         }
       }
-    } else if (warp == 1) {
-      // ---------------------------------------------------------- MMA issuer
+    } else if (warp == 3) {
+      // ---------------------------------------------------------- S issuer
       // KV tile j of the item belongs to softmax group w = j mod 2: its S goes
-      // to S buffer w (free once the group's previous P.V product, which read
-      // P from there, has completed) and its P.V product to O_w.
+      // to S buffer w as soon as the group has read its previous S (P lives
+      // in shared memory, so the S does not wait for any P.V product).
+      // Issued by its own thread, so an S never queues behind a wait for a P.
       if (lane == 0 && n_tiles > 0) {
         constexpr uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);
-        constexpr uint32_t idO = idesc_bf16_f32(128, D, 0, 1);
-        const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV);
-        bool ok = wait(&c.q_full, nq & 1, ctrl);
-        if (!ok) timeout(ctrl, c, 20);
-        auto issue_s = [&](int j) -> bool {
-          const uint32_t jg = jbase + j, ks = jg % 3;
-          const int w = j & 1;
-          const uint32_t gw = gbase[w] + (j >> 1);   // this group's tile count
-          if (!wait(&c.k_full[ks], (jg / 3) & 1, ctrl)) { timeout(ctrl, c, 21); return false; }
-          if (gw >= 1 && !wait(&c.pv_done[w], (gw - 1) & 1, ctrl)) { timeout(ctrl, c, 22); return false; }
-          tc_fence_after();
-          const uint32_t kbase = aK + ks * kTile;
+        const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK);
+        if (!wait(&c.q_full, nq & 1, ctrl)) {
+          timeout(ctrl, c, 20);
+        } else {
+          for (int j = 0; j < n_tiles; ++j) {
+            const uint32_t jg = jbase + j, ks = jg & 1;
+            const int w = j & 1;
+            const uint32_t gw = gbase[w] + (j >> 1);   // this group's tile count
+            if (!wait(&c.k_full[ks], (jg >> 1) & 1, ctrl)) { timeout(ctrl, c, 21); break; }
+            if (gw >= 1 && !wait(&c.s_free[w], (gw - 1) & 1, ctrl)) { timeout(ctrl, c, 22); break; }
+            tc_fence_after();
+            const uint32_t kbase = aK + ks * kTile;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
-            mma_ss(tmem + 128 * w, smem_desc_sw128(aQ + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024), idS,
-                   kk > 0);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
+              mma_ss(tmem + 128 * w, smem_desc_sw128(aQ + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024),
+                     idS, kk > 0);
+            }
+            mma_commit(&c.s_full[w]);
+            mma_commit(&c.k_empty[ks]);
           }
-          mma_commit(&c.s_full[w]);
-          mma_commit(&c.k_empty[ks]);
-          return true;
-        };
-        if (ok) ok = issue_s(0);
-        if (ok && n_tiles > 1) ok = issue_s(1);
-        for (int j = 0; ok && j < n_tiles; ++j) {
+        }
+      }
+    } else if (warp == 1) {
+      // ---------------------------------------------------------- P.V issuer
+      // O_w += P V for KV tile j (group w = j mod 2) once the group's softmax
+      // has written P to shared memory and V has landed.
+      if (lane == 0 && n_tiles > 0) {
+        constexpr uint32_t idO = idesc_bf16_f32(128, D, 0, 1);
+        const uint32_t aV = smem_addr(sV), aP = smem_addr(sP);
+        for (int j = 0; j < n_tiles; ++j) {
           const uint32_t jg = jbase + j, vs = jg & 1;
           const int w = j & 1;
           const uint32_t gw = gbase[w] + (j >> 1);
-          // S of tile j + 1 (the other group) as soon as its buffer is free:
-          // the P.V product of tile j - 1 was issued one iteration ago
-          if (j >= 1 && j + 1 < n_tiles && !(ok = issue_s(j + 1))) break;
           if (!wait(&c.p_full[w], gw & 1, ctrl)) { timeout(ctrl, c, 23); break; }
           if (!wait(&c.v_full[vs], (jg >> 1) & 1, ctrl)) { timeout(ctrl, c, 24); break; }
           tc_fence_after();
           const uint32_t vbase = aV + vs * kTile;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + kTmemO + 128 * w, tmem + 128 * w + kk * 8, smem_desc_sw128(vbase + kk * 2048, kChunk, 1024),
-                   idO, (j >= 2 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
+            mma_ss(tmem + kTmemO + 128 * w, smem_desc_sw128(aP + w * kPTile + off, 16, 1024),
+                   smem_desc_sw128(vbase + kk * 2048, kChunk, 1024), idO, (j >= 2 || kk > 0) ? 1u : 0u);
+          }
           mma_commit(&c.pv_done[w]);
           mma_commit(&c.v_empty[vs]);
         }
@@ -374,11 +388,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
           int key0, kept;
           if (E == 2) {
             const int idx = 2 * j + h;
-            kept = (idx < n_ent) ? ((c.mem[idx] >> half) & 1) : 0;
-            key0 = (idx < n_ent) ? (int)c.ent[idx] * 64 : 0;
+            kept = (idx < n_ent) ? ((c.ent[idx] >> (12 + half)) & 1) : 0;
+            key0 = (idx < n_ent) ? (int)(c.ent[idx] & kEntBlock) * 64 : 0;
           } else {
             kept = 1;
-            key0 = (int)c.ent[j] * 128 + 64 * h;
+            key0 = (int)(c.ent[j] & kEntBlock) * 128 + 64 * h;
           }
           lim[h] = kept ? max(0, min(64, g.N - key0)) : 0;
         }
@@ -413,12 +427,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
             mh[h] = mm;
           }
         }
+        // O_w and P buffer w are free once the group's previous P.V product
+        // has completed (normally long before: it was issued a tile ago).
+        if (gw >= 1 && !wait_warp(&c.pv_done[w], (gw - 1) & 1, ctrl)) { timeout(ctrl, c, 32); ok = false; break; }
+        tc_fence_after();
         const float mnew = fmaxf(m, fmaxf(mh[0], mh[1]) * scale_log2);
         // The running max moves only when it grows by more than 8 (a factor
         // 256 in p), or when it is set for the first time.  The O rescale uses
         // warp-collective TMEM accesses, so the whole warp takes it when any
         // lane needs it (lanes whose max did not move use alpha = 1).  O_w is
-        // stable: its last P.V product completed before this S was issued.
+        // stable: its last P.V product has completed (waited above).
         const bool grow = mnew > m + 8.0f;
         if (__any_sync(0xffffffffu, grow && m != -INFINITY)) {
           const float alpha = (grow && m != -INFINITY) ? ex2f(m - mnew) : 1.0f;
@@ -445,8 +463,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
         // unrounded ones.  Halves the row's query block does not keep cost
         // nothing.
         // Pass 2, 32 keys at a time (the next chunk's load in flight): their
-        // bf16 weights go to TMEM columns [16 c, 16 c + 16) of S buffer w,
-        // whose scores were read in this pass already.
+        // bf16 weights go to row r of the group's P tile in shared memory
+        // (K-major, 128-byte swizzle: 16-byte unit u of a row at u ^ (r mod 8)).
+        // S buffer w is released as soon as its last chunk has been read.
+        uint8_t* prow = sP + w * kPTile + r * 128;
         float rs[2] = {0.f, 0.f};
         float rx = 0.f;
         uint32_t sc[2][32];
@@ -455,7 +475,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
         for (int cch = 0; cch < 4; ++cch) {
           const int h = cch >> 1;
           tmem_wait_ld();
-          if (cch < 3) tmem_ld32(tS + 32 * (cch + 1), sc[(cch + 1) & 1]);
+          if (cch < 3) {
+            tmem_ld32(tS + 32 * (cch + 1), sc[(cch + 1) & 1]);
+          } else {
+            tc_fence_before();
+            mbar_arrive(&c.s_free[w]);
+          }
           const float* x = reinterpret_cast<const float*>(sc[cch & 1]);
           uint32_t pk[16];
           if (lim[h] > 0) {
@@ -482,12 +507,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
 #pragma unroll
             for (int i = 0; i < 16; ++i) pk[i] = 0u;
           }
-          tmem_st16(tS + 16 * cch, pk);
+          uint8_t* pc = prow + (cch >> 1) * kChunk;
+#pragma unroll
+          for (int u4 = 0; u4 < 4; ++u4) {
+            const int u = (cch & 1) * 4 + u4;
+            *reinterpret_cast<uint4*>(pc + ((u ^ (r & 7)) << 4)) =
+                make_uint4(pk[4 * u4], pk[4 * u4 + 1], pk[4 * u4 + 2], pk[4 * u4 + 3]);
+          }
         }
         l += rs[0] + rs[1];
         if (WITH_LSE) lx += rx;
-        tmem_wait_st();
-        tc_fence_before();
+        fence_proxy_async_smem();   // the P stores, visible to the tensor core
         mbar_arrive(&c.p_full[w]);
       }
 
@@ -501,16 +531,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
       if (ok && has0 && !wait_warp(&c.pv_done[0], (gbase[0] + cnt0 - 1) & 1, ctrl)) { timeout(ctrl, c, 31); ok = false; }
       if (ok && has1 && !wait_warp(&c.pv_done[1], (gbase[1] + cnt1 - 1) & 1, ctrl)) { timeout(ctrl, c, 31); ok = false; }
       tc_fence_after();
-      c.xm[w][r] = (mine > 0) ? m : -INFINITY;
-      c.xl[w][0][r] = l;
-      c.xl[w][1][r] = lx;
+      // The merge goes through the K stages: every S of the item has completed
+      // (its softmax ran) and the next item's K loads start after the item.
+      float* xm = reinterpret_cast<float*>(sK);   // [group][row]: running max
+      float* xl = xm + 2 * 128;                   // [group][sum kind][row]: row sums
+      xm[w * 128 + r] = (mine > 0) ? m : -INFINITY;
+      xl[(2 * w + 0) * 128 + r] = l;
+      xl[(2 * w + 1) * 128 + r] = lx;
       ok = pair_sync(q4, ok);
-      const float m0 = c.xm[0][r], m1 = c.xm[1][r];
+      const float m0 = xm[r], m1 = xm[128 + r];
       const float mt = fmaxf(m0, m1);
       const float a0 = (has0 && m0 != -INFINITY) ? ex2f(m0 - mt) : 0.f;
       const float a1 = (has1 && m1 != -INFINITY) ? ex2f(m1 - mt) : 0.f;
-      const float lt = c.xl[0][0][r] * a0 + c.xl[1][0][r] * a1;
-      const float lxt = c.xl[0][1][r] * a0 + c.xl[1][1][r] * a1;
+      const float lt = xl[r] * a0 + xl[2 * 128 + r] * a1;
+      const float lxt = xl[128 + r] * a0 + xl[3 * 128 + r] * a1;
       int grow;
       if (QB == 2) grow = qval[half] ? qblk[half] * 64 + (r & 63) : -1;
       else grow = qval[0] ? qblk[0] * 128 + r : -1;
@@ -550,6 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
       }
       if (WITH_LSE && w == 0 && store)
         lse[(size_t)bh * g.Npad + grow] = real ? (mt + __log2f(lxt)) * 0.69314718055994531f : 0.f;
+      fence_proxy_async_smem();   // the merge's accesses, ordered before the next K loads
     }
 
     tc_fence_before();
@@ -595,7 +630,8 @@ cudaError_t launch_tc2(const Dims& g, const void* q, const void* k, const void* 
     return cudaErrorInvalidValue;
   const int items_per_bh = (BS == 64) ? (g.nb + 1) / 2 : g.nb;
   const int n_items = (int)(bhs * items_per_bh);
-  const size_t smem = 6u * 128u * D * 2u + sizeof(Ctl) + 1024u;
+  const size_t smem = 5u * 128u * D * 2u + 2u * kPTile + sizeof(Ctl);
+  static_assert(5u * 128u * 128u * 2u + 2u * kPTile + sizeof(Ctl) <= 227u * 1024u, "shared memory layout");
   cudaError_t e =
       cudaFuncSetAttribute(attn_tc2_kernel<D, BS, WITH_LSE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

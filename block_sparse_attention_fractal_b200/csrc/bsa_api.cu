@@ -189,6 +189,7 @@ bsa_status bsa_check_device_status(void* workspace, bsa_stream_t stream) {
   if (word != 0u) {
     if (cudaMemset(workspace, 0, sizeof(Ctrl)) != cudaSuccess) return BSA_ERR_CUDA;
   }
+  if (word & bsa::kErrLayout) return BSA_ERR_CUDA;
   if (word & bsa::kErrTimeout) return BSA_ERR_TIMEOUT;
   if (word & (bsa::kErrIndex | bsa::kErrCount)) return BSA_ERR_DEVICE_INDEX;
   return BSA_OK;

@@ -15,6 +15,7 @@ enum : uint32_t {
   kErrIndex = 1u,    // a KV index outside [0, nb)
   kErrCount = 2u,    // a KV count outside [1, nb]
   kErrTimeout = 4u,  // a bounded wait expired
+  kErrLayout = 8u,   // shared memory not aligned as the kernel's layout needs
 };
 
 // Control block at the start of every workspace.

@@ -28,7 +28,8 @@
  *  - Argument errors are reported synchronously by the return value and
  *    launch nothing.  Errors found on the device (an out-of-range KV index or
  *    count, a bounded wait that expired) never trap: they set bits of an error
- *    word held in the workspace, which bsa_check_device_status reports.
+ *    word held in the workspace, which bsa_check_device_status reports
+ *    (BSA_ERR_CUDA for a shared-memory layout the device did not honour).
  */
 #ifndef BSA_H
 #define BSA_H
@@ -181,7 +182,9 @@ BSA_API bsa_status bsa_attn_fwd_baseline(const bsa_shape* s, const void* q, cons
  *   error_word_or_null: device, one uint32 (4-byte aligned), written at the end
  *       of the call with the device error bits of this call (0 = none,
  *       1 = a KV index outside [0, nb), 2 = a KV count outside [1, nb],
- *       4 = a bounded wait expired), or NULL to ignore them.
+ *       4 = a bounded wait expired, 8 = the attention kernel found its
+ *       shared memory not 1024-byte aligned and did nothing), or NULL to
+ *       ignore them.
  *
  * Limits and errors: a shape whose scratch exceeds BSA_NOALLOC_SCRATCH_BYTES
  * is refused with
