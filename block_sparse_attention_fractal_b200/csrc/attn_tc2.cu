@@ -320,7 +320,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
       // Issued by its own thread, so an S never queues behind a wait for a P.
       if (lane == 0 && n_tiles > 0) {
         constexpr uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);
-        const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK);
+        const uint64_t dQ = smem_desc_sw128(smem_addr(sQ), 16, 1024);
+        const uint32_t aK = smem_addr(sK);
         if (!wait(&c.q_full, nq & 1, ctrl)) {
           timeout(ctrl, c, 20);
         } else {
@@ -331,12 +332,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
             if (!wait(&c.k_full[ks], (jg >> 1) & 1, ctrl)) { timeout(ctrl, c, 21); break; }
             if (gw >= 1 && !wait(&c.s_free[w], (gw - 1) & 1, ctrl)) { timeout(ctrl, c, 22); break; }
             tc_fence_after();
-            const uint32_t kbase = aK + ks * kTile;
+            // descriptors built once per tile: the issuing thread shares its
+            // sub-partition with two softmax warps, so each MMA costs it only
+            // the two descriptor adds
+            const uint64_t dK = smem_desc_sw128(aK + ks * kTile, 16, 1024);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
-              mma_ss(tmem + 128 * w, smem_desc_sw128(aQ + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024),
-                     idS, kk > 0);
+              mma_ss(tmem + 128 * w, smem_desc_add(dQ, off), smem_desc_add(dK, off), idS, kk > 0);
             }
             mma_commit(&c.s_full[w]);
             mma_commit(&c.k_empty[ks]);
@@ -357,12 +360,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
           if (!wait(&c.p_full[w], gw & 1, ctrl)) { timeout(ctrl, c, 23); break; }
           if (!wait(&c.v_full[vs], (jg >> 1) & 1, ctrl)) { timeout(ctrl, c, 24); break; }
           tc_fence_after();
-          const uint32_t vbase = aV + vs * kTile;
+          const uint64_t dP = smem_desc_sw128(aP + w * kPTile, 16, 1024);
+          const uint64_t dV = smem_desc_sw128(aV + vs * kTile, kChunk, 1024);
+          const uint32_t acc0 = (j >= 2) ? 1u : 0u;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
-            mma_ss(tmem + kTmemO + 128 * w, smem_desc_sw128(aP + w * kPTile + off, 16, 1024),
-                   smem_desc_sw128(vbase + kk * 2048, kChunk, 1024), idO, (j >= 2 || kk > 0) ? 1u : 0u);
+            mma_ss(tmem + kTmemO + 128 * w, smem_desc_add(dP, off), smem_desc_add(dV, kk * 2048), idO,
+                   kk > 0 ? 1u : acc0);
           }
           mma_commit(&c.pv_done[w]);
           mma_commit(&c.v_empty[vs]);

@@ -147,6 +147,13 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// The descriptor of a matrix `bytes` further on (a multiple of 16): the start
+// address field holds address / 16 in 14 bits, and shared-memory addresses
+// stay below 256 KB, so the sum never carries out of the field.
+__device__ __forceinline__ uint64_t smem_desc_add(uint64_t desc, uint32_t bytes) {
+  return desc + (uint64_t)(bytes >> 4);
+}
+
 // Instruction descriptor of kind::f16 with bf16 inputs and fp32 accumulation.
 //   a_mn / b_mn: operand stored MN-major (1) instead of K-major (0).
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn) {
