@@ -474,6 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
         uint8_t* prow = sP + w * kPTile + r * 128;
         float rs[2] = {0.f, 0.f};
         float rx = 0.f;
+        const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(nm, nm);
         uint32_t sc[2][32];
         tmem_ld32(tS, sc[0]);
 #pragma unroll
@@ -491,7 +492,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
           if (lim[h] > 0) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const float y0 = fmaf(x[2 * i], scale_log2, nm), y1 = fmaf(x[2 * i + 1], scale_log2, nm);
+              // both arguments in one fma.rn.f32x2 (half the issue slots)
+              const float2 yy = ffma2(make_float2(x[2 * i], x[2 * i + 1]), sc2, nm2);
+              const float y0 = yy.x, y1 = yy.y;
               float2 p;
               if (kPolyEvery > 0 && (i % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
                 p = exp2_poly2(make_float2(y0, y1));
