@@ -257,3 +257,46 @@ def test_forced_timeout_is_reported_and_the_context_stays_usable(bsa, monkeypatc
     O_ref, _ = oracle.masked_attention(to64(plan.q), to64(plan.k), to64(plan.v), keep, w.N, w.block)
     mx, mean = compare_outputs(to64(plan.o)[:, :, :w.N], O_ref[:, :, :w.N])
     assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean)
+
+
+# Keys whose scale grows along the key blocks: each row's running max keeps
+# rising as the kernel walks its ascending list, so the lazy rescale of O (a
+# max that grows by more than 8 in log2 units) runs many times per row, in
+# both tile layouts (two 64-token blocks per 128-row tile, and 128-token
+# blocks).
+GROWTH = [
+    small("growth64", 1, 3, 16, 24, 2, 128, 64, 8, 0.0, seed=31),
+    small("growth128_d64", 1, 2, 16, 32, 2, 64, 128, 8, 0.0, seed=32),
+]
+
+
+@pytest.mark.parametrize("w", GROWTH, ids=lambda w: w.name)
+def test_running_max_growth_rescales(bsa, w):
+    q, k, v = synth.make_qkv(w)
+    plan = bsa.NablaAttention(_shape(bsa, w), with_lse=True)
+    for src, dst in ((q, plan.q), (k, plan.k), (v, plan.v)):
+        bsa.reorder(plan.shape, src.cuda(), dst)
+    nb = plan.nb
+    blk = torch.arange(plan.k.shape[2], device=plan.k.device) // w.block
+    ramp = 1.0 + 2.0 * blk.float() / nb
+    plan.k.copy_((plan.k.float() * ramp[None, None, :, None]).to(torch.bfloat16))
+    q64, k64, v64 = to64(plan.q), to64(plan.k), to64(plan.v)
+    # the case is meaningful only if many rows' max grows by more than 8
+    # (log2 units) after their first key block
+    s = np.einsum("bhnd,bhmd->bhnm", q64[:, :, :w.N], k64[:, :, :w.N]) / math.sqrt(w.d) / math.log(2.0)
+    first = s[..., :w.block].max(axis=-1)
+    assert np.mean(s.max(axis=-1) - first > 8.0) > 0.2
+    for dens in (1.0, 0.4):
+        cnt, idx = synth.random_block_lists(w.B, w.heads, nb, dens, seed=9)
+        plan.kv_count.copy_(cnt)
+        plan.kv_idx.copy_(idx)
+        plan.attention_step()
+        torch.cuda.synchronize()
+        assert plan.status() == 0
+        keep = lists_to_keep(cnt, idx, nb)
+        O_ref, lse_ref = oracle.masked_attention(q64, k64, v64, keep, w.N, w.block)
+        got, want = to64(plan.o)[:, :, :w.N], O_ref[:, :, :w.N]
+        assert np.all(np.abs(got - want) <= MAX_ABS + _half_ulp_bf16(want)), dens
+        assert np.abs(got - want).mean() <= MEAN_ABS, dens
+        lse = to64(plan.lse)[:, :, :w.N]
+        assert np.abs(lse - lse_ref[:, :, :w.N]).max() <= LSE_ABS * max(1.0, np.abs(lse_ref).max() / 16.0), dens
