@@ -187,7 +187,7 @@ def oracle_step_estimate(w, q, k, v, kv_count, kv_idx, budget_s=15.0, seed=0):
     # attention: query blocks of head 0, then of the next heads, in random
     # order until the budget is used (only the attention time is counted)
     t_spent, done, heads_used = 0.0, 0, 0
-    for hd in range(w.heads):
+    for hd in range(min(w.heads, kv_count.shape[1])):   # the heads whose lists were given
         if hd == 0:
             yq, ykk = y, yk
         else:
