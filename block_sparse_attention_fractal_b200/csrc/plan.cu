@@ -39,6 +39,11 @@ static_assert(kMatchThreads >= BSA_MAX_BLOCKS, "match_kernel handles one block r
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// match_kernel keeps the weights transposed in shared memory, [offset][row]
+// with this row stride (uint16 units): a warp's 32 rows read 32 neighbouring
+// entries of one offset, free of bank conflicts.
+__host__ __device__ inline int wts_stride(int nb) { return nb + (nb & 1) + 2; }
+
 // Plan region of the workspace: items | weights | counts (the last two only
 // with 64-token blocks).
 struct PlanRegion {
@@ -123,7 +128,7 @@ __global__ void __launch_bounds__(kMatchThreads) match_kernel(const int32_t* __r
   __shared__ int bin[BSA_MAX_BLOCKS];      // tiles per union size (bin nb - size), then their first slot
   __shared__ int wsum[32];
   __shared__ int n_unm;
-  extern __shared__ uint16_t wts[];   // [nb][kWindow] (QB == 2 only)
+  extern __shared__ uint16_t wts[];   // [kWindow][S]: weight of rows (r, r + off) at (off - 1) * S + r (QB == 2)
   const int nb = g.nb;
   const size_t bh = blockIdx.x;
   const int n_items = (nb + QB - 1) / QB;
@@ -140,10 +145,10 @@ __global__ void __launch_bounds__(kMatchThreads) match_kernel(const int32_t* __r
     cnt_s[r] = c;
     partner[r] = (QB == 2) ? -1 : r;
   }
+  const int S = wts_stride(nb);
   if (QB == 2) {
-    const uint4* src = reinterpret_cast<const uint4*>(weights + bh * nb * kWindow);
-    uint4* dst = reinterpret_cast<uint4*>(wts);
-    for (int i = threadIdx.x; i < nb * kWindow * 2 / 16; i += kMatchThreads) dst[i] = src[i];
+    const uint16_t* src = weights + bh * nb * kWindow;
+    for (int i = threadIdx.x; i < nb * kWindow; i += kMatchThreads) wts[(i % kWindow) * S + i / kWindow] = src[i];
   }
   __syncthreads();
 
@@ -156,11 +161,11 @@ __global__ void __launch_bounds__(kMatchThreads) match_kernel(const int32_t* __r
             const int lo = r - off, hi = r + off;
             // ties keep the nearer, then the lower, index
             if (lo >= 0 && partner[lo] < 0) {
-              const int w = wts[lo * kWindow + off - 1];
+              const int w = wts[(off - 1) * S + lo];
               if (w > bestw) { bestw = w; best = lo; }
             }
             if (hi < nb && partner[hi] < 0) {
-              const int w = wts[r * kWindow + off - 1];
+              const int w = wts[(off - 1) * S + r];
               if (w > bestw) { bestw = w; best = hi; }
             }
           }
@@ -226,7 +231,7 @@ __global__ void __launch_bounds__(kMatchThreads) match_kernel(const int32_t* __r
         int u = cnt_s[r];
         if (QB == 2 && p != r) {
           u += cnt_s[p];
-          if (p - r <= kWindow) u -= wts[r * kWindow + (p - r) - 1];
+          if (p - r <= kWindow) u -= wts[(p - r - 1) * S + r];
         }
         usz = min(max(u, 1), nb);
         ur = r;
@@ -285,7 +290,7 @@ cudaError_t launch_plan(const Dims& g, const int32_t* kv_count, const int32_t* k
     overlap_kernel<<<grid, kOverlapThreads, 0, st>>>(kv_count, kv_idx, g, weights, counts);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const size_t smem = (size_t)g.nb * kWindow * sizeof(uint16_t);
+    const size_t smem = (size_t)wts_stride(g.nb) * kWindow * sizeof(uint16_t);
     e = cudaFuncSetAttribute(match_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     match_kernel<2><<<bh, kMatchThreads, smem, st>>>(kv_count, weights, counts, g, items,
