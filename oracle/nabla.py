@@ -13,8 +13,7 @@ the exact float64 values of the bf16 inputs.  Library primitives (a matmul, a
 stable argsort, a cumulative sum, exp) serve as single steps; there is no
 blocking or fusion beyond what each definition states.
 
-Readings taken where the page is silent or garbled (each is listed in
-the design doc too):
+Readings taken where the page is silent or garbled:
 
 * fractal order: one level of P x P grouping, time outermost, patches in
   row-major order, tokens inside a patch in row-major order; edge patches are
@@ -33,10 +32,14 @@ the design doc too):
 
 Parity pins (tests/test_oracle_pins.py): a hand-derived permutation, the
 bijection, closed forms for pooling and the reduced map, brute force over all
-subsets for the CDF rule, the aligned tile grid for STA, and a library
+subsets for the CDF rule, hand-worked threshold rows including exact and
+near ties at the boundary, a hand-derived tile grid for STA on a ragged grid
+(blocks straddling patches and frames) and on an aligned one, and a library
 attention (torch scaled_dot_product_attention in float64) for the masked
-softmax.  The end-to-end combination beyond these invariants is
-"parity unpinned": the pages print no worked example.
+softmax.  The pages print no worked example of the whole path; each
+function is pinned on its own, and the composition is pinned at thr = 0,
+where reorder -> mask -> attention -> inverse reorder must equal dense
+attention on the model-order tokens.
 """
 from __future__ import annotations
 

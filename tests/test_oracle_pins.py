@@ -185,6 +185,56 @@ def test_cdf_flags_blocks_near_the_threshold():
     assert amb[0, 1] and not amb[0, 0]
 
 
+def test_cdf_flags_an_exact_tie_at_the_boundary():
+    # target 0.65: ranked 0.4 (J0), 0.3 (J1), 0.3 (J2); the tie J1/J2 decides
+    # which block is the last kept one, so both are ambiguous; J0 is not.
+    A = np.array([[0.4, 0.3, 0.3]])
+    keep, amb = oracle.cdf_keep(A, 0.35)
+    assert keep[0].tolist() == [True, True, False]
+    assert amb[0].tolist() == [False, True, True]
+
+
+def test_cdf_does_not_flag_a_tie_away_from_the_boundary():
+    # target 0.8: ranked 0.3 (J0), 0.3 (J1), 0.25 (J2), 0.15 (J3); the tie J0/J1
+    # lies inside the kept set and the boundary block J2 has no near-equal peer.
+    A = np.array([[0.3, 0.3, 0.25, 0.15]])
+    keep, amb = oracle.cdf_keep(A, 0.2)
+    assert keep[0].tolist() == [True, True, True, False]
+    assert not amb.any()
+
+
+def test_cdf_near_tie_window_is_relative_1e9():
+    # the boundary block J1 and J2 differ by 2e-12 relative: flagged; by 2e-6: not.
+    for rel, flagged in ((1e-12, True), (1e-6, False)):
+        A = np.array([[0.4, 0.3 * (1 + rel), 0.3 * (1 - rel)]])
+        keep, amb = oracle.cdf_keep(A, 0.35)
+        assert keep[0].tolist() == [True, True, False]
+        assert amb[0].tolist() == [False, flagged, flagged], rel
+
+
+def test_pins_catch_a_dropped_tie_rule(monkeypatch):
+    orig = nabla.cdf_keep
+
+    def no_tie_rule(A, thr):   # only the prefix-mass rule flags blocks
+        keep, _ = orig(A, thr)
+        amb = np.zeros_like(keep)
+        flat_a, flat_m = A.reshape(-1, A.shape[-1]), amb.reshape(-1, A.shape[-1])
+        for r in range(flat_a.shape[0]):
+            order = np.argsort(-flat_a[r], kind="stable")
+            before = np.concatenate([[0.0], np.cumsum(flat_a[r][order])[:-1]])
+            flat_m[r, order[np.abs(before - (1.0 - thr)) <= nabla.AMBIGUITY_MASS]] = True
+        return keep, amb
+    monkeypatch.setattr(oracle, "cdf_keep", no_tie_rule)
+    with pytest.raises(AssertionError):
+        test_cdf_flags_an_exact_tie_at_the_boundary()
+
+
+def test_pins_catch_a_tie_window_that_is_too_wide(monkeypatch):
+    monkeypatch.setattr(nabla, "AMBIGUITY_TIE_REL", 0.5)
+    with pytest.raises(AssertionError):
+        test_cdf_does_not_flag_a_tie_away_from_the_boundary()
+
+
 # ----------------------------------------------------------------- STA
 
 def test_sta_on_aligned_grid_is_the_tile_window():
@@ -203,6 +253,80 @@ def test_sta_on_aligned_grid_is_the_tile_window():
     # an interior block sees exactly 27 tiles; a corner block 8
     assert m[1 * nPr * nPc + 1 * nPc + 1].sum() == 27
     assert m[0].sum() == 2 * 2 * 2
+
+
+def _sta_golden(golden_dir):
+    return _read_golden(os.path.join(golden_dir, "sta_tiles_T2_H5_W7_P4_bs8.txt"))
+
+
+def _sta_golden_mismatches(g):
+    """Differences between the oracle's tiles / windows and the hand-derived
+    file (empty when they agree).  Looks the functions up on the module at
+    call time, so a planted mistake is seen."""
+    T, H, W, P, bs = g["T"][0], g["H"][0], g["W"][0], g["P"][0], g["block"][0]
+    bad = []
+    tiles = nabla.block_tiles(T, H, W, P, bs)
+    nb = tiles.shape[0]
+    if nb != len(g["first"]):
+        return [("nb", nb)]
+    for I in range(nb):
+        if tiles[I].tolist() != g[f"tile{I}"]:
+            bad.append(("tile", I, tiles[I].tolist(), g[f"tile{I}"]))
+    for half, key in (((0, 0, 0), "w000"), ((1, 0, 0), "w100"), ((0, 0, 1), "w001")):
+        m = nabla.sta_mask(T, H, W, P, bs, half)
+        for I in range(nb):
+            if np.nonzero(m[I])[0].tolist() != g[f"{key}_{I}"]:
+                bad.append((key, I, np.nonzero(m[I])[0].tolist(), g[f"{key}_{I}"]))
+    return bad
+
+
+def test_sta_on_ragged_grid_matches_hand_derivation(golden_dir):
+    g = _sta_golden(golden_dir)
+    o = oracle.fractal_order(g["T"][0], g["H"][0], g["W"][0], g["P"][0])
+    # the first token of each block is the position the file names
+    assert [8 * I for I in range(len(g["first"]))] == g["first"]
+    assert o.size == 70
+    assert _sta_golden_mismatches(g) == []
+
+
+def _tiles_of(token_of_block):
+    """block_tiles with another choice of the block's representative token."""
+    def tiles(T, H, W, P, block):
+        N = T * H * W
+        order = nabla.fractal_order(T, H, W, P)
+        nb = nabla.num_blocks(N, block)
+        out = np.zeros((nb, 3), dtype=np.int64)
+        for I in range(nb):
+            n = int(token_of_block(order, I, block, N))
+            t, rem = divmod(n, H * W)
+            h, w = divmod(rem, W)
+            out[I] = (t, h // P, w // P)
+        return out
+    return tiles
+
+
+@pytest.mark.parametrize("mistake", ["last_token", "majority_tile", "position_as_token"])
+def test_pins_catch_a_wrong_block_tile(monkeypatch, golden_dir, mistake):
+    if mistake == "last_token":
+        bad = _tiles_of(lambda order, I, bs, N: order[min((I + 1) * bs, N) - 1])
+    elif mistake == "position_as_token":
+        bad = _tiles_of(lambda order, I, bs, N: I * bs)
+    else:
+        def bad(T, H, W, P, block):
+            N = T * H * W
+            order = nabla.fractal_order(T, H, W, P)
+            nb = nabla.num_blocks(N, block)
+            out = np.zeros((nb, 3), dtype=np.int64)
+            for I in range(nb):
+                toks = order[I * block:min((I + 1) * block, N)]
+                t = toks // (H * W)
+                h = (toks % (H * W)) // W
+                w = toks % W
+                keys, counts = np.unique(np.stack([t, h // P, w // P], 1), axis=0, return_counts=True)
+                out[I] = keys[np.argmax(counts)]
+            return out
+    monkeypatch.setattr(nabla, "block_tiles", bad)
+    assert _sta_golden_mismatches(_sta_golden(golden_dir)) != []
 
 
 def test_hybrid_mask_contains_both_parts():
