@@ -147,6 +147,15 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def lists_to_keep(kv_count: np.ndarray, kv_idx: np.ndarray, nb: int) -> np.ndarray:
+    """KV lists -> bool block mask [B, heads, nb, nb] (entries past the count ignored)."""
+    keep = np.zeros(kv_count.shape + (nb,), dtype=bool)
+    flat_k, flat_c, flat_i = keep.reshape(-1, nb), kv_count.reshape(-1), kv_idx.reshape(-1, kv_idx.shape[-1])
+    for r in range(flat_c.size):
+        flat_k[r, flat_i[r, :flat_c[r]]] = True
+    return keep
+
+
 def max_over_ranks(value: float, dist, device) -> float:
     """The largest `value` over all ranks (the value itself without a process group)."""
     if dist is None:
@@ -164,96 +173,127 @@ def aggregate(per_rank_ms, per_rank_flops):
 
 # ------------------------------------------------------------------ oracle timing
 
-def oracle_step_estimate(w, q, k, v, kv_count, kv_idx, budget_s=15.0, seed=0):
-    """Times the fp64 oracle on a bounded sample of one step of workload `w`
-    and extrapolates to a whole step.  Returns (seconds per step, description)."""
-    import oracle
-    rng = np.random.default_rng(seed)
-    nb = w.nb
-    t0 = time.perf_counter()
-    # reorder: time a slice of the heads and scale
-    q64 = q[:, :, :1].to(torch.float64).numpy()
-    t = time.perf_counter()
-    y = oracle.reorder(q64, w.T, w.H, w.W, w.patch, w.block)
-    t_reorder = (time.perf_counter() - t) * w.heads * 3
-    # mask: one head in full
-    k64 = k[:, :, :1].to(torch.float64).numpy()
-    t = time.perf_counter()
-    yk = oracle.reorder(k64, w.T, w.H, w.W, w.patch, w.block)
-    t_mask_reorder = time.perf_counter() - t
-    t = time.perf_counter()
-    keep1, _ = oracle.block_mask(y, yk, w.T, w.H, w.W, w.patch, w.block, w.thr, w.sta) if not w.iid else (None, None)
-    t_mask = (time.perf_counter() - t) * w.heads * w.B
-    # attention: query blocks of head 0, then of the next heads, in random
-    # order until the budget is used (only the attention time is counted)
-    t_spent, done, heads_used = 0.0, 0, 0
-    for hd in range(min(w.heads, kv_count.shape[1])):   # the heads whose lists were given
-        if hd == 0:
-            yq, ykk = y, yk
+def block_flops(w, count: int) -> float:
+    """Effective FLOPs of one query block that keeps `count` KV blocks: its share
+    of 4 * N^2 * d (the metric's formula, summed over all blocks of a call)."""
+    return 4.0 * (w.N / w.nb) ** 2 * w.d * count
+
+
+def oracle_head_path(pool, w, b, h, blocks, counts):
+    """One sampled step of the fp64 oracle on the host cores: the whole path of
+    head (b, h) -- reorder of its Q, K and V, its block mask (adaptive
+    workloads), the attention of the query blocks `blocks` and the inverse
+    reorder of its output -- each stage spread over the pool.  Returns (wall
+    seconds, effective FLOPs of the attention done)."""
+    t = pool.reorder([(b, h)])
+    if not w.iid:
+        _, _, tm = pool.masks([(b, h)])
+        t += tm
+    t += pool.attention(b, h, blocks)
+    t += pool.inverse()
+    return t, sum(block_flops(w, int(counts[b, h, I])) for I in blocks)
+
+
+def oracle_block_seconds(pool, w):
+    """Wall seconds of one query block's oracle attention (a probe: one block
+    per worker, in parallel), with Q, K, V of head (0, 0) reordered first."""
+    pool.reorder([(0, 0)])
+    n = min(w.nb, pool.workers)
+    blocks = list(range(0, w.nb, max(1, w.nb // n)))[:n]
+    pool.attention(0, 0, blocks, chunk=1)          # first touch of the mapped inputs in every worker
+    return pool.attention(0, 0, blocks, chunk=1)
+
+
+def sample_blocks(w, workers, t_block, budget_s):
+    """The query blocks of a head that one sampled step runs: all of them when
+    the estimated wall time fits `budget_s`, else every k-th (first block 0,
+    the ragged last block always included)."""
+    fit = max(1, int(budget_s * workers / max(t_block, 1e-6)))
+    k = max(1, -(-w.nb // fit))
+    blocks = list(range(0, w.nb, k))
+    if blocks[-1] != w.nb - 1:
+        blocks.append(w.nb - 1)
+    return blocks, k
+
+
+def oracle_baseline(w, q, k, v, gpu_keep, budget_s=15.0):
+    """The GPU arm's ``cpu_baseline``: the fp64 oracle on the host cores.
+
+    First the oracle's block mask of every head (its ambiguous blocks counted,
+    and compared with the GPU's mask ``gpu_keep``), then one sampled step:
+    the whole path of head (0, 0) with as many query blocks as `budget_s` of
+    wall time allows.  Returns (cpu_baseline dict, mask report dict)."""
+    from oracle.parallel import OraclePool
+    with OraclePool(w, q, k, v) as pool:
+        report = {}
+        if not w.iid:
+            pool.reorder(pool.pairs(), (0, 1))
+            keep, amb, _ = pool.masks(pool.pairs())
+            report = {"ambiguous_blocks": int(amb.sum()),
+                      "mask_mismatch_unambiguous": int(((keep != gpu_keep) & ~amb).sum()),
+                      "oracle_density": float(keep.mean())}
         else:
-            yq = oracle.reorder(q[:, :, hd:hd + 1].to(torch.float64).numpy(), w.T, w.H, w.W, w.patch, w.block)
-            ykk = oracle.reorder(k[:, :, hd:hd + 1].to(torch.float64).numpy(), w.T, w.H, w.W, w.patch, w.block)
-        yv = oracle.reorder(v[:, :, hd:hd + 1].to(torch.float64).numpy(), w.T, w.H, w.W, w.patch, w.block)
-        keep = oracle.lists_to_mask(kv_count[:, hd:hd + 1].numpy(), kv_idx[:, hd:hd + 1].numpy(), nb)
-        heads_used += 1
-        t = time.perf_counter()
-        for I in rng.permutation(nb):
-            oracle.masked_attention(yq, ykk, yv, keep, w.N, w.block, blocks=[(0, 0, int(I))])
-            done += 1
-            if t_spent + (time.perf_counter() - t) > budget_s * 0.6:
-                break
-        t_spent += time.perf_counter() - t
-        if t_spent > budget_s * 0.6:
-            break
-    t_attn = t_spent / done * nb * w.heads * w.B
-    t_inverse = t_reorder / 3.0
-    total = t_reorder + t_mask + t_attn + t_inverse
-    desc = (f"fp64 oracle: reorder of 1 head x3 tensors, mask of 1 head in full, attention of {done} of "
-            f"{nb * w.heads * w.B} query blocks ({heads_used} heads); extrapolated linearly to one whole step "
-            f"(wall {time.perf_counter() - t0:.1f} s)")
-    return total, desc
-
-
-def cpu_threads():
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
-        return max(n) if n else 1
-    except Exception:
-        return os.cpu_count() or 1
+            pool.set_keep(gpu_keep)
+        counts = gpu_keep.sum(-1)
+        t_block = oracle_block_seconds(pool, w)
+        blocks, kstride = sample_blocks(w, pool.workers, t_block, budget_s)
+        secs, flops = oracle_head_path(pool, w, 0, 0, blocks, counts)
+        desc = (f"fp64 oracle, {pool.workers} host processes: the whole path of head 0 of {w.heads} (reorder Q, K, V; "
+                f"{'block mask; ' if not w.iid else ''}attention of {len(blocks)} of {w.nb} query blocks"
+                f"{'' if kstride == 1 else f' (every {kstride}th)'}; inverse reorder), {secs:.1f} s wall; "
+                f"value = effective FLOPs of those blocks / that time")
+        cpu = {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": pool.workers, "kind": "oracle",
+               "sample": desc}
+    return cpu, report
 
 
 # ------------------------------------------------------------------ main legs
 
 def run_reference(args, w):
-    """--impl reference: the fp64 oracle on host cores, a bounded sample per step."""
+    """--impl reference: the fp64 oracle on the host cores.  Untimed set-up: the
+    oracle's block mask of every head (so the workload and its density are the
+    GPU arm's).  Each step then runs the whole path of one head (heads in
+    turn), with as many of its query blocks as the step's time budget allows;
+    value = effective FLOPs done / wall time of the timed steps."""
     import block_sparse_attention_fractal_b200.synth as synth
+    from oracle.parallel import OraclePool
     q, k, v = synth.make_qkv(w)
-    if w.iid:
-        cnt, idx = synth.random_block_lists(w.B, w.heads, w.nb, 0.2, w.seed)
-    else:
-        import oracle
-        # the oracle's own mask for head 0 decides the sampled attention work
-        y = oracle.reorder(q[:, :, :1].double().numpy(), w.T, w.H, w.W, w.patch, w.block)
-        yk = oracle.reorder(k[:, :, :1].double().numpy(), w.T, w.H, w.W, w.patch, w.block)
-        keep, _ = oracle.block_mask(y, yk, w.T, w.H, w.W, w.patch, w.block, w.thr, w.sta)
-        c, i = oracle.mask_to_lists(keep)
-        cnt, idx = torch.from_numpy(c), torch.from_numpy(i)
-    dens = float(cnt[:, :1].sum()) / (w.B * 1 * w.nb * w.nb)
-    flops = 4.0 * w.N * w.N * w.d * w.heads * w.B * dens
-    budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
-    times = []
-    for s in range(args.warmup + args.steps):
-        t, desc = oracle_step_estimate(w, q, k, v, cnt, idx, budget_s=budget, seed=s)
-        if s >= args.warmup:
-            times.append(t)
-    step_s = statistics.mean(times)
-    value = flops / step_s / 1e12
+    with OraclePool(w, q, k, v) as pool:
+        if w.iid:
+            dens_req = args.density if args.density is not None else 0.2
+            cnt, idx = synth.random_block_lists(w.B, w.heads, w.nb, dens_req, w.seed)
+            keep = np.zeros((w.B, w.heads, w.nb, w.nb), dtype=bool)
+            c, ix = cnt.numpy(), idx.numpy()
+            for b in range(w.B):
+                for h in range(w.heads):
+                    for I in range(w.nb):
+                        keep[b, h, I, ix[b, h, I, :c[b, h, I]]] = True
+            pool.set_keep(keep)
+        else:
+            pool.reorder(pool.pairs(), (0, 1))
+            keep, _, _ = pool.masks(pool.pairs())
+        dens = float(keep.mean())
+        counts = keep.sum(-1)
+        budget = max(1.5, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+        t_block = oracle_block_seconds(pool, w)
+        blocks, kstride = sample_blocks(w, pool.workers, t_block, budget)
+        times, flops = [], []
+        for s in range(args.warmup + args.steps):
+            b, h = (s // w.heads) % w.B, s % w.heads
+            t, f = oracle_head_path(pool, w, b, h, blocks, counts)
+            if s >= args.warmup:
+                times.append(t)
+                flops.append(f)
+        workers = pool.workers
+    value = sum(flops) / sum(times) / 1e12
+    desc = (f"fp64 oracle, {workers} host processes; each step is the whole path of one head (heads in turn): "
+            f"reorder Q, K, V; {'block mask; ' if not w.iid else ''}attention of {len(blocks)} of {w.nb} query blocks"
+            f"{'' if kstride == 1 else f' (every {kstride}th)'}; inverse reorder")
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "impl": "reference", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "density": dens},
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.mean(times) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "density": dens, "sample": desc},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": workers, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -294,7 +334,7 @@ def run_ours(args, w, rank, world, dist):
             plan.mask_step(w.thr, w.sta)
         plan.join_side()
         if e: e[2].record(stream)
-        plan.attention_step()
+        plan.attention_step(baseline=args.baseline_kernel)
         if e: e[3].record(stream)
         bsa.inverse_reorder(shape, plan.o, out)
         if e:
@@ -407,12 +447,10 @@ def run_ours(args, w, rank, world, dist):
     mask_ms = float(br[1])
     # the reorder_qk part moves Q and K (V's reorder overlaps the mask stage on a side stream)
     reorder_bytes = 2 * 2 * (w.B * w.heads * w.N * w.d * 2) + 2 * 2 * w.B * w.heads * (plan.Npad - w.N) * w.d
-    cpu = None
-    if args.cpu_baseline:
-        cnt_cpu, idx_cpu = plan.kv_count.cpu(), plan.kv_idx.cpu()
-        t_cpu, desc = oracle_step_estimate(w, q_h, k_h, v_h, cnt_cpu, idx_cpu, budget_s=args.cpu_budget)
-        cpu = {"value": flops_step / t_cpu / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
-               "sample": desc}
+    cpu, mask_report = None, {}
+    if args.cpu_baseline and world == 1:
+        gpu_keep = lists_to_keep(plan.kv_count.cpu().numpy(), plan.kv_idx.cpu().numpy(), plan.nb)
+        cpu, mask_report = oracle_baseline(w, q_h, k_h, v_h, gpu_keep, budget_s=args.cpu_budget)
     clk = clocks.summary()
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -422,6 +460,7 @@ def run_ours(args, w, rank, world, dist):
             "workload": w.name, "B": w.B, "T": w.T, "H": w.H, "W": w.W, "N": w.N, "Npad": plan.Npad,
             "heads": w.heads, "d": w.d, "block": w.block, "patch": w.patch, "thr": w.thr,
             "sta": list(w.sta) if w.sta else None, "density": dens, "parallelism": f"replicas x{world}",
+            "attn_kernel": "mma.sync (legacy baseline)" if args.baseline_kernel else "tcgen05",
             "l2": "flushed between steps (write of a 2x L2 buffer, outside the step events)",
             "attn_ms": attn_ms, "attn_tflops": attn_tf, "attn_pct_bf16_peak": 100.0 * attn_tf / peak_tf,
             "breakdown_ms": {"reorder_qk": float(br[0]), "mask_and_reorder_v": mask_ms, "attn": attn_ms,
@@ -430,6 +469,7 @@ def run_ours(args, w, rank, world, dist):
             "mask_pct_hbm": 100.0 * mask_bytes / (mask_ms * 1e-3) / 1e9 / hbm if mask_ms > 0 else None,
             "reorder_gbs": reorder_bytes / (float(br[0]) * 1e-3) / 1e9,
             "mask_precision": "f64 pooled means, dots and masses",
+            **mask_report,
             "step_ms_median": float(np.median(parts.sum(axis=1))),
             "step_ms_min": float(parts.sum(axis=1).min()),
             "attn_ms_median": float(np.median(parts[:, 2])),
@@ -457,6 +497,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="wan480p")
     ap.add_argument("--density", type=float, default=None, help="density-sweep workload: kept fraction")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--baseline-kernel", action="store_true",
+                    help="time the legacy mma.sync attention kernel instead of the tcgen05 one")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     args = ap.parse_args(argv)
     if args.warmup < 3:

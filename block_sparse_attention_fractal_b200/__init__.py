@@ -18,12 +18,19 @@ from typing import Optional, Tuple
 import torch
 
 from ._lib import (BsaError, Shape, attn_fwd, attn_fwd_baseline, build_block_mask, check_device_status, inverse_reorder,  # noqa: F401
-                   lib, make_shape, num_blocks, padded_len, reorder, seq_len, validate_shape, workspace_bytes,
+                   get_lib, make_shape, num_blocks, padded_len, reorder, seq_len, validate_shape, workspace_bytes,
                    workspace_init, LIB_PATH)
+
+def __getattr__(name):
+    # ``lib`` (the ctypes handle of libbsa.so) is loaded on first access
+    if name == "lib":
+        return get_lib()
+    raise AttributeError(name)
+
 
 __all__ = ["BsaError", "Shape", "make_shape", "NablaAttention", "reorder", "inverse_reorder", "build_block_mask",
            "attn_fwd", "attn_fwd_baseline", "check_device_status", "workspace_bytes", "workspace_init", "padded_len", "num_blocks",
-           "seq_len", "validate_shape", "LIB_PATH"]
+           "seq_len", "validate_shape", "get_lib", "LIB_PATH"]
 
 
 class NablaAttention:

@@ -2,8 +2,10 @@
 
 Every function takes torch tensors (device memory owned by the caller), passes
 their raw pointers, sizes and the current CUDA stream to the C ABI declared in
-include/bsa.h, and raises ``BsaError`` on a non-OK status.  There is no
-fallback: if the shared library is missing, importing this module fails.
+include/bsa.h, and raises ``BsaError`` on a non-OK status.  The library is
+loaded on the first call (so that importing the package, e.g. for its input
+generator, maps nothing); there is no fallback: if libbsa.so is missing, that
+first call raises ImportError.
 """
 from __future__ import annotations
 
@@ -65,7 +67,21 @@ def _load() -> ctypes.CDLL:
     return lib
 
 
-lib = _load()
+_LIB = None
+
+
+def get_lib() -> ctypes.CDLL:
+    """libbsa.so, loaded on first use; ImportError if it has not been built."""
+    global _LIB
+    if _LIB is None:
+        _LIB = _load()
+    return _LIB
+
+
+def __getattr__(name):
+    if name == "lib":
+        return get_lib()
+    raise AttributeError(name)
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
@@ -90,36 +106,36 @@ def make_shape(B: int, T: int, H: int, W: int, heads: int, d: int, block: int, p
 
 
 def validate_shape(s: Shape) -> int:
-    return lib.bsa_validate_shape(ctypes.byref(s))
+    return get_lib().bsa_validate_shape(ctypes.byref(s))
 
 
 def seq_len(s: Shape) -> int:
-    return lib.bsa_seq_len(ctypes.byref(s))
+    return get_lib().bsa_seq_len(ctypes.byref(s))
 
 
 def padded_len(s: Shape) -> int:
-    return lib.bsa_padded_len(ctypes.byref(s))
+    return get_lib().bsa_padded_len(ctypes.byref(s))
 
 
 def num_blocks(s: Shape) -> int:
-    return lib.bsa_num_blocks(ctypes.byref(s))
+    return get_lib().bsa_num_blocks(ctypes.byref(s))
 
 
 def workspace_bytes(s: Shape) -> int:
-    return lib.bsa_workspace_bytes(ctypes.byref(s))
+    return get_lib().bsa_workspace_bytes(ctypes.byref(s))
 
 
 def workspace_init(ws: torch.Tensor) -> None:
-    _check(lib.bsa_workspace_init(_ptr(ws), ws.numel() * ws.element_size(), _stream(ws.device)),
+    _check(get_lib().bsa_workspace_init(_ptr(ws), ws.numel() * ws.element_size(), _stream(ws.device)),
            "bsa_workspace_init")
 
 
 def reorder(s: Shape, x_bnhd: torch.Tensor, y_bhnd: torch.Tensor) -> None:
-    _check(lib.bsa_reorder(ctypes.byref(s), _ptr(x_bnhd), _ptr(y_bhnd), _stream(x_bnhd.device)), "bsa_reorder")
+    _check(get_lib().bsa_reorder(ctypes.byref(s), _ptr(x_bnhd), _ptr(y_bhnd), _stream(x_bnhd.device)), "bsa_reorder")
 
 
 def inverse_reorder(s: Shape, y_bhnd: torch.Tensor, x_bnhd: torch.Tensor) -> None:
-    _check(lib.bsa_inverse_reorder(ctypes.byref(s), _ptr(y_bhnd), _ptr(x_bnhd), _stream(y_bhnd.device)),
+    _check(get_lib().bsa_inverse_reorder(ctypes.byref(s), _ptr(y_bhnd), _ptr(x_bnhd), _stream(y_bhnd.device)),
            "bsa_inverse_reorder")
 
 
@@ -127,7 +143,7 @@ def build_block_mask(s: Shape, q_bhnd: torch.Tensor, k_bhnd: torch.Tensor, thr: 
                      sta: Optional[Tuple[int, int, int]], kv_count: torch.Tensor, kv_idx: torch.Tensor,
                      mask: Optional[torch.Tensor], ws: torch.Tensor) -> None:
     st_t, st_h, st_w = sta if sta is not None else (-1, -1, -1)
-    _check(lib.bsa_build_block_mask(ctypes.byref(s), _ptr(q_bhnd), _ptr(k_bhnd), float(thr), st_t, st_h, st_w,
+    _check(get_lib().bsa_build_block_mask(ctypes.byref(s), _ptr(q_bhnd), _ptr(k_bhnd), float(thr), st_t, st_h, st_w,
                                     _ptr(kv_count), _ptr(kv_idx), _ptr(mask), _ptr(ws),
                                     ws.numel() * ws.element_size(), _stream(q_bhnd.device)),
            "bsa_build_block_mask")
@@ -136,7 +152,7 @@ def build_block_mask(s: Shape, q_bhnd: torch.Tensor, k_bhnd: torch.Tensor, thr: 
 def attn_fwd(s: Shape, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, kv_count: torch.Tensor,
              kv_idx: torch.Tensor, scale: float, o: torch.Tensor, lse: Optional[torch.Tensor],
              ws: torch.Tensor) -> None:
-    _check(lib.bsa_attn_fwd(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(kv_count), _ptr(kv_idx),
+    _check(get_lib().bsa_attn_fwd(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(kv_count), _ptr(kv_idx),
                             float(scale), _ptr(o), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(),
                             _stream(q.device)),
            "bsa_attn_fwd")
@@ -146,7 +162,7 @@ def attn_fwd_baseline(s: Shape, q: torch.Tensor, k: torch.Tensor, v: torch.Tenso
                       kv_idx: torch.Tensor, scale: float, o: torch.Tensor, lse: Optional[torch.Tensor],
                       ws: torch.Tensor) -> None:
     """The legacy mma.sync kernel with the same contract (the measured baseline)."""
-    _check(lib.bsa_attn_fwd_baseline(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(kv_count), _ptr(kv_idx),
+    _check(get_lib().bsa_attn_fwd_baseline(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(kv_count), _ptr(kv_idx),
                                      float(scale), _ptr(o), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(),
                                      _stream(q.device)),
            "bsa_attn_fwd_baseline")
@@ -154,4 +170,4 @@ def attn_fwd_baseline(s: Shape, q: torch.Tensor, k: torch.Tensor, v: torch.Tenso
 
 def check_device_status(ws: torch.Tensor) -> int:
     """Synchronises the current stream; returns the device status (0 = OK) and clears it."""
-    return lib.bsa_check_device_status(_ptr(ws), _stream(ws.device))
+    return get_lib().bsa_check_device_status(_ptr(ws), _stream(ws.device))

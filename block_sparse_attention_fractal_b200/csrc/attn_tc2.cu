@@ -29,7 +29,9 @@
 // MMAs and warp 1 the P.V MMAs (one elected thread each), warps 4-11 run the
 // softmax and the epilogue (warp w reads TMEM lanes 32 (w mod 4) .. +31).
 // Every mbarrier wait is bounded; on expiry the CTA records BSA_ERR_TIMEOUT in
-// the workspace error word and leaves.
+// the workspace error word, tells the launch's other CTAs to give up (its own
+// launch sequence number in the control block), waits (bounded) for the
+// copies and MMAs it has already issued, frees its TMEM and leaves.
 #include <cmath>
 #include <cstdlib>
 
@@ -53,13 +55,12 @@ constexpr uint64_t kWaitNs = 250ull * 1000ull * 1000ull;  // 250 ms: far beyond 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 256;     // O_0 at 256, O_1 at 384; S_0 at 0, S_1 at 128
 constexpr uint32_t kPTile = 128u * 128u * 2u;  // bf16 P of one 128 x 128 tile in shared memory
-// One pair of scores in kPolyEvery takes the software exp2 (0 = none).
-constexpr int kPolyEvery = 0;
 
 struct Ctl {
   uint64_t q_full;
   uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
   uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];   // per softmax group
+  uint64_t drain[2];   // final commit of each MMA issuer (S, P.V) before TMEM is freed
   uint32_t tmem_base;
   int n_ent;
   int item;
@@ -71,20 +72,22 @@ struct Ctl {
 };
 constexpr uint16_t kEntBlock = 0x0FFFu;
 
-__device__ __forceinline__ void timeout(Ctrl* ctrl, Ctl& c, uint32_t site) {
+__device__ __forceinline__ void timeout(Ctrl* ctrl, Ctl& c, uint32_t seq, uint32_t site) {
   report_error(ctrl, kErrTimeout, blockIdx.x, threadIdx.x, site);
+  atomicExch(&ctrl->abort_seq, seq);
   c.abort = 1;
 }
 
-// Bounded wait; gives up early once any CTA of the launch has timed out.
-__device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity, Ctrl* ctrl) {
-  return mbar_wait_ns(bar, parity, kWaitNs, &ctrl->error, kErrTimeout);
+// Bounded wait; gives up early once a CTA of this launch (sequence number
+// `seq`) has timed out.
+__device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity, Ctrl* ctrl, uint32_t seq) {
+  return mbar_wait_ns(bar, parity, kWaitNs, &ctrl->abort_seq, seq);
 }
 
 // Same, with one verdict for the whole warp (the tcgen05.ld/st that follow
 // are warp-collective and must not run in a partial warp).
-__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, Ctrl* ctrl) {
-  const bool ok = wait(bar, parity, ctrl);
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, Ctrl* ctrl, uint32_t seq) {
+  const bool ok = wait(bar, parity, ctrl, seq);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -115,7 +118,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
                                                                const int2* __restrict__ items, int* work,
                                                                float scale_log2, __nv_bfloat16* __restrict__ o,
                                                                float* __restrict__ lse, Ctrl* ctrl, Dims g,
-                                                               int items_per_bh, int n_items, int force_timeout) {
+                                                               int items_per_bh, int n_items, uint32_t seq,
+                                                               int force_timeout) {
   constexpr int QB = 128 / BS;          // query blocks per tile
   constexpr int E = 128 / BS;           // list entries per KV tile
   constexpr int CH = D / 64;            // 64-column (128-byte) chunks of a row
@@ -156,6 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
       mbar_init(&c.s_free[w], kGroupThreads);
       mbar_init(&c.p_full[w], kGroupThreads);
       mbar_init(&c.pv_done[w], 1);
+      mbar_init(&c.drain[w], 1);
     }
     c.abort = 0;
     fence_mbar_init();
@@ -178,13 +183,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
   // that nothing arrives on, before any copy or MMA is issued; it records
   // BSA_ERR_TIMEOUT and the CTA does no work.
   if (force_timeout) {
-    if (tid == 0 && !mbar_wait_ns(&c.q_full, 0, 2ull * 1000ull * 1000ull, &ctrl->error, 0u)) timeout(ctrl, c, 1);
+    if (tid == 0 && !mbar_wait_ns(&c.q_full, 0, 2ull * 1000ull * 1000ull, nullptr, 0u)) timeout(ctrl, c, seq, 1);
     __syncthreads();
   }
 
   uint32_t jbase = 0;  // KV tiles this CTA has run so far (phase counter of the K/V stages)
   uint32_t gbase[2] = {0u, 0u};  // KV tiles each softmax group has run so far
   uint32_t nq = 0;     // Q loads so far (phase of q_full)
+  uint32_t armed = 0;  // K (warp 0) or V (warp 2) stage loads this producer thread has issued
 
   for (;;) {
     if (tid == 0) c.item = atomicAdd(work, 1);
@@ -291,8 +297,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
           }
           if (is_k) {
             const uint32_t s = jg & 1;
-            if (jg >= 2 && !wait(&c.k_empty[s], ((jg - 2) >> 1) & 1, ctrl)) { timeout(ctrl, c, 10); break; }
+            if (jg >= 2 && !wait(&c.k_empty[s], ((jg - 2) >> 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 10); break; }
             mbar_arrive_expect_tx(&c.k_full[s], kTile);
+            ++armed;
             uint8_t* dk = sK + s * kTile;
 #pragma unroll
             for (int ch = 0; ch < CH; ++ch)
@@ -301,8 +308,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
                 tma_load_3d(dk + ch * kChunk + h * (kChunk / 2), &mk, &c.k_full[s], ch * 64, krow[h], bh);
           } else {
             const uint32_t s = jg & 1;
-            if (jg >= 2 && !wait(&c.v_empty[s], ((jg - 2) >> 1) & 1, ctrl)) { timeout(ctrl, c, 11); break; }
+            if (jg >= 2 && !wait(&c.v_empty[s], ((jg - 2) >> 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 11); break; }
             mbar_arrive_expect_tx(&c.v_full[s], kTile);
+            ++armed;
             uint8_t* dv = sV + s * kTile;
 #pragma unroll
             for (int ch = 0; ch < CH; ++ch)
@@ -322,15 +330,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
         constexpr uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);
         const uint64_t dQ = smem_desc_sw128(smem_addr(sQ), 16, 1024);
         const uint32_t aK = smem_addr(sK);
-        if (!wait(&c.q_full, nq & 1, ctrl)) {
-          timeout(ctrl, c, 20);
+        if (!wait(&c.q_full, nq & 1, ctrl, seq)) {
+          timeout(ctrl, c, seq, 20);
         } else {
           for (int j = 0; j < n_tiles; ++j) {
             const uint32_t jg = jbase + j, ks = jg & 1;
             const int w = j & 1;
             const uint32_t gw = gbase[w] + (j >> 1);   // this group's tile count
-            if (!wait(&c.k_full[ks], (jg >> 1) & 1, ctrl)) { timeout(ctrl, c, 21); break; }
-            if (gw >= 1 && !wait(&c.s_free[w], (gw - 1) & 1, ctrl)) { timeout(ctrl, c, 22); break; }
+            if (!wait(&c.k_full[ks], (jg >> 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 21); break; }
+            if (gw >= 1 && !wait(&c.s_free[w], (gw - 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 22); break; }
             tc_fence_after();
             // descriptors built once per tile: the issuing thread shares its
             // sub-partition with two softmax warps, so each MMA costs it only
@@ -357,8 +365,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
           const uint32_t jg = jbase + j, vs = jg & 1;
           const int w = j & 1;
           const uint32_t gw = gbase[w] + (j >> 1);
-          if (!wait(&c.p_full[w], gw & 1, ctrl)) { timeout(ctrl, c, 23); break; }
-          if (!wait(&c.v_full[vs], (jg >> 1) & 1, ctrl)) { timeout(ctrl, c, 24); break; }
+          if (!wait(&c.p_full[w], gw & 1, ctrl, seq)) { timeout(ctrl, c, seq, 23); break; }
+          if (!wait(&c.v_full[vs], (jg >> 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 24); break; }
           tc_fence_after();
           const uint64_t dP = smem_desc_sw128(aP + w * kPTile, 16, 1024);
           const uint64_t dV = smem_desc_sw128(aV + vs * kTile, kChunk, 1024);
@@ -401,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
           }
           lim[h] = kept ? max(0, min(64, g.N - key0)) : 0;
         }
-        if (!wait_warp(&c.s_full[w], gw & 1, ctrl)) { timeout(ctrl, c, 30); ok = false; break; }
+        if (!wait_warp(&c.s_full[w], gw & 1, ctrl, seq)) { timeout(ctrl, c, seq, 30); ok = false; break; }
         tc_fence_after();
         // Pass 1: row max of the raw scores over the kept, real keys (scale > 0
         // keeps the order), 64 columns at a time.
@@ -434,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
         }
         // O_w and P buffer w are free once the group's previous P.V product
         // has completed (normally long before: it was issued a tile ago).
-        if (gw >= 1 && !wait_warp(&c.pv_done[w], (gw - 1) & 1, ctrl)) { timeout(ctrl, c, 32); ok = false; break; }
+        if (gw >= 1 && !wait_warp(&c.pv_done[w], (gw - 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 32); ok = false; break; }
         tc_fence_after();
         const float mnew = fmaxf(m, fmaxf(mh[0], mh[1]) * scale_log2);
         // The running max moves only when it grows by more than 8 (a factor
@@ -460,8 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
         }
         if (grow) m = mnew;
         const float nm = (m == -INFINITY) ? 0.f : -m;
-        // p = 2^(s * scale_log2 - m): one FFMA and one MUFU ex2 per score (or,
-        // for one pair in kPolyEvery, the FMA-pipe polynomial).  O is
+        // p = 2^(s * scale_log2 - m): one FFMA and one MUFU ex2 per score.  O is
         // normalised by the sum of the bf16-rounded weights the P.V product
         // uses (an exact convex combination of V rows up to accumulation
         // rounding); the LSE, when asked for, uses the fp32 sum of the
@@ -496,12 +503,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
               const float2 yy = ffma2(make_float2(x[2 * i], x[2 * i + 1]), sc2, nm2);
               const float y0 = yy.x, y1 = yy.y;
               float2 p;
-              if (kPolyEvery > 0 && (i % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
-                p = exp2_poly2(make_float2(y0, y1));
-              } else {
-                p.x = ex2f(y0);
-                p.y = ex2f(y1);
-              }
+              p.x = ex2f(y0);
+              p.y = ex2f(y1);
               if (lim[h] < 64) {
                 const int kc = (cch & 1) * 32 + 2 * i;   // key within the half
                 p.x = (kc < lim[h]) ? p.x : 0.f;
@@ -536,8 +539,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
       // product of each group that ran a tile.
       const int cnt0 = (n_tiles + 1) / 2, cnt1 = n_tiles / 2;
       const bool has0 = cnt0 > 0, has1 = cnt1 > 0;
-      if (ok && has0 && !wait_warp(&c.pv_done[0], (gbase[0] + cnt0 - 1) & 1, ctrl)) { timeout(ctrl, c, 31); ok = false; }
-      if (ok && has1 && !wait_warp(&c.pv_done[1], (gbase[1] + cnt1 - 1) & 1, ctrl)) { timeout(ctrl, c, 31); ok = false; }
+      // The pv_done parity waits protect this group's own accumulator; the
+      // other group's is covered by its own wait, ordered before this
+      // thread's reads by the pair barrier below (and the fence after it).
+      if (ok && has0 && !wait_warp(&c.pv_done[0], (gbase[0] + cnt0 - 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 31); ok = false; }
+      if (ok && has1 && !wait_warp(&c.pv_done[1], (gbase[1] + cnt1 - 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 31); ok = false; }
       tc_fence_after();
       // The merge goes through the K stages: every S of the item has completed
       // (its softmax ran) and the next item's K loads start after the item.
@@ -546,7 +552,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
       xm[w * 128 + r] = (mine > 0) ? m : -INFINITY;
       xl[(2 * w + 0) * 128 + r] = l;
       xl[(2 * w + 1) * 128 + r] = lx;
+      tc_fence_before();
       ok = pair_sync(q4, ok);
+      tc_fence_after();
       const float m0 = xm[r], m1 = xm[128 + r];
       const float mt = fmaxf(m0, m1);
       const float a0 = (has0 && m0 != -INFINITY) ? ex2f(m0 - mt) : 0.f;
@@ -604,6 +612,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
     if (n_tiles > 0) ++nq;
   }
 
+  // Drain: every copy and MMA this CTA issued completes before its TMEM is
+  // freed and it exits (after a timeout some may still be in flight).  In a
+  // normal exit all of them have completed already and these waits return
+  // at once.
+  if (lane == 0) {
+    if (warp == 0) {
+      mbar_drain_ring(&c.q_full, 1, nq, kWaitNs);
+      mbar_drain_ring(c.k_full, 2, armed, kWaitNs);
+    } else if (warp == 2) {
+      mbar_drain_ring(c.v_full, 2, armed, kWaitNs);
+    } else if (warp == 3 || warp == 1) {
+      uint64_t* d = &c.drain[warp == 3 ? 0 : 1];
+      mma_commit(d);
+      mbar_wait_ns(d, 0, kWaitNs, nullptr, 0u);
+    }
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -630,7 +654,7 @@ int num_sms() {
 template <int D, int BS, bool WITH_LSE>
 cudaError_t launch_tc2(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
                        const int32_t* kv_idx, const int2* items, int* work, float scale, void* o, float* lse,
-                       Ctrl* ctrl, cudaStream_t st) {
+                       Ctrl* ctrl, uint32_t seq, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
   const uint64_t rows = (uint64_t)g.Npad, bhs = (uint64_t)g.B * g.heads;
   if (!make_map_bf16_3d(&mq, q, D, rows, bhs, 64, 64) || !make_map_bf16_3d(&mk, k, D, rows, bhs, 64, 64) ||
@@ -646,31 +670,32 @@ cudaError_t launch_tc2(const Dims& g, const void* q, const void* k, const void* 
   const int grid = n_items < num_sms() ? n_items : num_sms();
   attn_tc2_kernel<D, BS, WITH_LSE><<<grid, kThreads, smem, st>>>(mq, mk, mv, kv_count, kv_idx, items, work,
                                                                  scale * 1.4426950408889634f, (__nv_bfloat16*)o, lse,
-                                                                 ctrl, g, items_per_bh, n_items, force_timeout_requested());
+                                                                 ctrl, g, items_per_bh, n_items, seq,
+                                                                 force_timeout_requested());
   return cudaGetLastError();
 }
 
 template <int D, int BS>
 cudaError_t launch_tc2_lse(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
                            const int32_t* kv_idx, const int2* items, int* work, float scale, void* o, float* lse,
-                           Ctrl* ctrl, cudaStream_t st) {
+                           Ctrl* ctrl, uint32_t seq, cudaStream_t st) {
   if (lse != nullptr)
-    return launch_tc2<D, BS, true>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, st);
-  return launch_tc2<D, BS, false>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, st);
+    return launch_tc2<D, BS, true>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, seq, st);
+  return launch_tc2<D, BS, false>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, seq, st);
 }
 
 }  // namespace
 
 cudaError_t launch_attn_tc2(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
                             const int32_t* kv_idx, const int2* items, int* work, float scale, void* o, float* lse,
-                            Ctrl* ctrl, cudaStream_t st) {
+                            Ctrl* ctrl, uint32_t seq, cudaStream_t st) {
   if (g.d == 128 && g.bs == 64)
-    return launch_tc2_lse<128, 64>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, st);
+    return launch_tc2_lse<128, 64>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, seq, st);
   if (g.d == 128 && g.bs == 128)
-    return launch_tc2_lse<128, 128>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, st);
+    return launch_tc2_lse<128, 128>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, seq, st);
   if (g.d == 64 && g.bs == 64)
-    return launch_tc2_lse<64, 64>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, st);
-  return launch_tc2_lse<64, 128>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, st);
+    return launch_tc2_lse<64, 64>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, seq, st);
+  return launch_tc2_lse<64, 128>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, seq, st);
 }
 
 }  // namespace bsa

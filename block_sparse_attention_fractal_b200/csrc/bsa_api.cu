@@ -1,6 +1,7 @@
 // C ABI of libbsa (declared in include/bsa.h): argument checking, workspace
 // layout and kernel launches.  No entry point allocates, frees or
 // synchronises, except bsa_check_device_status.
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -10,6 +11,19 @@
 
 using bsa::Ctrl;
 using bsa::Dims;
+
+namespace bsa {
+
+uint32_t next_launch_seq() {
+  static std::atomic<uint32_t> counter{0};
+  uint32_t s;
+  do {
+    s = counter.fetch_add(1, std::memory_order_relaxed) + 1u;
+  } while (s == 0u);
+  return s;
+}
+
+}  // namespace bsa
 
 namespace {
 
@@ -126,7 +140,7 @@ bsa_status bsa_build_block_mask(const bsa_shape* s, const void* q_bhnd, const vo
   double* qbar = (double*)((char*)workspace + sizeof(Ctrl));
   double* kbar = qbar + pooled_bytes(g) / sizeof(double);
   cudaStream_t cs = (cudaStream_t)stream;
-  cudaError_t e = bsa::launch_pool(g, q_bhnd, k_bhnd, qbar, kbar, (Ctrl*)workspace, cs);
+  cudaError_t e = bsa::launch_pool(g, q_bhnd, k_bhnd, qbar, kbar, (Ctrl*)workspace, bsa::next_launch_seq(), cs);
   if (e != cudaSuccess) return BSA_ERR_CUDA;
   e = bsa::launch_mask(g, qbar, kbar, (double)thr, sta ? sta_t : -1, sta ? sta_h : -1, sta ? sta_w : -1, kv_count,
                        kv_idx, mask_or_null, cs);
@@ -160,8 +174,8 @@ bsa_status attn_common(const bsa_shape* s, const void* q, const void* k, const v
   int2* items = (int2*)((char*)workspace + plan_offset(g));
   cudaError_t e = bsa::launch_plan(g, kv_count, kv_idx, items, (cudaStream_t)stream);
   if (e != cudaSuccess) return BSA_ERR_CUDA;
-  return from_cuda(bsa::launch_attn_tc2(g, q, k, v, kv_count, kv_idx, items, bsa::plan_work_counter(g, items), scale, o, lse_or_null, ctrl,
-                                       (cudaStream_t)stream));
+  return from_cuda(bsa::launch_attn_tc2(g, q, k, v, kv_count, kv_idx, items, bsa::plan_work_counter(g, items), scale,
+                                       o, lse_or_null, ctrl, bsa::next_launch_seq(), (cudaStream_t)stream));
 }
 
 }  // namespace

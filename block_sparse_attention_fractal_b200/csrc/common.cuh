@@ -22,7 +22,12 @@ enum : uint32_t {
 struct Ctrl {
   uint32_t error;       // OR of kErr* bits
   uint32_t detail[3];   // first offending (row, value, site) for diagnostics
-  uint32_t pad[60];
+  // Sequence number of the launch whose CTAs are giving up after a bounded
+  // wait expired.  Every launch gets its own nonzero number, and a CTA gives
+  // up early only on its own launch's number, so a timeout left behind by an
+  // earlier call never cuts a later call short.
+  uint32_t abort_seq;
+  uint32_t pad[59];
 };
 static_assert(sizeof(Ctrl) == 256, "control block is 256 bytes");
 

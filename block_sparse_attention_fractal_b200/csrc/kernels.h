@@ -7,13 +7,17 @@
 
 namespace bsa {
 
+// A fresh nonzero launch sequence number (host side, thread safe); kernels
+// with bounded waits compare it with Ctrl::abort_seq.
+uint32_t next_launch_seq();
+
 cudaError_t launch_reorder(const Dims& g, const void* x_bnhd, void* y_bhnd, cudaStream_t st);
 cudaError_t launch_inverse_reorder(const Dims& g, const void* y_bhnd, void* x_bnhd, cudaStream_t st);
 
 // Block means of Q and K (double): `qbar` [B, heads, nb, d], `kbar`
 // transposed [B, heads, d, nb].
 cudaError_t launch_pool(const Dims& g, const void* q, const void* k, double* qbar, double* kbar, Ctrl* ctrl,
-                        cudaStream_t st);
+                        uint32_t seq, cudaStream_t st);
 
 // Reduced attention + CDF threshold (+ STA union) -> KV lists.
 cudaError_t launch_mask(const Dims& g, const double* qbar, const double* kbar, double thr, int sta_t, int sta_h,
@@ -39,6 +43,6 @@ cudaError_t launch_plan(const Dims& g, const int32_t* kv_count, const int32_t* k
 // alternating KV tiles, query tiles fetched from the plan's work counter.
 cudaError_t launch_attn_tc2(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
                             const int32_t* kv_idx, const int2* items, int* work, float scale, void* o, float* lse,
-                            Ctrl* ctrl, cudaStream_t st);
+                            Ctrl* ctrl, uint32_t seq, cudaStream_t st);
 
 }  // namespace bsa

@@ -44,7 +44,7 @@ template <int D, int BS>
 __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __nv_bfloat16* __restrict__ q,
                                                             const __nv_bfloat16* __restrict__ k,
                                                             double* __restrict__ qbar, double* __restrict__ kbar,
-                                                            Ctrl* ctrl, Dims g) {
+                                                            Ctrl* ctrl, Dims g, uint32_t seq) {
   constexpr uint32_t kTileBytes = BS * D * 2;
   constexpr int kPoolStages = pool_stages<D, BS>();
   constexpr int kPairs = D / 2;                    // bf16 column pairs of a row
@@ -71,10 +71,12 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __nv_bfloat16*
     sm100::fence_mbar_init();
   }
   __syncthreads();
+  uint32_t armed = 0;   // stage loads issued (thread 0)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPoolStages; ++s) {
       const int it = blockIdx.x + s * G;
       if (it >= total) break;
+      ++armed;
       sm100::mbar_arrive_expect_tx(&full[s], kTileBytes);
       sm100::bulk_load(tiles + s * kTileBytes, item_ptr(it), kTileBytes, &full[s]);
     }
@@ -85,9 +87,12 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __nv_bfloat16*
     const int it = blockIdx.x + n * G;
     if (it >= total) break;
     const int s = n % kPoolStages;
-    const bool ok = sm100::mbar_wait_ns(&full[s], (n / kPoolStages) & 1, kPoolWaitNs, &ctrl->error, kErrTimeout);
+    const bool ok = sm100::mbar_wait_ns(&full[s], (n / kPoolStages) & 1, kPoolWaitNs, &ctrl->abort_seq, seq);
     if (!ok) {
-      if (threadIdx.x == 0) report_error(ctrl, kErrTimeout, blockIdx.x, (uint32_t)it, 40u);
+      if (threadIdx.x == 0) {
+        report_error(ctrl, kErrTimeout, blockIdx.x, (uint32_t)it, 40u);
+        atomicExch(&ctrl->abort_seq, seq);
+      }
       stop = 1;
     }
     __syncthreads();
@@ -106,6 +111,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __nv_bfloat16*
     part[rg * D + 2 * cp + 1] = a1;
     __syncthreads();   // the stage is read and the partial sums are in place
     if (threadIdx.x == 0 && it + kPoolStages * G < total) {
+      ++armed;
       sm100::mbar_arrive_expect_tx(&full[s], kTileBytes);
       sm100::bulk_load(tiles + s * kTileBytes, item_ptr(it + kPoolStages * G), kTileBytes, &full[s]);
     }
@@ -124,6 +130,8 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __nv_bfloat16*
     }
     __syncthreads();   // part is rewritten by the next block
   }
+  // no bulk copy of this CTA may still be in flight when it exits
+  if (threadIdx.x == 0) sm100::mbar_drain_ring(full, kPoolStages, armed, kPoolWaitNs);
 }
 
 // ------------------------------------------------------------- mask rows
@@ -411,7 +419,7 @@ __global__ void __launch_bounds__(kMaskThreads) mask_kernel(const double* __rest
 
 template <int D, int BS>
 cudaError_t launch_pool_t(const Dims& g, const void* q, const void* k, double* qbar, double* kbar, Ctrl* ctrl,
-                          cudaStream_t st) {
+                          uint32_t seq, cudaStream_t st) {
   const size_t smem = (size_t)pool_stages<D, BS>() * BS * D * 2 + (size_t)(kPoolThreads / (D / 2)) * D * sizeof(double);
   cudaError_t e = cudaFuncSetAttribute(pool_kernel<D, BS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -424,16 +432,16 @@ cudaError_t launch_pool_t(const Dims& g, const void* q, const void* k, double* q
   const int total = 2 * g.B * g.heads * g.nb;
   const int grid = std::max(1, std::min(total, sms * std::max(1, per_sm)));
   pool_kernel<D, BS><<<grid, kPoolThreads, smem, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qbar,
-                                                       kbar, ctrl, g);
+                                                       kbar, ctrl, g, seq);
   return cudaGetLastError();
 }
 
 cudaError_t launch_pool(const Dims& g, const void* q, const void* k, double* qbar, double* kbar, Ctrl* ctrl,
-                        cudaStream_t st) {
-  if (g.d == 128 && g.bs == 64) return launch_pool_t<128, 64>(g, q, k, qbar, kbar, ctrl, st);
-  if (g.d == 128 && g.bs == 128) return launch_pool_t<128, 128>(g, q, k, qbar, kbar, ctrl, st);
-  if (g.d == 64 && g.bs == 64) return launch_pool_t<64, 64>(g, q, k, qbar, kbar, ctrl, st);
-  return launch_pool_t<64, 128>(g, q, k, qbar, kbar, ctrl, st);
+                        uint32_t seq, cudaStream_t st) {
+  if (g.d == 128 && g.bs == 64) return launch_pool_t<128, 64>(g, q, k, qbar, kbar, ctrl, seq, st);
+  if (g.d == 128 && g.bs == 128) return launch_pool_t<128, 128>(g, q, k, qbar, kbar, ctrl, seq, st);
+  if (g.d == 64 && g.bs == 64) return launch_pool_t<64, 64>(g, q, k, qbar, kbar, ctrl, seq, st);
+  return launch_pool_t<64, 128>(g, q, k, qbar, kbar, ctrl, seq, st);
 }
 
 template <int D, int NJ>

@@ -17,6 +17,8 @@
 #include <cstdint>
 #include <mutex>
 
+#include <cuda.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -31,25 +33,55 @@ constexpr int kMaxDevices = 64;
 static __device__ __align__(256) uint8_t g_noalloc_scratch[BSA_NOALLOC_SCRATCH_BYTES];
 
 // Device address of g_noalloc_scratch for each device ordinal (in host code the
-// symbol itself is only a host-side stand-in, not a device address).
-void* g_scratch_addr[kMaxDevices] = {};
+// symbol itself is only a host-side stand-in, not a device address), with the
+// context it was looked up in: a device reset (or a context destroyed and made
+// again) loads the module anew, so an address from another context is stale
+// and is looked up again.
+struct ScratchAddr {
+  CUcontext ctx;
+  void* addr;
+};
+ScratchAddr g_scratch[kMaxDevices] = {};
 std::mutex g_scratch_mu;
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (CtxGetCurrentFn)p;
+  }
+  return fn;
+}
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// Looks up (once per device, with that device current) the device address of
-// the scratch array.
+// The device address of the scratch array on the current device, looked up
+// (cudaGetSymbolAddress, with that device current) on the first call in each
+// context.
 bsa_status scratch_for_current_device(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return BSA_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return BSA_ERR_UNSUPPORTED;
+  CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+  if (get_ctx == nullptr) return BSA_ERR_CUDA;
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS) return BSA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+  if (ctx == nullptr || g_scratch[dev].addr == nullptr || g_scratch[dev].ctx != ctx) {
+    // (the lookup also makes the device's primary context current when this
+    // thread has none yet)
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return BSA_ERR_CUDA;
-    g_scratch_addr[dev] = p;
+    if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return BSA_ERR_CUDA;
+    g_scratch[dev].ctx = ctx;
+    g_scratch[dev].addr = p;
   }
-  *out = g_scratch_addr[dev];
+  *out = g_scratch[dev].addr;
   return BSA_OK;
 }
 
@@ -98,7 +130,8 @@ bsa_status bsa_attn_fwd_noalloc(const bsa_shape* s, const void* q, const void* k
   // The control block keeps the last call's contents: clear it first.
   if (cudaMemsetAsync(ctrl, 0, sizeof(Ctrl), cs) != cudaSuccess) return BSA_ERR_CUDA;
   if (bsa::launch_plan(g, kv_count, kv_idx, items, cs) != cudaSuccess) return BSA_ERR_CUDA;
-  if (bsa::launch_attn_tc2(g, q, k, v, kv_count, kv_idx, items, bsa::plan_work_counter(g, items), scale, o, lse_or_null, ctrl, cs) != cudaSuccess)
+  if (bsa::launch_attn_tc2(g, q, k, v, kv_count, kv_idx, items, bsa::plan_work_counter(g, items), scale, o,
+                           lse_or_null, ctrl, bsa::next_launch_seq(), cs) != cudaSuccess)
     return BSA_ERR_CUDA;
   if (error_word_or_null != nullptr &&
       cudaMemcpyAsync(error_word_or_null, &ctrl->error, sizeof(uint32_t), cudaMemcpyDeviceToDevice, cs) !=

@@ -1,9 +1,9 @@
 // Thin inline-PTX wrappers for the sm_100a features the attention kernel uses:
 // mbarriers, TMA tiled loads (no multicast), and the 5th-generation tensor
 // core (tcgen05: TMEM allocation, MMA, commit, TMEM loads and stores).
-// Every wait on an mbarrier is bounded: it gives up after `limit` polls and
-// returns false, so a kernel can record the failure and leave instead of
-// hanging.
+// Every wait on an mbarrier is bounded: it gives up after a time limit (or
+// when its launch is giving up) and returns false, so a kernel can record the
+// failure and leave instead of hanging.
 #pragma once
 
 #include <cstdint>
@@ -49,15 +49,6 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0u;
 }
 
-// Waits until the phase with the given parity has completed; false after
-// `limit` unsuccessful polls (each try_wait itself blocks for a short while).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit) {
-  for (uint32_t i = 0; i < limit; ++i) {
-    if (mbar_test(bar, parity)) return true;
-  }
-  return false;
-}
-
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;\n" : "=l"(t));
@@ -65,10 +56,11 @@ __device__ __forceinline__ uint64_t global_ns() {
 }
 
 // Waits until the phase with the given parity has completed.  Gives up and
-// returns false after `limit_ns` nanoseconds, or as soon as `abort_word`
-// (a global flag other CTAs set when they give up) has any of `abort_bits`.
+// returns false after `limit_ns` nanoseconds, or, when `abort_value` is
+// nonzero, as soon as the global word `abort_word` equals it (another CTA of
+// the same launch has given up).
 __device__ __forceinline__ bool mbar_wait_ns(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
-                                             const volatile uint32_t* abort_word, uint32_t abort_bits) {
+                                             const volatile uint32_t* abort_word, uint32_t abort_value) {
   if (mbar_test(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (;;) {
@@ -76,7 +68,18 @@ __device__ __forceinline__ bool mbar_wait_ns(uint64_t* bar, uint32_t parity, uin
     for (int i = 0; i < 32; ++i)
       if (mbar_test(bar, parity)) return true;
     if (global_ns() - t0 > limit_ns) return false;
-    if (*abort_word & abort_bits) return false;
+    if (abort_value != 0u && *abort_word == abort_value) return false;
+  }
+}
+
+// Waits (bounded by `limit_ns`, never cut short) for the last phase armed on
+// each of `stages` ring barriers, where `armed` arms have been made so far and
+// arm a went to barrier a mod stages, phase a / stages.  Used before a CTA
+// exits, so no copy it issued is still in flight.
+__device__ __forceinline__ void mbar_drain_ring(uint64_t* bars, int stages, uint32_t armed, uint64_t limit_ns) {
+  for (int back = 1; back <= stages && back <= (int)armed; ++back) {
+    const uint32_t a = armed - back;
+    mbar_wait_ns(&bars[a % stages], (a / stages) & 1, limit_ns, nullptr, 0u);
   }
 }
 
@@ -178,19 +181,6 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_
       : "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem]
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                       uint32_t accumulate) {
-  asm volatile(
-      "{\n"
-      ".reg .pred p;\n"
-      "setp.ne.b32 p, %4, 0;\n"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n"
-      "}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 // Arrives once on `bar` when every tcgen05 operation issued so far by this
 // thread has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
@@ -223,16 +213,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
-}
-
-// 32 lanes x 16 columns: thread t writes lane (base + t), columns [col, col + 16).
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-      "%14, %15, %16};\n" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
 }
 
 // 32 lanes x 32 columns store.

@@ -195,8 +195,11 @@ BSA_API bsa_status bsa_attn_fwd_baseline(const bsa_shape* s, const void* q, cons
  * bytes.  Argument errors are those of bsa_attn_fwd.
  *
  * Set-up: the first call on each device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current).  Make that first call
- * before any stream capture.
+ * (cudaGetSymbolAddress, with that device current) and remembers it with the
+ * current CUDA context.  Make that first call before any stream capture.  A
+ * device reset (cudaDeviceReset, or a context destroyed and created again)
+ * gives the array a new address: the next call notices the new context and
+ * looks the address up again, so it too must come before any capture.
  *
  * Sharing: every call on a device uses the same array.  The call clears the
  * error word at its start and rewrites the plan, so nothing carries over from

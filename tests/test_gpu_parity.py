@@ -259,6 +259,34 @@ def test_forced_timeout_is_reported_and_the_context_stays_usable(bsa, monkeypatc
     assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean)
 
 
+def test_a_timeout_left_by_an_earlier_call_does_not_cut_the_next_call_short(bsa):
+    """The error word is sticky until bsa_check_device_status reads it.  A
+    timeout bit and an abort mark left in the workspace by an earlier call
+    must not make the next mask or attention call give up: its output is the
+    oracle's, and the stale bit is still reported (then cleared) afterwards."""
+    w = small("stale_timeout", 1, 2, 16, 16, 2, 128, 64, 8, 0.2, seed=33)
+    q, k, v = synth.make_qkv(w)
+    plan = bsa.NablaAttention(_shape(bsa, w))
+    for src, dst in ((q, plan.q), (k, plan.k), (v, plan.v)):
+        bsa.reorder(plan.shape, src.cuda(), dst)
+    torch.cuda.synchronize()
+    ctrl = plan.ws[:256].view(torch.int32)
+    ctrl[0] = 4                      # kErrTimeout, as an earlier timed-out call leaves it
+    ctrl[4:5].fill_(-1)              # an abort mark of an earlier launch
+    plan.o.fill_(float("nan"))
+    plan.mask_step(w.thr, w.sta)
+    plan.attention_step()
+    torch.cuda.synchronize()
+    assert plan.status() == 5        # the stale bit is reported once ...
+    assert plan.status() == 0        # ... and cleared
+    keep_ref, amb = oracle.nabla.block_mask(to64(plan.q), to64(plan.k), w.T, w.H, w.W, w.patch, w.block, w.thr)
+    keep = lists_to_keep(plan.kv_count, plan.kv_idx, plan.nb)
+    assert not ((keep != keep_ref) & ~amb).any()
+    O_ref, _ = oracle.masked_attention(to64(plan.q), to64(plan.k), to64(plan.v), keep, w.N, w.block)
+    mx, mean = compare_outputs(to64(plan.o)[:, :, :w.N], O_ref[:, :, :w.N])
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean)
+
+
 # Keys whose scale grows along the key blocks: each row's running max keeps
 # rising as the kernel walks its ascending list, so the lazy rescale of O (a
 # max that grows by more than 8 in log2 units) runs many times per row, in
