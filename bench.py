@@ -42,10 +42,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 def kernel_launches_per_step(w) -> int:
-    """Our kernels in one step: reorder x3, pool + mask (adaptive workloads),
-    plan (overlap + matching with 64-token blocks, one kernel with 128),
-    attention, inverse reorder."""
-    return 3 + (0 if w.iid else 2) + (2 if w.block == 64 else 1) + 1 + 1
+    """Our kernels in one step: the Q/K reorder with block pooling, V's
+    reorder, the mask (adaptive workloads), the plan (overlap + matching with
+    64-token blocks, one kernel with 128), attention, inverse reorder."""
+    return 2 + (0 if w.iid else 1) + (2 if w.block == 64 else 1) + 1 + 1
 
 
 # ------------------------------------------------------------------ helpers
@@ -326,19 +326,22 @@ def run_ours(args, w, rank, world, dist):
     ev = lambda: torch.cuda.Event(enable_timing=True)
 
     def step(times=None):
-        e = [ev() for _ in range(5)] if times is not None else None
+        # events on the launching stream: 0 | Q/K reorder + pooling | 1 | mask | 2 |
+        # wait for V's reorder (side stream, overlapping the mask) | 3 | attention | 4 | inverse | 5
+        e = [ev() for _ in range(6)] if times is not None else None
         if e: e[0].record(stream)
-        plan.reorder_inputs(qd, kd, vd)     # V on the side stream, overlapping the mask
+        plan.reorder_inputs(qd, kd, vd)
         if e: e[1].record(stream)
         if not w.iid:
             plan.mask_step(w.thr, w.sta)
-        plan.join_side()
         if e: e[2].record(stream)
-        plan.attention_step(baseline=args.baseline_kernel)
+        plan.join_side()
         if e: e[3].record(stream)
+        plan.attention_step(baseline=args.baseline_kernel)
+        if e: e[4].record(stream)
         bsa.inverse_reorder(shape, plan.o, out)
         if e:
-            e[4].record(stream)
+            e[5].record(stream)
             times.append(e)
 
     for _ in range(args.warmup):
@@ -361,14 +364,14 @@ def run_ours(args, w, rank, world, dist):
         torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
-    parts = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in events])  # ms
+    parts = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(5)] for e in events])  # ms
     step_ms = float(parts.sum(axis=1).sum())   # total over K steps
     t_max = max_over_ranks(step_ms, dist, dev)
     total_flops = flops_step * args.steps * world
     value = total_flops / (t_max * 1e-3) / 1e12
     ms_per_step = t_max / args.steps
     br = parts.mean(axis=0)
-    attn_ms = float(br[2])
+    attn_ms = float(br[3])
 
     # ---- end to end through the public API with host buffers: every step
     # copies its Q, K, V from pinned host memory and its output back to pinned
@@ -441,12 +444,21 @@ def run_ours(args, w, rank, world, dist):
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     attn_tf = flops_step / (attn_ms * 1e-3) / 1e12
     traffic = recorded_traffic("attn", w.name)
-    qk_bytes = 2 * w.B * w.heads * w.N * w.d * 2
+    # algorithmic bytes: the fused Q/K pass reads Q and K once, writes them
+    # reordered (zero tail included) and writes the block means; the mask
+    # kernel reads the means and writes the lists; V's reorder moves V
+    tok_bytes = w.B * w.heads * w.N * w.d * 2
+    pad_bytes = w.B * w.heads * (plan.Npad - w.N) * w.d * 2
+    means_bytes = 2 * w.B * w.heads * plan.nb * w.d * 8
     kept = float(plan.kv_count.sum().item())
-    mask_bytes = qk_bytes + 2 * 2 * w.B * w.heads * plan.nb * w.d * 8 + 4 * (kept + w.B * w.heads * plan.nb)
-    mask_ms = float(br[1])
-    # the reorder_qk part moves Q and K (V's reorder overlaps the mask stage on a side stream)
-    reorder_bytes = 2 * 2 * (w.B * w.heads * w.N * w.d * 2) + 2 * 2 * w.B * w.heads * (plan.Npad - w.N) * w.d
+    qk_pool_bytes = 2 * (2 * tok_bytes + pad_bytes) + means_bytes
+    mask_kernel_bytes = means_bytes + 4 * (kept + w.B * w.heads * plan.nb)
+    v_bytes = 2 * tok_bytes + pad_bytes
+    qk_ms, mask_ms, vjoin_ms = float(br[0]), float(br[1]), float(br[2])
+    gbs = lambda nbytes, ms: nbytes / (ms * 1e-3) / 1e9 if ms > 0 else None
+    mask_gbs = gbs(qk_pool_bytes + mask_kernel_bytes, qk_ms + mask_ms)
+    stage_gbs = gbs(qk_pool_bytes + mask_kernel_bytes + v_bytes, qk_ms + mask_ms + vjoin_ms)
+    reduced_flops = 2.0 * w.B * w.heads * plan.nb * plan.nb * w.d
     cpu, mask_report = None, {}
     if args.cpu_baseline and world == 1:
         gpu_keep = lists_to_keep(plan.kv_count.cpu().numpy(), plan.kv_idx.cpu().numpy(), plan.nb)
@@ -463,17 +475,24 @@ def run_ours(args, w, rank, world, dist):
             "attn_kernel": "mma.sync (legacy baseline)" if args.baseline_kernel else "tcgen05",
             "l2": "flushed between steps (write of a 2x L2 buffer, outside the step events)",
             "attn_ms": attn_ms, "attn_tflops": attn_tf, "attn_pct_bf16_peak": 100.0 * attn_tf / peak_tf,
-            "breakdown_ms": {"reorder_qk": float(br[0]), "mask_and_reorder_v": mask_ms, "attn": attn_ms,
-                             "inverse_reorder": float(br[3])},
-            "mask_gbs": mask_bytes / (mask_ms * 1e-3) / 1e9 if mask_ms > 0 else None,
-            "mask_pct_hbm": 100.0 * mask_bytes / (mask_ms * 1e-3) / 1e9 / hbm if mask_ms > 0 else None,
-            "reorder_gbs": reorder_bytes / (float(br[0]) * 1e-3) / 1e9,
+            "breakdown_ms": {"reorder_pool_qk": qk_ms, "mask": mask_ms, "wait_reorder_v": vjoin_ms, "attn": attn_ms,
+                             "inverse_reorder": float(br[4])},
+            "reorder_pool_qk_gbs": gbs(qk_pool_bytes, qk_ms),
+            "reorder_pool_qk_pct_hbm": 100.0 * gbs(qk_pool_bytes, qk_ms) / hbm,
+            "mask_kernel_f64_tflops": reduced_flops / (mask_ms * 1e-3) / 1e12 if mask_ms > 0 else None,
+            # mask construction: the fused Q/K reorder + pooling and the mask kernel
+            "mask_gbs": mask_gbs,
+            "mask_pct_hbm": 100.0 * mask_gbs / hbm if mask_gbs else None,
+            # the whole stage before attention: the above with V's reorder overlapping the mask kernel
+            "mask_stage_gbs": stage_gbs,
+            "mask_stage_pct_hbm": 100.0 * stage_gbs / hbm if stage_gbs else None,
+            "inverse_reorder_gbs": gbs(v_bytes - pad_bytes, float(br[4])),
             "mask_precision": "f64 pooled means, dots and masses",
             **mask_report,
             "step_ms_median": float(np.median(parts.sum(axis=1))),
             "step_ms_min": float(parts.sum(axis=1).min()),
-            "attn_ms_median": float(np.median(parts[:, 2])),
-            "attn_ms_min": float(parts[:, 2].min()),
+            "attn_ms_median": float(np.median(parts[:, 3])),
+            "attn_ms_min": float(parts[:, 3].min()),
         },
         "roofline": {"bound": "tensor", "achieved": attn_tf, "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": attn_tf / peak_tf, "traffic": traffic,

@@ -17,8 +17,8 @@ from typing import Optional, Tuple
 
 import torch
 
-from ._lib import (BsaError, Shape, attn_fwd, attn_fwd_baseline, build_block_mask, check_device_status, inverse_reorder,  # noqa: F401
-                   get_lib, make_shape, num_blocks, padded_len, reorder, seq_len, validate_shape, workspace_bytes,
+from ._lib import (BsaError, Shape, attn_fwd, attn_fwd_baseline, build_block_mask, build_block_mask_pooled,  # noqa: F401
+                   check_device_status, inverse_reorder, reorder_qk_pooled, get_lib, make_shape, num_blocks, padded_len, reorder, seq_len, validate_shape, workspace_bytes,
                    workspace_init, LIB_PATH)
 
 def __getattr__(name):
@@ -29,16 +29,18 @@ def __getattr__(name):
 
 
 __all__ = ["BsaError", "Shape", "make_shape", "NablaAttention", "reorder", "inverse_reorder", "build_block_mask",
+           "reorder_qk_pooled", "build_block_mask_pooled",
            "attn_fwd", "attn_fwd_baseline", "check_device_status", "workspace_bytes", "workspace_init", "padded_len", "num_blocks",
            "seq_len", "validate_shape", "get_lib", "LIB_PATH"]
 
 
 class NablaAttention:
     """Owns the device buffers of one shape and runs the whole path: reorder
-    Q, K, V -> block mask -> block-sparse attention -> inverse reorder, ordered
-    on the current stream.  V's reorder runs on a side stream, concurrently
-    with the block mask (which needs only Q and K); the attention waits for
-    both.  Buffers are allocated once (torch) and reused."""
+    Q and K with their block means -> block mask -> block-sparse attention ->
+    inverse reorder, ordered on the current stream.  V's reorder runs on a
+    side stream after the Q/K reorder, concurrently with the block mask (which
+    needs only Q and K); the attention waits for both.  Buffers are allocated
+    once (torch) and reused."""
 
     def __init__(self, shape: Shape, device="cuda", with_mask: bool = False, with_lse: bool = False):
         st = validate_shape(shape)
@@ -64,11 +66,13 @@ class NablaAttention:
         self.side = torch.cuda.Stream(device=dev)
 
     def reorder_inputs(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor) -> None:
-        """Q and K on the current stream, V on the side stream (joined by
+        """Q and K in one launch on the current stream, with their block means
+        kept in the workspace for mask_step; V on the side stream (joined by
         join_side before the attention)."""
         main = torch.cuda.current_stream(q.device)
-        reorder(self.shape, q, self.q)
-        reorder(self.shape, k, self.k)
+        reorder_qk_pooled(self.shape, q, k, self.q, self.k, self.ws)
+        # V after the Q/K launch: its reorder then overlaps the (compute-bound)
+        # mask kernel rather than sharing HBM with the Q/K pass
         self.side.wait_stream(main)
         with torch.cuda.stream(self.side):
             reorder(self.shape, v, self.v)
@@ -77,7 +81,8 @@ class NablaAttention:
         torch.cuda.current_stream(self.q.device).wait_stream(self.side)
 
     def mask_step(self, thr: float, sta: Optional[Tuple[int, int, int]] = None) -> None:
-        build_block_mask(self.shape, self.q, self.k, thr, sta, self.kv_count, self.kv_idx, self.mask, self.ws)
+        """The block mask from the block means reorder_inputs left in the workspace."""
+        build_block_mask_pooled(self.shape, thr, sta, self.kv_count, self.kv_idx, self.mask, self.ws)
 
     def attention_step(self, scale: float = 0.0, baseline: bool = False) -> None:
         fn = attn_fwd_baseline if baseline else attn_fwd

@@ -55,6 +55,9 @@ def _load() -> ctypes.CDLL:
         "bsa_inverse_reorder": (st, [S, P, P, P]),
         "bsa_build_block_mask": (st, [S, P, P, ctypes.c_float, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                       P, P, P, P, ctypes.c_size_t, P]),
+        "bsa_reorder_qk_pooled": (st, [S, P, P, P, P, P, ctypes.c_size_t, P]),
+        "bsa_build_block_mask_pooled": (st, [S, ctypes.c_float, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                             P, P, P, P, ctypes.c_size_t, P]),
         "bsa_attn_fwd": (st, [S, P, P, P, P, P, ctypes.c_float, P, P, P, ctypes.c_size_t, P]),
         "bsa_attn_fwd_baseline": (st, [S, P, P, P, P, P, ctypes.c_float, P, P, P, ctypes.c_size_t, P]),
         "bsa_check_device_status": (st, [P, P]),
@@ -147,6 +150,22 @@ def build_block_mask(s: Shape, q_bhnd: torch.Tensor, k_bhnd: torch.Tensor, thr: 
                                     _ptr(kv_count), _ptr(kv_idx), _ptr(mask), _ptr(ws),
                                     ws.numel() * ws.element_size(), _stream(q_bhnd.device)),
            "bsa_build_block_mask")
+
+
+def reorder_qk_pooled(s: Shape, q_bnhd: torch.Tensor, k_bnhd: torch.Tensor, q_bhnd: torch.Tensor,
+                      k_bhnd: torch.Tensor, ws: torch.Tensor) -> None:
+    _check(get_lib().bsa_reorder_qk_pooled(ctypes.byref(s), _ptr(q_bnhd), _ptr(k_bnhd), _ptr(q_bhnd), _ptr(k_bhnd),
+                                           _ptr(ws), ws.numel() * ws.element_size(), _stream(q_bnhd.device)),
+           "bsa_reorder_qk_pooled")
+
+
+def build_block_mask_pooled(s: Shape, thr: float, sta: Optional[Tuple[int, int, int]], kv_count: torch.Tensor,
+                            kv_idx: torch.Tensor, mask: Optional[torch.Tensor], ws: torch.Tensor) -> None:
+    st_t, st_h, st_w = sta if sta is not None else (-1, -1, -1)
+    _check(get_lib().bsa_build_block_mask_pooled(ctypes.byref(s), float(thr), st_t, st_h, st_w, _ptr(kv_count),
+                                                 _ptr(kv_idx), _ptr(mask), _ptr(ws), ws.numel() * ws.element_size(),
+                                                 _stream(kv_count.device)),
+           "bsa_build_block_mask_pooled")
 
 
 def attn_fwd(s: Shape, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, kv_count: torch.Tensor,

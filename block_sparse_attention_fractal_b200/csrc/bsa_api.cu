@@ -122,6 +122,39 @@ bsa_status bsa_inverse_reorder(const bsa_shape* s, const void* y_bhnd, void* x_b
   return from_cuda(bsa::launch_inverse_reorder(g, y_bhnd, x_bnhd, (cudaStream_t)stream));
 }
 
+bsa_status bsa_reorder_qk_pooled(const bsa_shape* s, const void* q_bnhd, const void* k_bnhd, void* q_bhnd,
+                                 void* k_bhnd, void* workspace, size_t ws_bytes, bsa_stream_t stream) {
+  Dims g;
+  bsa_status st = check_shape(s, &g);
+  if (st != BSA_OK) return st;
+  const void* ptrs[5] = {q_bnhd, k_bnhd, q_bhnd, k_bhnd, workspace};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return BSA_ERR_INVALID_ARG;
+  if (q_bnhd == q_bhnd || k_bnhd == k_bhnd || q_bhnd == k_bhnd) return BSA_ERR_INVALID_ARG;
+  if (ws_bytes < workspace_bytes(g)) return BSA_ERR_INVALID_ARG;
+  double* qbar = (double*)((char*)workspace + sizeof(Ctrl));
+  double* kbar = qbar + pooled_bytes(g) / sizeof(double);
+  return from_cuda(bsa::launch_reorder_qk_pool(g, q_bnhd, k_bnhd, q_bhnd, k_bhnd, qbar, kbar, (cudaStream_t)stream));
+}
+
+bsa_status bsa_build_block_mask_pooled(const bsa_shape* s, float thr, int32_t sta_t, int32_t sta_h, int32_t sta_w,
+                                       int32_t* kv_count, int32_t* kv_idx, uint8_t* mask_or_null, void* workspace,
+                                       size_t ws_bytes, bsa_stream_t stream) {
+  Dims g;
+  bsa_status st = check_shape(s, &g);
+  if (st != BSA_OK) return st;
+  if (g.nb > BSA_MAX_BLOCKS) return BSA_ERR_UNSUPPORTED;
+  if (!(thr >= 0.0f && thr < 1.0f)) return BSA_ERR_INVALID_ARG;
+  if (kv_count == nullptr || kv_idx == nullptr || workspace == nullptr) return BSA_ERR_INVALID_ARG;
+  if (!aligned16(kv_count) || !aligned16(kv_idx) || !aligned16(workspace)) return BSA_ERR_INVALID_ARG;
+  if (ws_bytes < workspace_bytes(g)) return BSA_ERR_INVALID_ARG;
+  const bool sta = sta_t >= 0 && sta_h >= 0 && sta_w >= 0;
+  double* qbar = (double*)((char*)workspace + sizeof(Ctrl));
+  double* kbar = qbar + pooled_bytes(g) / sizeof(double);
+  return from_cuda(bsa::launch_mask(g, qbar, kbar, (double)thr, sta ? sta_t : -1, sta ? sta_h : -1, sta ? sta_w : -1,
+                                    kv_count, kv_idx, mask_or_null, (cudaStream_t)stream));
+}
+
 bsa_status bsa_build_block_mask(const bsa_shape* s, const void* q_bhnd, const void* k_bhnd, float thr,
                                 int32_t sta_t, int32_t sta_h, int32_t sta_w, int32_t* kv_count, int32_t* kv_idx,
                                 uint8_t* mask_or_null, void* workspace, size_t ws_bytes, bsa_stream_t stream) {

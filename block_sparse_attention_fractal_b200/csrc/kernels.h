@@ -13,6 +13,10 @@ uint32_t next_launch_seq();
 
 cudaError_t launch_reorder(const Dims& g, const void* x_bnhd, void* y_bhnd, cudaStream_t st);
 cudaError_t launch_inverse_reorder(const Dims& g, const void* y_bhnd, void* x_bnhd, cudaStream_t st);
+// Q and K reordered in one launch, their block means written on the way:
+// `qbar` [B, heads, nb, d], `kbar` transposed [B, heads, d, nb] (double).
+cudaError_t launch_reorder_qk_pool(const Dims& g, const void* q_bnhd, const void* k_bnhd, void* q_bhnd,
+                                   void* k_bhnd, double* qbar, double* kbar, cudaStream_t st);
 
 // Block means of Q and K (double): `qbar` [B, heads, nb, d], `kbar`
 // transposed [B, heads, d, nb].

@@ -133,6 +133,31 @@ BSA_API bsa_status bsa_build_block_mask(const bsa_shape* s, const void* q_bhnd, 
                                 int32_t* kv_count, int32_t* kv_idx, uint8_t* mask_or_null,
                                 void* workspace, size_t ws_bytes, bsa_stream_t stream);
 
+/* Reorder of Q and K (as bsa_reorder, one launch for both) fused with the
+ * first step of the adaptive mask, NABLA summary, Metodologia 2
+ * "Submuestreo": on the way, the mean of the valid tokens of every block of Q
+ * and of K is computed in double and kept in the workspace, where
+ * bsa_build_block_mask_pooled reads it.  Q and K are then read from HBM once
+ * for both the reorder and the pooling.
+ *   q_bnhd, k_bnhd: device, [B, N, heads, d] bf16 model order, read only.
+ *   q_bhnd, k_bhnd: device, [B, heads, Npad, d] bf16 kernel order, written
+ *       (zero tail); neither may overlap an input or the other output.
+ *   workspace / ws_bytes: at least bsa_workspace_bytes(s); its pooled-mean
+ *       region is overwritten. */
+BSA_API bsa_status bsa_reorder_qk_pooled(const bsa_shape* s, const void* q_bnhd, const void* k_bnhd, void* q_bhnd,
+                                         void* k_bhnd, void* workspace, size_t ws_bytes, bsa_stream_t stream);
+
+/* bsa_build_block_mask from the block means that bsa_reorder_qk_pooled left
+ * in `workspace` (same rule, arguments and outputs otherwise): the reduced
+ * attention, the CDF threshold and the optional STA union, NABLA summary,
+ * Metodologia 2 ("Atencion Reducida", "Umbralizacion CDF", "Expansion") and 3.
+ * Must follow bsa_reorder_qk_pooled of the same shape on the same workspace
+ * (stream order). */
+BSA_API bsa_status bsa_build_block_mask_pooled(const bsa_shape* s, float thr, int32_t sta_t, int32_t sta_h,
+                                               int32_t sta_w, int32_t* kv_count, int32_t* kv_idx,
+                                               uint8_t* mask_or_null, void* workspace, size_t ws_bytes,
+                                               bsa_stream_t stream);
+
 /* Block-sparse attention forward, NABLA summary, Metodologia 2 "Expansion":
  * for every valid query row q of block I,
  *   O[q] = sum_k softmax_k(scale * Q[q] . K[k]) V[k],

@@ -54,11 +54,25 @@ def _shape(bsa, w):
     return bsa.make_shape(w.B, w.T, w.H, w.W, w.heads, w.d, w.block, w.patch)
 
 
-def _run_mask(bsa, w, plan, q, k):
-    bsa.reorder(plan.shape, q, plan.q)
-    bsa.reorder(plan.shape, k, plan.k)
-    plan.mask_step(w.thr, w.sta)
+def _run_mask(bsa, w, plan, q, k, fused=True):
+    """The block mask of q, k (model order) into the plan's lists: the fused
+    path (Q/K reorder with the block means, then the mask from those means)
+    or the separate one (reorder, then pooling and mask from the reordered
+    tensors)."""
+    if fused:
+        bsa.reorder_qk_pooled(plan.shape, q, k, plan.q, plan.k, plan.ws)
+        plan.mask_step(w.thr, w.sta)
+    else:
+        bsa.reorder(plan.shape, q, plan.q)
+        bsa.reorder(plan.shape, k, plan.k)
+        bsa.build_block_mask(plan.shape, plan.q, plan.k, w.thr, w.sta, plan.kv_count, plan.kv_idx, plan.mask,
+                             plan.ws)
     torch.cuda.synchronize()
+
+
+def _reorder_all(bsa, plan, q, k, v):
+    bsa.reorder_qk_pooled(plan.shape, q.cuda(), k.cuda(), plan.q, plan.k, plan.ws)
+    bsa.reorder(plan.shape, v.cuda(), plan.v)
 
 
 @pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
@@ -78,10 +92,36 @@ def test_reorder_bit_exact(bsa, w):
 
 
 @pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
-def test_block_mask_matches_oracle(bsa, w):
+def test_fused_qk_reorder_and_block_means(bsa, w):
+    """bsa_reorder_qk_pooled: both reorders bit-exact, and the block means it
+    leaves in the workspace equal the oracle's (sums of bf16 values in double
+    are exact here, so the means agree to the last bit)."""
+    q, k, _ = synth.make_qkv(w)
+    s = _shape(bsa, w)
+    Npad, nb = bsa.padded_len(s), bsa.num_blocks(s)
+    yq = torch.full((w.B, w.heads, Npad, w.d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    yk = torch.full_like(yq, float("nan"))
+    ws = torch.full(((bsa.workspace_bytes(s) + 15) // 16 * 16,), 0xFF, dtype=torch.uint8, device="cuda")
+    bsa.workspace_init(ws)
+    bsa.reorder_qk_pooled(s, q.cuda(), k.cuda(), yq, yk, ws)
+    torch.cuda.synchronize()
+    want_q = oracle.reorder(to64(q), w.T, w.H, w.W, w.patch, w.block)
+    want_k = oracle.reorder(to64(k), w.T, w.H, w.W, w.patch, w.block)
+    assert np.array_equal(to64(yq), want_q) and np.array_equal(to64(yk), want_k)
+    n = w.B * w.heads * nb * w.d
+    means = ws[256:256 + 16 * n].view(torch.float64).cpu().numpy()
+    qbar = means[:n].reshape(w.B, w.heads, nb, w.d)
+    kbar = means[n:].reshape(w.B, w.heads, w.d, nb).swapaxes(-1, -2)
+    assert np.array_equal(qbar, oracle.block_means(want_q, w.N, w.block))
+    assert np.array_equal(kbar, oracle.block_means(want_k, w.N, w.block))
+
+
+@pytest.mark.parametrize("fused", [True, False], ids=["fused_pool", "separate_pool"])
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_block_mask_matches_oracle(bsa, w, fused):
     q, k, _ = synth.make_qkv(w)
     plan = bsa.NablaAttention(_shape(bsa, w), with_mask=True)
-    _run_mask(bsa, w, plan, q.cuda(), k.cuda())
+    _run_mask(bsa, w, plan, q.cuda(), k.cuda(), fused)
     assert plan.status() == 0
     keep_ref, amb = oracle.block_mask(to64(plan.q), to64(plan.k), w.T, w.H, w.W, w.patch, w.block, w.thr, w.sta)
     keep = lists_to_keep(plan.kv_count, plan.kv_idx, plan.nb)
@@ -243,8 +283,7 @@ def test_forced_timeout_is_reported_and_the_context_stays_usable(bsa, monkeypatc
     w = small("forced_timeout", 1, 2, 16, 16, 2, 128, 64, 8, 0.2, seed=31)
     q, k, v = synth.make_qkv(w)
     plan = bsa.NablaAttention(_shape(bsa, w))
-    for src, dst in ((q, plan.q), (k, plan.k), (v, plan.v)):
-        bsa.reorder(plan.shape, src.cuda(), dst)
+    _reorder_all(bsa, plan, q, k, v)
     plan.mask_step(w.thr, w.sta)
     monkeypatch.setenv("BSA_TEST_FORCE_TIMEOUT", "1")
     plan.attention_step()
@@ -267,14 +306,14 @@ def test_a_timeout_left_by_an_earlier_call_does_not_cut_the_next_call_short(bsa)
     w = small("stale_timeout", 1, 2, 16, 16, 2, 128, 64, 8, 0.2, seed=33)
     q, k, v = synth.make_qkv(w)
     plan = bsa.NablaAttention(_shape(bsa, w))
-    for src, dst in ((q, plan.q), (k, plan.k), (v, plan.v)):
-        bsa.reorder(plan.shape, src.cuda(), dst)
+    _reorder_all(bsa, plan, q, k, v)
     torch.cuda.synchronize()
     ctrl = plan.ws[:256].view(torch.int32)
     ctrl[0] = 4                      # kErrTimeout, as an earlier timed-out call leaves it
     ctrl[4:5].fill_(-1)              # an abort mark of an earlier launch
     plan.o.fill_(float("nan"))
-    plan.mask_step(w.thr, w.sta)
+    # the separate pooling path: its bulk-copy waits and the attention's both run
+    bsa.build_block_mask(plan.shape, plan.q, plan.k, w.thr, w.sta, plan.kv_count, plan.kv_idx, None, plan.ws)
     plan.attention_step()
     torch.cuda.synchronize()
     assert plan.status() == 5        # the stale bit is reported once ...

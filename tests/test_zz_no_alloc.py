@@ -57,8 +57,8 @@ def test_noalloc_matches_workspace_entry_point_twice_in_a_row(w):
     fn = _fn(bsa.lib)
     q, k, v = synth.make_qkv(w)
     plan = bsa.NablaAttention(bsa.make_shape(w.B, w.T, w.H, w.W, w.heads, w.d, w.block, w.patch), with_lse=True)
-    for src, dst in ((q, plan.q), (k, plan.k), (v, plan.v)):
-        bsa.reorder(plan.shape, src.cuda(), dst)
+    bsa.reorder_qk_pooled(plan.shape, q.cuda(), k.cuda(), plan.q, plan.k, plan.ws)
+    bsa.reorder(plan.shape, v.cuda(), plan.v)
     plan.mask_step(w.thr, w.sta)
     plan.attention_step()                     # the workspace entry point: the expected output
     torch.cuda.synchronize()
