@@ -4,6 +4,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 
 #include "common.cuh"
@@ -13,6 +14,15 @@ using bsa::Ctrl;
 using bsa::Dims;
 
 namespace bsa {
+
+cudaError_t launch_attn(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
+                        const int32_t* kv_idx, const int2* items, int* work, float scale, void* o, float* lse,
+                        Ctrl* ctrl, uint32_t seq, cudaStream_t st) {
+  const char* pick = std::getenv("BSA_ATTN_KERNEL");
+  if (pick != nullptr && std::strcmp(pick, "tc2") == 0)
+    return launch_attn_tc2(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, seq, st);
+  return launch_attn_tc3(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, seq, st);
+}
 
 uint32_t next_launch_seq() {
   static std::atomic<uint32_t> counter{0};
@@ -207,8 +217,8 @@ bsa_status attn_common(const bsa_shape* s, const void* q, const void* k, const v
   int2* items = (int2*)((char*)workspace + plan_offset(g));
   cudaError_t e = bsa::launch_plan(g, kv_count, kv_idx, items, (cudaStream_t)stream);
   if (e != cudaSuccess) return BSA_ERR_CUDA;
-  return from_cuda(bsa::launch_attn_tc2(g, q, k, v, kv_count, kv_idx, items, bsa::plan_work_counter(g, items), scale,
-                                       o, lse_or_null, ctrl, bsa::next_launch_seq(), (cudaStream_t)stream));
+  return from_cuda(bsa::launch_attn(g, q, k, v, kv_count, kv_idx, items, bsa::plan_work_counter(g, items), scale, o,
+                                   lse_or_null, ctrl, bsa::next_launch_seq(), (cudaStream_t)stream));
 }
 
 }  // namespace

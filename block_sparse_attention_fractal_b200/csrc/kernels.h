@@ -45,6 +45,14 @@ cudaError_t launch_plan(const Dims& g, const int32_t* kv_count, const int32_t* k
 // Block-sparse attention on the tcgen05 tensor cores (TMEM accumulators,
 // TMA-staged tiles): persistent, one CTA per SM, two softmax groups on
 // alternating KV tiles, query tiles fetched from the plan's work counter.
+// tc2 stages P in shared memory, tc3 in tensor memory; launch_attn picks the
+// kernel the entry points use.
+cudaError_t launch_attn(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
+                        const int32_t* kv_idx, const int2* items, int* work, float scale, void* o, float* lse,
+                        Ctrl* ctrl, uint32_t seq, cudaStream_t st);
+cudaError_t launch_attn_tc3(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
+                            const int32_t* kv_idx, const int2* items, int* work, float scale, void* o, float* lse,
+                            Ctrl* ctrl, uint32_t seq, cudaStream_t st);
 cudaError_t launch_attn_tc2(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
                             const int32_t* kv_idx, const int2* items, int* work, float scale, void* o, float* lse,
                             Ctrl* ctrl, uint32_t seq, cudaStream_t st);

@@ -136,15 +136,14 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __nv_bfloat16*
 
 // ------------------------------------------------------------- mask rows
 
-constexpr int kMaskRows = 16;                 // query-block rows per CTA (one warp each)
-constexpr int kMaskThreads = 32 * kMaskRows;  // 512
+constexpr int kMaskThreads = 256;             // 8 warps
+constexpr int kMaskWarps = kMaskThreads / 32;
+// Query-block rows per CTA: 16, or 8 when rows are longer than 512 blocks
+// (the CTA's scores then stay at 64 KB of shared memory, two CTAs per SM).
+template <int NJ>
+constexpr int mask_rows() { return NJ <= 16 ? 16 : 8; }
 
 __device__ __forceinline__ double warp_sum(double v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-__device__ __forceinline__ int warp_sum(int v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
@@ -162,6 +161,25 @@ __device__ __forceinline__ unsigned long long warp_max(unsigned long long v) {
   }
   return v;
 }
+__device__ __forceinline__ unsigned long long warp_min(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long w = __shfl_xor_sync(0xffffffffu, v, o);
+    v = w < v ? w : v;
+  }
+  return v;
+}
+
+// A probability in fixed point, units of 2^-52, in bits 11-63, and a count of
+// one in bits 0-10: sums of up to 1024 of these add both fields at once
+// without carrying from one into the other (the masses of a row sum to
+// about 2^52 < 2^53).  Rounding each probability to 2^-53 moves a row's
+// prefix masses by less than 1024 * 2^-53 = 1.1e-13, far inside the 1e-6
+// window within which a threshold decision counts as ambiguous.
+constexpr double kMassScale = 4503599627370496.0;   // 2^52
+__device__ __forceinline__ unsigned long long packed_mass(double a) {
+  return (__double2ull_rn(a * kMassScale) << 11) | 1ull;
+}
 
 __device__ __forceinline__ void block_tile(int I, const Dims& g, int& t, int& th, int& tw) {
   const int n = fractal_token(I * g.bs, g.H, g.W, g.P);
@@ -173,245 +191,306 @@ __device__ __forceinline__ void block_tile(int I, const Dims& g, int& t, int& th
   tw = (rem - h * g.W) / g.P;
 }
 
-// Persistent grid: CTA c handles the groups of kMaskRows rows c, c + gridDim.x,
-// ... of all (b, head).  Dynamic smem: qbar rows [kMaskRows][D] then scores
-// [kMaskRows][nb], both double.  NJ = ceil(nb / 32) rounded up to a power of
-// two: the values of a row that each lane holds in phase 2.
+// Persistent grid: CTA c handles the groups of R rows c, c + gridDim.x, ...
+// of all (b, head).  Dynamic shared memory: qbar rows [R][D], scores [R][nb]
+// (double), then a 256-bucket histogram per warp (uint64).  NJ = ceil(nb / 32)
+// rounded up to a power of two: the values of a row that each lane holds.
 template <int D, int NJ>
-__global__ void __launch_bounds__(kMaskThreads) mask_kernel(const double* __restrict__ qbar,
-                                                            const double* __restrict__ kbar, Dims g, double thr,
-                                                            double scale, int sta_t, int sta_h, int sta_w,
-                                                            int32_t* __restrict__ kv_count,
-                                                            int32_t* __restrict__ kv_idx, uint8_t* __restrict__ mask) {
-  constexpr int kMaxJ = NJ;
+__global__ void __launch_bounds__(kMaskThreads, 2) mask_kernel(const double* __restrict__ qbar,
+                                                               const double* __restrict__ kbar, Dims g, double thr,
+                                                               double scale, int sta_t, int sta_h, int sta_w,
+                                                               int32_t* __restrict__ kv_count,
+                                                               int32_t* __restrict__ kv_idx,
+                                                               uint8_t* __restrict__ mask) {
+  constexpr int R = mask_rows<NJ>();
+  constexpr int MT = R / 8;                                    // 8-row MMA tiles
   extern __shared__ __align__(16) double smem[];
-  double* qs = smem;                       // [kMaskRows][D]
-  double* sc = smem + kMaskRows * D;       // [kMaskRows][nb]
+  double* qs = smem;                                           // [R][D]
+  double* sc = smem + R * D;                                   // [R][nb]
   const int nb = g.nb;
-  const int groups = (nb + kMaskRows - 1) / kMaskRows;
+  unsigned long long* hist = reinterpret_cast<unsigned long long*>(sc + R * nb);   // [warps][256]
+  const int groups = (nb + R - 1) / R;
   const int total = groups * g.B * g.heads;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  unsigned long long* my_hist = hist + wid * 256;
+  const unsigned long long target = __double2ull_rn((1.0 - thr) * kMassScale);
+
   for (int grp = blockIdx.x; grp < total; grp += gridDim.x) {
-  const size_t bh = (size_t)(grp / groups);
-  const int I0 = (grp % groups) * kMaskRows;
-  const int rows = min(kMaskRows, nb - I0);
+    const size_t bh = (size_t)(grp / groups);
+    const int I0 = (grp % groups) * R;
+    const int rows = min(R, nb - I0);
 
-  for (int i = threadIdx.x; i < kMaskRows * D; i += kMaskThreads) {
-    const int r = i / D;
-    qs[i] = (r < rows) ? qbar[(bh * nb + I0 + r) * D + (i % D)] : 0.0;
-  }
-  __syncthreads();
+    for (int i = threadIdx.x; i < R * D; i += kMaskThreads) {
+      const int r = i / D;
+      qs[i] = (r < rows) ? qbar[(bh * nb + I0 + r) * D + (i % D)] : 0.0;
+    }
+    __syncthreads();
 
-  // Phase 1: scores s[r][J] = scale * qbar_r . kbar_J on the fp64 tensor
-  // cores (mma.sync m8n8k4, fp64 multiply-add): warp w computes both 8-row
-  // halves of the CTA's rows against the 8-column tiles w, w + 16, ... of J.
-  // A fragments (qbar rows) come from shared memory, B fragments from the
-  // transposed kbar [bh][d][nb] in global memory (64 contiguous bytes per
-  // fragment row).
-  {
-    constexpr int kWarps = kMaskThreads / 32;
-    constexpr int NT = (NJ * 32 / 8 + kWarps - 1) / kWarps;   // 8-column tiles per warp
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    const int gq = lane >> 2, tq = lane & 3;                   // fragment row / column group
-    const double* kt = kbar + bh * D * (size_t)nb;
-    double acc[2][NT][2];
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int n = 0; n < NT; ++n) acc[mt][n][0] = acc[mt][n][1] = 0.0;
-    // B fragments are loaded PD k-steps ahead of their use (a register ring),
-    // so the L2 latency of kbar overlaps the MMAs of the steps in between.
-    constexpr int PD = (NT <= 4) ? 4 : 2;
-    constexpr int KS = D / 4;                                  // k-steps of 4
-    double bq[PD][NT];
-    auto load_b = [&](int ks, double (&dst)[NT]) {
-#pragma unroll
-      for (int n = 0; n < NT; ++n) {
-        const int J = (wid + n * kWarps) * 8 + gq;
-        dst[n] = (J < nb) ? __ldg(kt + (size_t)(4 * ks + tq) * nb + J) : 0.0;
-      }
-    };
-#pragma unroll
-    for (int p = 0; p < PD; ++p) load_b(p, bq[p]);
+    // Phase 1: scores s[r][J] = scale * qbar_r . kbar_J on the fp64 tensor
+    // cores (mma.sync m8n8k4, fp64 multiply-add): warp w computes the R rows
+    // against the 8-column tiles w, w + 8, ... of J.  A fragments (qbar rows)
+    // come from shared memory, B fragments from the transposed kbar
+    // [bh][d][nb] in global memory (64 contiguous bytes per fragment row),
+    // loaded PD k-steps ahead of their use.
+    // (in passes of at most 8 column tiles, so the accumulators and the B
+    // prefetch fit in registers for long rows)
+    {
+      constexpr int NTW = NJ / 2;                                // 8-column tiles per warp
+      constexpr int NT = NTW < 8 ? NTW : 8;                      // ... per pass
+      const int gq = lane >> 2, tq = lane & 3;
+      const double* kt = kbar + bh * D * (size_t)nb;
 #pragma unroll 1
-    for (int ks0 = 0; ks0 < KS; ks0 += PD) {
+      for (int pass = 0; pass < NTW / NT; ++pass) {
+        double acc[MT][NT][2];
 #pragma unroll
-      for (int p = 0; p < PD; ++p) {
-        const int ks = ks0 + p;
-        const double a0 = qs[gq * D + 4 * ks + tq];
-        const double a1 = qs[(8 + gq) * D + 4 * ks + tq];
-        double bv[NT];
+        for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-        for (int n = 0; n < NT; ++n) bv[n] = bq[p][n];
-        if (ks + PD < KS) load_b(ks + PD, bq[p]);
+          for (int n = 0; n < NT; ++n) acc[mt][n][0] = acc[mt][n][1] = 0.0;
+        constexpr int PD = 2;
+        constexpr int KS = D / 4;
+        double bq[PD][NT];
+        auto load_b = [&](int ks, double (&dst)[NT]) {
 #pragma unroll
-        for (int n = 0; n < NT; ++n) {
-          asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};\n"
-                       : "+d"(acc[0][n][0]), "+d"(acc[0][n][1])
-                       : "d"(a0), "d"(bv[n]));
-          asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};\n"
-                       : "+d"(acc[1][n][0]), "+d"(acc[1][n][1])
-                       : "d"(a1), "d"(bv[n]));
+          for (int n = 0; n < NT; ++n) {
+            const int J = (wid + (pass * NT + n) * kMaskWarps) * 8 + gq;
+            dst[n] = (J < nb) ? __ldg(kt + (size_t)(4 * ks + tq) * nb + J) : 0.0;
+          }
+        };
+#pragma unroll
+        for (int p = 0; p < PD; ++p) load_b(p, bq[p]);
+#pragma unroll 1
+        for (int ks0 = 0; ks0 < KS; ks0 += PD) {
+#pragma unroll
+          for (int p = 0; p < PD; ++p) {
+            const int ks = ks0 + p;
+            double av[MT];
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) av[mt] = qs[(mt * 8 + gq) * D + 4 * ks + tq];
+            double bv[NT];
+#pragma unroll
+            for (int n = 0; n < NT; ++n) bv[n] = bq[p][n];
+            if (ks + PD < KS) load_b(ks + PD, bq[p]);
+#pragma unroll
+            for (int n = 0; n < NT; ++n)
+#pragma unroll
+              for (int mt = 0; mt < MT; ++mt)
+                asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};\n"
+                             : "+d"(acc[mt][n][0]), "+d"(acc[mt][n][1])
+                             : "d"(av[mt]), "d"(bv[n]));
+          }
+        }
+        // accumulator element (row gq + 8 mt, column 2 tq + e) of each tile
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+          for (int n = 0; n < NT; ++n) {
+            const int Jb = (wid + (pass * NT + n) * kMaskWarps) * 8 + 2 * tq;
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+              if (Jb + e < nb) sc[(mt * 8 + gq) * nb + Jb + e] = acc[mt][n][e] * scale;
+          }
+      }
+    }
+    __syncthreads();
+
+    // Phase 2: warp w takes rows w, w + 8, ...  Lane L owns J = L + 32 i of
+    // the row; the probabilities replace the scores in shared memory (each
+    // lane rereads only its own entries), so long rows need no registers.
+    for (int rr = wid; rr < rows; rr += kMaskWarps) {
+      const int I = I0 + rr;
+      double* srow = sc + rr * nb;
+      auto key_of = [&](int J) { return (unsigned long long)__double_as_longlong(srow[J]); };
+      double mx = -DBL_MAX;
+#pragma unroll
+      for (int i = 0; i < NJ; ++i) {
+        const int J = lane + 32 * i;
+        if (J < nb) mx = fmax(mx, srow[J]);
+      }
+      mx = warp_max(mx);
+      double z = 0.0;
+#pragma unroll
+      for (int i = 0; i < NJ; ++i) {
+        const int J = lane + 32 * i;
+        if (J < nb) {
+          const double e = exp(srow[J] - mx);
+          srow[J] = e;
+          z += e;
         }
       }
-    }
-    // accumulator element (row gq + 8 mt, column 2 tq + e) of each tile
+      z = warp_sum(z);
+      const double rz = 1.0 / z;
+      unsigned long long tot = 0ull;
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int n = 0; n < NT; ++n) {
-        const int Jb = (wid + n * kWarps) * 8 + 2 * tq;
-#pragma unroll
-        for (int e = 0; e < 2; ++e)
-          if (Jb + e < nb) sc[(mt * 8 + gq) * nb + Jb + e] = acc[mt][n][e] * scale;
+      for (int i = 0; i < NJ; ++i) {
+        const int J = lane + 32 * i;
+        if (J < nb) {
+          const double pr = srow[J] * rz;   // A = e / sum(e)
+          srow[J] = pr;
+          tot += packed_mass(pr);
+        }
       }
-  }
-  __syncthreads();
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
 
-  // Phase 2: one warp per row.  Lane L holds J = L + 32 i.
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  if (warp < rows) {
-  const int I = I0 + warp;
-  const double* srow = sc + warp * nb;
-
-  double a[kMaxJ];
-  double mx = -DBL_MAX;
+      // keep bits: bit i of `keep` <-> J = lane + 32 i
+      uint32_t keep = 0u;
+      if (thr == 0.0 || (tot >> 11) < target) {
+        // thr == 0 keeps every block; so does a row whose whole mass rounds below 1 - thr.
 #pragma unroll
-  for (int i = 0; i < kMaxJ; ++i) {
-    const int J = lane + 32 * i;
-    a[i] = (J < nb) ? srow[J] : -DBL_MAX;
-    mx = fmax(mx, a[i]);
-  }
-  mx = warp_max(mx);
-  double z = 0.0;
-#pragma unroll
-  for (int i = 0; i < kMaxJ; ++i) {
-    const int J = lane + 32 * i;
-    a[i] = (J < nb) ? exp(a[i] - mx) : 0.0;
-    z += a[i];
-  }
-  z = warp_sum(z);
-  const double rz = 1.0 / z;
-#pragma unroll
-  for (int i = 0; i < kMaxJ; ++i) a[i] *= rz;  // A = e / sum(e)
-
-  // keep bits: bit i of `keep` <-> J = lane + 32 i
-  uint32_t keep = 0u;
-  const double target = 1.0 - thr;
-  double total = 0.0;
-#pragma unroll
-  for (int i = 0; i < kMaxJ; ++i) total += a[i];
-  total = warp_sum(total);
-  if (thr == 0.0 || total < target) {
-    // thr == 0 keeps every block; so does a row whose whole mass rounds below 1 - thr.
-#pragma unroll
-    for (int i = 0; i < kMaxJ; ++i)
-      if (lane + 32 * i < nb) keep |= 1u << i;
-  } else {
-    // Largest key v (bit pattern of a non-negative double, monotone in value)
-    // with mass(A >= v) >= target: the probability of the last kept block.
-    // Bits above the largest key's highest set bit are 0 in v: the search
-    // starts below them (every key is below hi = 2^(top + 1)).
-    unsigned long long kmax = 0ull;
-#pragma unroll
-    for (int i = 0; i < kMaxJ; ++i) {
-      const unsigned long long key = (unsigned long long)__double_as_longlong(a[i]);
-      kmax = (lane + 32 * i < nb && key > kmax) ? key : kmax;
-    }
-    kmax = warp_max(kmax);
-    const int top = 63 - __clzll((long long)kmax);
-    unsigned long long lo = 0ull, hi = (top >= 63) ? ~0ull : (1ull << (top + 1));
-    int cnt_lo = nb, cnt_hi = 0;
-    bool unique = false;
-    for (int bit = top; bit >= 0; --bit) {
-      const unsigned long long cand = lo | (1ull << bit);
-      double m = 0.0;
-      int c = 0;
-#pragma unroll
-      for (int i = 0; i < kMaxJ; ++i) {
-        const bool ge = (lane + 32 * i < nb) && (unsigned long long)__double_as_longlong(a[i]) >= cand;
-        m += ge ? a[i] : 0.0;
-        c += ge ? 1 : 0;
-      }
-      m = warp_sum(m);
-      c = __reduce_add_sync(0xffffffffu, c);
-      if (m >= target) {
-        lo = cand;
-        cnt_lo = c;
+        for (int i = 0; i < NJ; ++i)
+          if (lane + 32 * i < nb) keep |= 1u << i;
       } else {
-        hi = cand;
-        cnt_hi = c;
-      }
-      if (cnt_lo - cnt_hi == 1) {
-        unique = true;
-        break;
-      }
-    }
-    unsigned long long vb = lo;
-    if (unique) {  // the single block with lo <= key < hi
-      unsigned long long best = 0ull;
+        // Radix select of the boundary probability vb: the smallest kept
+        // value, i.e. the largest v whose mass(A >= v) reaches the target.
+        // Keys are the bit patterns of the (non-negative) probabilities,
+        // ordered like the values.  Each round histograms one 8-bit digit of
+        // the candidates' keys (fixed-point mass and count per bucket), scans
+        // the buckets from the top and keeps the bucket where the running
+        // mass reaches the target; the keys above it are kept for sure.  The
+        // search starts at the highest bit in which the keys differ and ends
+        // when one candidate is left, or when all bits are fixed (ties).
+        unsigned long long kmax = 0ull, kmin = ~0ull;
 #pragma unroll
-      for (int i = 0; i < kMaxJ; ++i) {
-        const unsigned long long key = (unsigned long long)__double_as_longlong(a[i]);
-        if (lane + 32 * i < nb && key < hi && key > best) best = key;
-      }
-      vb = warp_max(best);
-    }
-    // Every block above the boundary value is kept; blocks equal to it are
-    // added in ascending index order until the mass reaches the target.
-    double run = 0.0;
+        for (int i = 0; i < NJ; ++i) {
+          const int J = lane + 32 * i;
+          if (J < nb) {
+            const unsigned long long key = key_of(J);
+            kmax = key > kmax ? key : kmax;
+            kmin = key < kmin ? key : kmin;
+          }
+        }
+        kmax = warp_max(kmax);
+        kmin = warp_min(kmin);
+        unsigned long long vb = kmax;      // the boundary key
+        unsigned long long above = 0ull;   // packed mass of the keys above the candidates
+        bool single = true;
+        if (kmax != kmin) {
+          int top = 63 - __clzll((long long)(kmax ^ kmin));   // highest bit in which keys differ (< 63)
+          unsigned long long pref = kmax >> (top + 1);         // the bits above it, common to all keys
+          int cnt = 0;
+          int s = 0;
+          for (;;) {
+            const int w = min(8, top + 1);
+            s = top + 1 - w;
 #pragma unroll
-    for (int i = 0; i < kMaxJ; ++i) {
-      const unsigned long long key = (unsigned long long)__double_as_longlong(a[i]);
-      if (lane + 32 * i < nb && key > vb) {
-        keep |= 1u << i;
-        run += a[i];
-      }
-    }
-    run = warp_sum(run);
-    const double vval = __longlong_as_double((long long)vb);
+            for (int k = 0; k < 8; ++k) my_hist[lane + 32 * k] = 0ull;
+            __syncwarp();
 #pragma unroll
-    for (int i = 0; i < kMaxJ; ++i) {
-      if (run >= target) break;
-      const unsigned long long key = (unsigned long long)__double_as_longlong(a[i]);
-      uint32_t ties = __ballot_sync(0xffffffffu, (lane + 32 * i < nb) && key == vb);
-      while (ties != 0u && run < target) {
-        const int src = __ffs(ties) - 1;
-        ties &= ties - 1u;
-        if (lane == src) keep |= 1u << i;
-        run += vval;
+            for (int i = 0; i < NJ; ++i) {
+              const int J = lane + 32 * i;
+              if (J < nb) {
+                const unsigned long long key = key_of(J);
+                if ((key >> (top + 1)) == pref)
+                  atomicAdd(&my_hist[(key >> s) & ((1u << w) - 1u)], packed_mass(srow[J]));
+              }
+            }
+            __syncwarp();
+            // lane L scans buckets 255 - 8 L down to 248 - 8 L
+            unsigned long long loc[8], lsum = 0ull;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              loc[e] = my_hist[255 - 8 * lane - e];
+              lsum += loc[e];
+            }
+            unsigned long long incl = lsum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+              const unsigned long long t = __shfl_up_sync(0xffffffffu, incl, o);
+              if (lane >= o) incl += t;
+            }
+            unsigned long long cum = above + (incl - lsum), before = 0ull;
+            int found = -1;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const unsigned long long nc = cum + loc[e];
+              if (found < 0 && (nc >> 11) >= target) {
+                found = e;
+                before = cum;
+              }
+              cum = nc;
+            }
+            const uint32_t bal = __ballot_sync(0xffffffffu, found >= 0);
+            const int src = __ffs(bal) - 1;   // bal != 0: the candidates and `above` reach the target
+            const int e_sel = __shfl_sync(0xffffffffu, found, src);
+            above = __shfl_sync(0xffffffffu, before, src);
+            const int d_sel = 255 - 8 * src - e_sel;
+            cnt = (int)(my_hist[d_sel] & 2047ull);
+            pref = (pref << w) | (unsigned long long)d_sel;
+            __syncwarp();   // the histogram is cleared by the next round
+            if (cnt == 1 || s == 0) break;
+            top = s - 1;
+          }
+          if (cnt == 1) {
+            // the one key with these leading bits
+            unsigned long long best = 0ull;
+#pragma unroll
+            for (int i = 0; i < NJ; ++i) {
+              const int J = lane + 32 * i;
+              if (J < nb && (key_of(J) >> s) == pref) best = key_of(J);
+            }
+            vb = warp_max(best);
+          } else {
+            vb = pref;          // all bits fixed: cnt equal keys
+            single = false;
+          }
+        }
+        // Every block above vb is kept.  With a single block at vb it is kept
+        // too; equal keys at vb are added in ascending index order until the
+        // mass reaches the target.
+#pragma unroll
+        for (int i = 0; i < NJ; ++i) {
+          const int J = lane + 32 * i;
+          if (J < nb) {
+            const unsigned long long key = key_of(J);
+            if (key > vb || (single && key == vb)) keep |= 1u << i;
+          }
+        }
+        if (!single) {
+          unsigned long long run = above >> 11;
+          const unsigned long long mv = packed_mass(__longlong_as_double((long long)vb)) >> 11;
+#pragma unroll
+          for (int i = 0; i < NJ; ++i) {
+            if (run >= target) break;
+            const int J = lane + 32 * i;
+            uint32_t ties = __ballot_sync(0xffffffffu, J < nb && key_of(J) == vb);
+            while (ties != 0u && run < target) {
+              const int srcl = __ffs(ties) - 1;
+              ties &= ties - 1u;
+              if (lane == srcl) keep |= 1u << i;
+              run += mv;
+            }
+          }
+        }
       }
-    }
-  }
 
-  if (sta_t >= 0) {
-    int ti, hi_, wi;
-    block_tile(I, g, ti, hi_, wi);
+      if (sta_t >= 0) {
+        int ti, hi_, wi;
+        block_tile(I, g, ti, hi_, wi);
 #pragma unroll 1
-    for (int i = 0; i < kMaxJ; ++i) {
-      const int J = lane + 32 * i;
-      if (J >= nb) break;
-      int tj, hj, wj;
-      block_tile(J, g, tj, hj, wj);
-      if (abs(ti - tj) <= sta_t && abs(hi_ - hj) <= sta_h && abs(wi - wj) <= sta_w) keep |= 1u << i;
-    }
-  }
+        for (int i = 0; i < NJ; ++i) {
+          const int J = lane + 32 * i;
+          if (J >= nb) break;
+          int tj, hj, wj;
+          block_tile(J, g, tj, hj, wj);
+          if (abs(ti - tj) <= sta_t && abs(hi_ - hj) <= sta_h && abs(wi - wj) <= sta_w) keep |= 1u << i;
+        }
+      }
 
-  const size_t row = bh * nb + I;
-  int base = 0;
-  const uint32_t lt = (1u << lane) - 1u;
+      const size_t row = bh * nb + I;
+      int base = 0;
+      const uint32_t lt = (1u << lane) - 1u;
 #pragma unroll
-  for (int i = 0; i < kMaxJ; ++i) {
-    const int J = lane + 32 * i;
-    const bool k = (keep >> i) & 1u;
-    const uint32_t bal = __ballot_sync(0xffffffffu, k);
-    if (k) kv_idx[row * nb + base + __popc(bal & lt)] = J;
-    if (mask != nullptr && J < nb) mask[row * nb + J] = k ? 1 : 0;
-    base += __popc(bal);
-  }
-  if (lane == 0) kv_count[row] = base;
-  }  // warp < rows
-  __syncthreads();   // qs and sc are rewritten by the next group
+      for (int i = 0; i < NJ; ++i) {
+        const int J = lane + 32 * i;
+        const bool k = (keep >> i) & 1u;
+        const uint32_t bal = __ballot_sync(0xffffffffu, k);
+        if (k) kv_idx[row * nb + base + __popc(bal & lt)] = J;
+        if (mask != nullptr && J < nb) mask[row * nb + J] = k ? 1 : 0;
+        base += __popc(bal);
+      }
+      if (lane == 0) kv_count[row] = base;
+    }  // rows of this warp
+    __syncthreads();   // qs and sc are rewritten by the next group
   }  // groups
 }
 
@@ -447,7 +526,8 @@ cudaError_t launch_pool(const Dims& g, const void* q, const void* k, double* qba
 template <int D, int NJ>
 cudaError_t launch_mask_t(const Dims& g, const double* qbar, const double* kbar, double thr, int sta_t, int sta_h,
                           int sta_w, int32_t* kv_count, int32_t* kv_idx, uint8_t* mask, cudaStream_t st) {
-  const size_t smem = (size_t)kMaskRows * (g.d + g.nb) * sizeof(double);
+  constexpr int R = mask_rows<NJ>();
+  const size_t smem = (size_t)R * (g.d + g.nb) * sizeof(double) + (size_t)kMaskWarps * 256 * sizeof(uint64_t);
   const double scale = 1.0 / std::sqrt((double)g.d);
   cudaError_t e = cudaFuncSetAttribute(mask_kernel<D, NJ>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -457,7 +537,7 @@ cudaError_t launch_mask_t(const Dims& g, const double* qbar, const double* kbar,
   if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, mask_kernel<D, NJ>, kMaskThreads, smem)) !=
       cudaSuccess)
     return e;
-  const int total = (g.nb + kMaskRows - 1) / kMaskRows * g.B * g.heads;
+  const int total = (g.nb + R - 1) / R * g.B * g.heads;
   const int grid = std::max(1, std::min(total, sms * std::max(1, per_sm)));
   mask_kernel<D, NJ><<<grid, kMaskThreads, smem, st>>>(qbar, kbar, g, thr, scale, sta_t, sta_h, sta_w, kv_count,
                                                        kv_idx, mask);

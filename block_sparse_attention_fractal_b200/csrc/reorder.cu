@@ -7,9 +7,10 @@
 // one block of `BS` consecutive kernel-order positions of one (tensor, b,
 // head); threads of a row cover its 16-byte vectors, so both the gathered
 // model-order rows and the contiguous kernel-order run are whole 128-byte
-// lines.  Every thread issues all its loads before its first store, so each
-// SM keeps BS * d * 2 bytes per resident CTA in flight (the latency of one
-// load is paid once per block, not once per row).  CTAs are numbered heads
+// lines.  The block's token indices are computed once per row into shared
+// memory, and every thread issues all its loads before its first store, so
+// each SM keeps BS * d * 2 bytes per resident CTA in flight (the latency of
+// one load is paid once per block, not once per row).  CTAs are numbered heads
 // fastest: the CTAs that run together move the same positions of every head,
 // i.e. the neighbouring rows of the same model-order tokens.
 //
@@ -54,12 +55,22 @@ __global__ void __launch_bounds__(kThreads) reorder_kernel(Tensors a, Dims g) {
   const uint4* __restrict__ src = t ? a.src[1] : a.src[0];
   uint4* __restrict__ dst = t ? a.dst[1] : a.dst[0];
 
+  // The block's token indices, computed once per row (the integer divisions
+  // of the fractal order would otherwise run in each of the row's VEC
+  // threads and dominate the kernel's instruction count).
+  __shared__ int tok[BS];
+  if (threadIdx.x < BS) {
+    const int p = I * BS + threadIdx.x;
+    tok[threadIdx.x] = (p < g.N) ? fractal_token(p, g.H, g.W, g.P) : -1;
+  }
+  __syncthreads();
+
   uint4 v[VPT];
   int n[VPT];
 #pragma unroll
   for (int j = 0; j < VPT; ++j) {
     const int p = I * BS + r0 + j * RPP;
-    n[j] = (p < g.N) ? fractal_token(p, g.H, g.W, g.P) : -1;
+    n[j] = tok[r0 + j * RPP];
     const size_t kidx = (bh * g.Npad + p) * VEC + c;                                   // kernel order
     const size_t midx = (((size_t)b * g.N + (n[j] < 0 ? 0 : n[j])) * g.heads + head) * VEC + c;  // model order
     if (kInverse) v[j] = __ldcs(src + kidx);

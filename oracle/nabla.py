@@ -301,6 +301,61 @@ def masked_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, keep: np.ndarr
     return O, lse
 
 
+# ------------------------------------------ block-sparse attention backward
+
+def masked_attention_backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, keep: np.ndarray, dO: np.ndarray,
+                              N: int, block: int, scale: Optional[float] = None
+                              ) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Gradients of ``masked_attention`` with respect to q, k and v, given the
+    gradient dO of its output.
+
+    NABLA summary, "Contribuciones Clave" ("Aceleracion de Doble Fase"): the
+    block-sparse attention also runs in pre-training and fine-tuning, so its
+    backward pass follows the same block mask.  Per query block I, with the
+    valid keys of its kept blocks as columns:
+
+        P  = softmax(scale * Q_I K^T)           (as in the forward pass)
+        dV += P^T dO_I
+        dP = dO_I V^T
+        dS = P * (dP - rowsum(dO_I * O_I))     (O_I = P V: the softmax Jacobian)
+        dQ_I = scale * dS K,    dK += scale * dS^T Q_I
+
+    Padded query rows take part in nothing (their dO is ignored, their dQ is
+    0); padded keys are never columns.  Returns (dq, dk, dv) [B, heads, Npad, d].
+    """
+    B, heads, Npad, d = q.shape
+    nb = Npad // block
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = np.zeros_like(q, dtype=np.float64)
+    dk = np.zeros_like(k, dtype=np.float64)
+    dv = np.zeros_like(v, dtype=np.float64)
+    for b in range(B):
+        for h in range(heads):
+            for I in range(nb):
+                qlo, qhi = I * block, min((I + 1) * block, N)
+                if qhi <= qlo:
+                    continue
+                cols = []
+                for J in np.nonzero(keep[b, h, I])[0]:
+                    klo, khi = int(J) * block, min((int(J) + 1) * block, N)
+                    cols.extend(range(klo, khi))
+                cols = np.asarray(cols, dtype=np.int64)
+                if cols.size == 0:
+                    continue
+                qI, kc, vc, dOI = q[b, h, qlo:qhi], k[b, h, cols], v[b, h, cols], dO[b, h, qlo:qhi]
+                s = (qI @ kc.T) * scale
+                e = np.exp(s - s.max(axis=1, keepdims=True))
+                P = e / e.sum(axis=1, keepdims=True)
+                OI = P @ vc
+                dv[b, h, cols] += P.T @ dOI
+                dP = dOI @ vc.T
+                dS = P * (dP - (dOI * OI).sum(axis=1, keepdims=True))
+                dq[b, h, qlo:qhi] += scale * (dS @ kc)
+                dk[b, h, cols] += scale * (dS.T @ qI)
+    return dq, dk, dv
+
+
 # ------------------------------------------------------------ full path
 
 def nabla_attention(q_bnhd: np.ndarray, k_bnhd: np.ndarray, v_bnhd: np.ndarray,

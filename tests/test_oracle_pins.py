@@ -415,6 +415,87 @@ def test_thr_zero_pipeline_is_dense_attention_in_model_order():
         assert np.allclose(O[0, :, h], ref, rtol=1e-12, atol=1e-12)
 
 
+# ------------------------------------------------------------- backward
+
+@pytest.mark.parametrize("N,bs", [(96, 32), (100, 32)])
+def test_backward_equals_library_autograd(N, bs):
+    """The oracle's gradients equal torch autograd (float64) through the
+    library attention (scaled_dot_product_attention) with the expanded mask."""
+    rng = np.random.default_rng(11)
+    d, heads = 16, 2
+    Npad = nabla.padded_len(N, bs)
+    nb = Npad // bs
+    q = rng.standard_normal((1, heads, Npad, d)) * 1.5
+    k = rng.standard_normal((1, heads, Npad, d)) * 1.5
+    v = rng.standard_normal((1, heads, Npad, d))
+    dO = rng.standard_normal((1, heads, Npad, d))
+    keep = rng.random((1, heads, nb, nb)) < 0.5
+    keep[..., np.arange(nb), np.arange(nb)] = True
+    dq, dk, dv = oracle.masked_attention_backward(q, k, v, keep, dO, N, bs)
+    scale = 1 / math.sqrt(d)
+    for h in range(heads):
+        tokmask = torch.from_numpy(np.kron(keep[0, h], np.ones((bs, bs), dtype=bool))[:N, :N])
+        tq, tk, tv = (torch.from_numpy(x[0, h, :N].copy()).requires_grad_() for x in (q, k, v))
+        out = F.scaled_dot_product_attention(tq[None, None], tk[None, None], tv[None, None],
+                                             attn_mask=tokmask[None, None], scale=scale)[0, 0]
+        out.backward(torch.from_numpy(dO[0, h, :N].copy()))
+        assert np.allclose(dq[0, h, :N], tq.grad.numpy(), rtol=1e-11, atol=1e-12)
+        assert np.allclose(dk[0, h, :N], tk.grad.numpy(), rtol=1e-11, atol=1e-12)
+        assert np.allclose(dv[0, h, :N], tv.grad.numpy(), rtol=1e-11, atol=1e-12)
+    for g in (dq, dk, dv):
+        assert np.all(g[:, :, N:] == 0)
+
+
+def test_backward_matches_central_differences():
+    """d<O, dO>/dx by central differences (step 1e-6) at a few entries of
+    q, k and v, on a tiny masked problem with a ragged last block."""
+    rng = np.random.default_rng(12)
+    N, bs, d = 40, 16, 4
+    Npad = nabla.padded_len(N, bs)
+    nb = Npad // bs
+    x = {n: rng.standard_normal((1, 1, Npad, d)) for n in ("q", "k", "v")}
+    dO = rng.standard_normal((1, 1, Npad, d))
+    keep = np.array([[[[True, False, True], [True, True, False], [False, True, True]]]])
+    grads = dict(zip(("q", "k", "v"), oracle.masked_attention_backward(x["q"], x["k"], x["v"], keep, dO, N, bs)))
+
+    def loss(xx):
+        O, _ = oracle.masked_attention(xx["q"], xx["k"], xx["v"], keep, N, bs)
+        return float((O[:, :, :N] * dO[:, :, :N]).sum())
+
+    eps = 1e-6
+    for name in ("q", "k", "v"):
+        for (row, col) in ((0, 0), (17, 2), (N - 1, 3), (33, 1)):
+            xp = {n: a.copy() for n, a in x.items()}
+            xm = {n: a.copy() for n, a in x.items()}
+            xp[name][0, 0, row, col] += eps
+            xm[name][0, 0, row, col] -= eps
+            fd = (loss(xp) - loss(xm)) / (2 * eps)
+            assert abs(fd - grads[name][0, 0, row, col]) < 1e-7 * max(1.0, abs(fd)), (name, row, col)
+
+
+def test_pins_catch_a_backward_without_the_softmax_jacobian_term(monkeypatch):
+    def bad(q, k, v, keep, dO, N, block, scale=None):   # dS = P * dP: the rowsum(dO * O) term dropped
+        B, heads, Npad, d = q.shape
+        scale = 1.0 / math.sqrt(d) if scale is None else scale
+        dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+        for h in range(heads):
+            for I in range(Npad // block):
+                lo, hi = I * block, min((I + 1) * block, N)
+                cols = np.concatenate([np.arange(J * block, min((J + 1) * block, N))
+                                       for J in np.nonzero(keep[0, h, I])[0]])
+                s_ = (q[0, h, lo:hi] @ k[0, h, cols].T) * scale
+                P = np.exp(s_ - s_.max(1, keepdims=True))
+                P /= P.sum(1, keepdims=True)
+                dS = P * (dO[0, h, lo:hi] @ v[0, h, cols].T)
+                dv[0, h, cols] += P.T @ dO[0, h, lo:hi]
+                dq[0, h, lo:hi] += scale * dS @ k[0, h, cols]
+                dk[0, h, cols] += scale * dS.T @ q[0, h, lo:hi]
+        return dq, dk, dv
+    monkeypatch.setattr(oracle, "masked_attention_backward", bad)
+    with pytest.raises(AssertionError):
+        test_backward_equals_library_autograd(96, 32)
+
+
 def test_lists_roundtrip():
     rng = np.random.default_rng(9)
     keep = rng.random((2, 3, 7, 7)) < 0.4
