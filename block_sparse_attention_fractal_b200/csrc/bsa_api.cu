@@ -70,8 +70,9 @@ size_t pooled_bytes(const Dims& g) { return (size_t)g.B * g.heads * g.nb * g.d *
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// Workspace: control block | qbar | kbar | attention plan region.
-size_t plan_offset(const Dims& g) { return sizeof(Ctrl) + align256(2 * pooled_bytes(g)); }
+// Workspace: control block | qbar | kbar | reduced scores | attention plan region.
+size_t scores_offset(const Dims& g) { return sizeof(Ctrl) + align256(2 * pooled_bytes(g)); }
+size_t plan_offset(const Dims& g) { return scores_offset(g) + align256(bsa::mask_scores_bytes(g)); }
 
 size_t workspace_bytes(const Dims& g) { return plan_offset(g) + align256(bsa::plan_region_bytes(g)); }
 
@@ -161,8 +162,9 @@ bsa_status bsa_build_block_mask_pooled(const bsa_shape* s, float thr, int32_t st
   const bool sta = sta_t >= 0 && sta_h >= 0 && sta_w >= 0;
   double* qbar = (double*)((char*)workspace + sizeof(Ctrl));
   double* kbar = qbar + pooled_bytes(g) / sizeof(double);
-  return from_cuda(bsa::launch_mask(g, qbar, kbar, (double)thr, sta ? sta_t : -1, sta ? sta_h : -1, sta ? sta_w : -1,
-                                    kv_count, kv_idx, mask_or_null, (cudaStream_t)stream));
+  double* scores = (double*)((char*)workspace + scores_offset(g));
+  return from_cuda(bsa::launch_mask(g, qbar, kbar, scores, (double)thr, sta ? sta_t : -1, sta ? sta_h : -1,
+                                    sta ? sta_w : -1, kv_count, kv_idx, mask_or_null, (cudaStream_t)stream));
 }
 
 bsa_status bsa_build_block_mask(const bsa_shape* s, const void* q_bhnd, const void* k_bhnd, float thr,
@@ -185,8 +187,9 @@ bsa_status bsa_build_block_mask(const bsa_shape* s, const void* q_bhnd, const vo
   cudaStream_t cs = (cudaStream_t)stream;
   cudaError_t e = bsa::launch_pool(g, q_bhnd, k_bhnd, qbar, kbar, (Ctrl*)workspace, bsa::next_launch_seq(), cs);
   if (e != cudaSuccess) return BSA_ERR_CUDA;
-  e = bsa::launch_mask(g, qbar, kbar, (double)thr, sta ? sta_t : -1, sta ? sta_h : -1, sta ? sta_w : -1, kv_count,
-                       kv_idx, mask_or_null, cs);
+  double* scores = (double*)((char*)workspace + scores_offset(g));
+  e = bsa::launch_mask(g, qbar, kbar, scores, (double)thr, sta ? sta_t : -1, sta ? sta_h : -1, sta ? sta_w : -1,
+                       kv_count, kv_idx, mask_or_null, cs);
   return from_cuda(e);
 }
 

@@ -23,9 +23,12 @@ cudaError_t launch_reorder_qk_pool(const Dims& g, const void* q_bnhd, const void
 cudaError_t launch_pool(const Dims& g, const void* q, const void* k, double* qbar, double* kbar, Ctrl* ctrl,
                         uint32_t seq, cudaStream_t st);
 
-// Reduced attention + CDF threshold (+ STA union) -> KV lists.
-cudaError_t launch_mask(const Dims& g, const double* qbar, const double* kbar, double thr, int sta_t, int sta_h,
-                        int sta_w, int32_t* kv_count, int32_t* kv_idx, uint8_t* mask, cudaStream_t st);
+// Reduced attention + CDF threshold (+ STA union) -> KV lists: the fp64
+// scores go through `scores` ([B, heads, nb, nb] double, mask_scores_bytes).
+size_t mask_scores_bytes(const Dims& g);
+cudaError_t launch_mask(const Dims& g, const double* qbar, const double* kbar, double* scores, double thr,
+                        int sta_t, int sta_h, int sta_w, int32_t* kv_count, int32_t* kv_idx, uint8_t* mask,
+                        cudaStream_t st);
 
 // Block-sparse attention on the legacy warp-level mma.sync tensor-core path
 // (baseline kernel; any supported shape).

@@ -1,9 +1,10 @@
 // Adaptive block mask (NABLA summary, Metodologia 2 and 3):
 //   pool_kernel: block means of Q and K ("Submuestreo"), double precision;
-//   mask_kernel: reduced attention softmax(qbar kbar^T / sqrt(d)) per row
-//                ("Atencion Reducida"), the CDF threshold ("Umbralizacion CDF"),
-//                the optional STA union, and the ascending KV index lists that
-//                the attention kernel walks ("Expansion").
+//   scores_kernel: the reduced scores qbar kbar^T / sqrt(d) ("Atencion
+//                Reducida") on the fp64 tensor cores, into the workspace;
+//   select_kernel: per row, the softmax, the CDF threshold ("Umbralizacion
+//                CDF"), the optional STA union, and the ascending KV index
+//                lists that the attention kernel walks ("Expansion").
 //
 // Precision: bf16 values summed in double are exact, so the block means equal
 // the exact mean rounded once.  Dot products, exp and the probability masses
@@ -134,23 +135,90 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __nv_bfloat16*
   if (threadIdx.x == 0) sm100::mbar_drain_ring(full, kPoolStages, armed, kPoolWaitNs);
 }
 
-// ------------------------------------------------------------- mask rows
+// ------------------------------------------------------- reduced scores
 
-constexpr int kMaskThreads = 256;             // 8 warps
-constexpr int kMaskWarps = kMaskThreads / 32;
-// Query-block rows per CTA: 16, or 8 when rows are longer than 512 blocks
-// (the CTA's scores then stay at 64 KB of shared memory, two CTAs per SM).
-template <int NJ>
-constexpr int mask_rows() { return NJ <= 16 ? 16 : 8; }
+// scores_kernel: S[bh][I][J] = scale * qbar_I . kbar_J for one 32 x 64 tile of
+// one (b, head) per CTA, on the fp64 tensor cores (mma.sync m8n8k4, fp64
+// multiply-add).  The tile's qbar rows and kbar columns are staged in shared
+// memory first (rows padded so the fragment loads of a half-warp hit 16
+// different banks); each of the 4 warps computes 32 rows x 16 columns.
+constexpr int kScoreRows = 32, kScoreCols = 64, kScoreThreads = 128;
+constexpr int kAStride = 132;                 // doubles per staged qbar row (D = 128 + 4)
+constexpr int kBStride = kScoreCols + 4;      // doubles per staged kbar row
+
+template <int D>
+__global__ void __launch_bounds__(kScoreThreads) scores_kernel(const double* __restrict__ qbar,
+                                                               const double* __restrict__ kbar, Dims g,
+                                                               double scale, double* __restrict__ scores) {
+  extern __shared__ __align__(16) double sm[];
+  double* As = sm;                                  // [kScoreRows][kAStride]
+  double* Bs = sm + kScoreRows * kAStride;          // [D][kBStride]
+  const int nb = g.nb;
+  const int tiles_i = (nb + kScoreRows - 1) / kScoreRows, tiles_j = (nb + kScoreCols - 1) / kScoreCols;
+  const int tj = blockIdx.x % tiles_j;
+  const int ti = (blockIdx.x / tiles_j) % tiles_i;
+  const size_t bh = blockIdx.x / ((unsigned)tiles_j * tiles_i);
+  const int I0 = ti * kScoreRows, J0 = tj * kScoreCols;
+  const double* qsrc = qbar + (bh * nb) * D;
+  const double* ksrc = kbar + bh * D * (size_t)nb;
+  for (int i = threadIdx.x; i < kScoreRows * D; i += kScoreThreads) {
+    const int r = i / D, c = i % D;
+    As[r * kAStride + c] = (I0 + r < nb) ? qsrc[(size_t)(I0 + r) * D + c] : 0.0;
+  }
+  for (int i = threadIdx.x; i < D * kScoreCols; i += kScoreThreads) {
+    const int k = i / kScoreCols, c = i % kScoreCols;
+    Bs[k * kBStride + c] = (J0 + c < nb) ? ksrc[(size_t)k * nb + J0 + c] : 0.0;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int gq = lane >> 2, tq = lane & 3;
+  double acc[4][2][2];
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+    for (int n = 0; n < 2; ++n) acc[mt][n][0] = acc[mt][n][1] = 0.0;
+#pragma unroll 4
+  for (int ks = 0; ks < D / 4; ++ks) {
+    double av[4], bv[2];
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) av[mt] = As[(mt * 8 + gq) * kAStride + 4 * ks + tq];
+#pragma unroll
+    for (int n = 0; n < 2; ++n) bv[n] = Bs[(4 * ks + tq) * kBStride + wid * 16 + n * 8 + gq];
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+      for (int n = 0; n < 2; ++n)
+        asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};\n"
+                     : "+d"(acc[mt][n][0]), "+d"(acc[mt][n][1])
+                     : "d"(av[mt]), "d"(bv[n]));
+  }
+  // accumulator element (row gq + 8 mt, column 2 tq + e) of each 8 x 8 tile
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt) {
+    const int I = I0 + mt * 8 + gq;
+    if (I >= nb) continue;
+#pragma unroll
+    for (int n = 0; n < 2; ++n) {
+      const int J = J0 + wid * 16 + n * 8 + 2 * tq;
+      double* dst = scores + (bh * nb + I) * (size_t)nb + J;
+      if (J + 1 < nb) {
+        dst[0] = acc[mt][n][0] * scale;
+        dst[1] = acc[mt][n][1] * scale;
+      } else if (J < nb) {
+        dst[0] = acc[mt][n][0] * scale;
+      }
+    }
+  }
+}
+
+// --------------------------------------------------------- selection rows
+
+constexpr int kSelThreads = 256;             // 8 warps, one row each at a time
+constexpr int kSelWarps = kSelThreads / 32;
 
 __device__ __forceinline__ double warp_sum(double v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-__device__ __forceinline__ double warp_max(double v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
 }
 __device__ __forceinline__ unsigned long long warp_max(unsigned long long v) {
@@ -158,14 +226,6 @@ __device__ __forceinline__ unsigned long long warp_max(unsigned long long v) {
   for (int o = 16; o > 0; o >>= 1) {
     const unsigned long long w = __shfl_xor_sync(0xffffffffu, v, o);
     v = w > v ? w : v;
-  }
-  return v;
-}
-__device__ __forceinline__ unsigned long long warp_min(unsigned long long v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const unsigned long long w = __shfl_xor_sync(0xffffffffu, v, o);
-    v = w < v ? w : v;
   }
   return v;
 }
@@ -191,235 +251,164 @@ __device__ __forceinline__ void block_tile(int I, const Dims& g, int& t, int& th
   tw = (rem - h * g.W) / g.P;
 }
 
-// Persistent grid: CTA c handles the groups of R rows c, c + gridDim.x, ...
-// of all (b, head).  Dynamic shared memory: qbar rows [R][D], scores [R][nb]
-// (double), then a 256-bucket histogram per warp (uint64).  NJ = ceil(nb / 32)
-// rounded up to a power of two: the values of a row that each lane holds.
-template <int D, int NJ>
-__global__ void __launch_bounds__(kMaskThreads, 2) mask_kernel(const double* __restrict__ qbar,
-                                                               const double* __restrict__ kbar, Dims g, double thr,
-                                                               double scale, int sta_t, int sta_h, int sta_w,
-                                                               int32_t* __restrict__ kv_count,
-                                                               int32_t* __restrict__ kv_idx,
-                                                               uint8_t* __restrict__ mask) {
-  constexpr int R = mask_rows<NJ>();
-  constexpr int MT = R / 8;                                    // 8-row MMA tiles
-  extern __shared__ __align__(16) double smem[];
-  double* qs = smem;                                           // [R][D]
-  double* sc = smem + R * D;                                   // [R][nb]
+// select_kernel: one warp per row of the reduced map (grid-stride over all
+// rows of all (b, head)).  The row's scores are copied to the warp's slice of
+// shared memory, turned into probabilities in place (fp64 softmax), and the
+// CDF threshold picks the kept blocks (radix select below); the optional STA
+// union is added and the ascending KV list written.  Lane L owns J = L + 32 i.
+template <int NJ>
+__global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __restrict__ scores, Dims g, double thr,
+                                                             int sta_t, int sta_h, int sta_w,
+                                                             int32_t* __restrict__ kv_count,
+                                                             int32_t* __restrict__ kv_idx,
+                                                             uint8_t* __restrict__ mask) {
+  extern __shared__ __align__(16) double ssm[];
   const int nb = g.nb;
-  unsigned long long* hist = reinterpret_cast<unsigned long long*>(sc + R * nb);   // [warps][256]
-  const int groups = (nb + R - 1) / R;
-  const int total = groups * g.B * g.heads;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  unsigned long long* my_hist = hist + wid * 256;
+  double* srow = ssm + wid * (NJ * 32);                                     // this warp's row
+  unsigned long long* my_hist =
+      reinterpret_cast<unsigned long long*>(ssm + kSelWarps * NJ * 32) + wid * 256;
   const unsigned long long target = __double2ull_rn((1.0 - thr) * kMassScale);
+  const size_t total_rows = (size_t)g.B * g.heads * nb;
 
-  for (int grp = blockIdx.x; grp < total; grp += gridDim.x) {
-    const size_t bh = (size_t)(grp / groups);
-    const int I0 = (grp % groups) * R;
-    const int rows = min(R, nb - I0);
-
-    for (int i = threadIdx.x; i < R * D; i += kMaskThreads) {
-      const int r = i / D;
-      qs[i] = (r < rows) ? qbar[(bh * nb + I0 + r) * D + (i % D)] : 0.0;
-    }
-    __syncthreads();
-
-    // Phase 1: scores s[r][J] = scale * qbar_r . kbar_J on the fp64 tensor
-    // cores (mma.sync m8n8k4, fp64 multiply-add): warp w computes the R rows
-    // against the 8-column tiles w, w + 8, ... of J.  A fragments (qbar rows)
-    // come from shared memory, B fragments from the transposed kbar
-    // [bh][d][nb] in global memory (64 contiguous bytes per fragment row),
-    // loaded PD k-steps ahead of their use.
-    // (in passes of at most 8 column tiles, so the accumulators and the B
-    // prefetch fit in registers for long rows)
-    {
-      constexpr int NTW = NJ / 2;                                // 8-column tiles per warp
-      constexpr int NT = NTW < 8 ? NTW : 8;                      // ... per pass
-      const int gq = lane >> 2, tq = lane & 3;
-      const double* kt = kbar + bh * D * (size_t)nb;
-#pragma unroll 1
-      for (int pass = 0; pass < NTW / NT; ++pass) {
-        double acc[MT][NT][2];
+  for (size_t row = (size_t)blockIdx.x * kSelWarps + wid; row < total_rows; row += (size_t)gridDim.x * kSelWarps) {
+    const int I = (int)(row % nb);
+    const double* src = scores + row * nb;
+    // the row into shared memory, its largest and smallest score on the way
+    double mx = -DBL_MAX, mn = DBL_MAX;
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-          for (int n = 0; n < NT; ++n) acc[mt][n][0] = acc[mt][n][1] = 0.0;
-        constexpr int PD = 2;
-        constexpr int KS = D / 4;
-        double bq[PD][NT];
-        auto load_b = [&](int ks, double (&dst)[NT]) {
-#pragma unroll
-          for (int n = 0; n < NT; ++n) {
-            const int J = (wid + (pass * NT + n) * kMaskWarps) * 8 + gq;
-            dst[n] = (J < nb) ? __ldg(kt + (size_t)(4 * ks + tq) * nb + J) : 0.0;
-          }
-        };
-#pragma unroll
-        for (int p = 0; p < PD; ++p) load_b(p, bq[p]);
-#pragma unroll 1
-        for (int ks0 = 0; ks0 < KS; ks0 += PD) {
-#pragma unroll
-          for (int p = 0; p < PD; ++p) {
-            const int ks = ks0 + p;
-            double av[MT];
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt) av[mt] = qs[(mt * 8 + gq) * D + 4 * ks + tq];
-            double bv[NT];
-#pragma unroll
-            for (int n = 0; n < NT; ++n) bv[n] = bq[p][n];
-            if (ks + PD < KS) load_b(ks + PD, bq[p]);
-#pragma unroll
-            for (int n = 0; n < NT; ++n)
-#pragma unroll
-              for (int mt = 0; mt < MT; ++mt)
-                asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};\n"
-                             : "+d"(acc[mt][n][0]), "+d"(acc[mt][n][1])
-                             : "d"(av[mt]), "d"(bv[n]));
-          }
-        }
-        // accumulator element (row gq + 8 mt, column 2 tq + e) of each tile
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-          for (int n = 0; n < NT; ++n) {
-            const int Jb = (wid + (pass * NT + n) * kMaskWarps) * 8 + 2 * tq;
-#pragma unroll
-            for (int e = 0; e < 2; ++e)
-              if (Jb + e < nb) sc[(mt * 8 + gq) * nb + Jb + e] = acc[mt][n][e] * scale;
-          }
+    for (int i = 0; i < NJ; ++i) {
+      const int J = lane + 32 * i;
+      if (J < nb) {
+        const double v = src[J];
+        srow[J] = v;
+        mx = fmax(mx, v);
+        mn = fmin(mn, v);
       }
     }
-    __syncthreads();
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      mn = fmin(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    }
+    double z = 0.0;
+#pragma unroll
+    for (int i = 0; i < NJ; ++i) {
+      const int J = lane + 32 * i;
+      if (J < nb) {
+        const double e = exp(srow[J] - mx);
+        srow[J] = e;
+        z += e;
+      }
+    }
+    z = warp_sum(z);
+    const double rz = 1.0 / z;
+#pragma unroll
+    for (int i = 0; i < NJ; ++i) {
+      const int J = lane + 32 * i;
+      if (J < nb) srow[J] *= rz;        // A = e / sum(e)
+    }
+    // The largest and smallest probabilities, by the same arithmetic as the
+    // row's own entries (exp(0) = 1 exactly): their bit patterns bound the
+    // keys of the radix select.
+    const unsigned long long kmax = (unsigned long long)__double_as_longlong(1.0 * rz);
+    const unsigned long long kmin = (unsigned long long)__double_as_longlong(exp(mn - mx) * rz);
+    auto key_of = [&](int J) { return (unsigned long long)__double_as_longlong(srow[J]); };
 
-    // Phase 2: warp w takes rows w, w + 8, ...  Lane L owns J = L + 32 i of
-    // the row; the probabilities replace the scores in shared memory (each
-    // lane rereads only its own entries), so long rows need no registers.
-    for (int rr = wid; rr < rows; rr += kMaskWarps) {
-      const int I = I0 + rr;
-      double* srow = sc + rr * nb;
-      auto key_of = [&](int J) { return (unsigned long long)__double_as_longlong(srow[J]); };
-      double mx = -DBL_MAX;
-#pragma unroll
-      for (int i = 0; i < NJ; ++i) {
-        const int J = lane + 32 * i;
-        if (J < nb) mx = fmax(mx, srow[J]);
-      }
-      mx = warp_max(mx);
-      double z = 0.0;
-#pragma unroll
-      for (int i = 0; i < NJ; ++i) {
-        const int J = lane + 32 * i;
-        if (J < nb) {
-          const double e = exp(srow[J] - mx);
-          srow[J] = e;
-          z += e;
-        }
-      }
-      z = warp_sum(z);
-      const double rz = 1.0 / z;
-      unsigned long long tot = 0ull;
-#pragma unroll
-      for (int i = 0; i < NJ; ++i) {
-        const int J = lane + 32 * i;
-        if (J < nb) {
-          const double pr = srow[J] * rz;   // A = e / sum(e)
-          srow[J] = pr;
-          tot += packed_mass(pr);
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
-
-      // keep bits: bit i of `keep` <-> J = lane + 32 i
-      uint32_t keep = 0u;
-      if (thr == 0.0 || (tot >> 11) < target) {
-        // thr == 0 keeps every block; so does a row whose whole mass rounds below 1 - thr.
+    // keep bits: bit i of `keep` <-> J = lane + 32 i
+    uint32_t keep = 0u;
+    bool keep_all = (thr == 0.0);       // thr == 0 keeps every block
+    if (!keep_all) {
+      // Radix select of the boundary probability vb: the smallest kept
+      // value, i.e. the largest v whose mass(A >= v) reaches the target.
+      // Keys are the bit patterns of the (non-negative) probabilities,
+      // ordered like the values.  Each round histograms one 8-bit digit of
+      // the candidates' keys (fixed-point mass and count per bucket, shared
+      // memory atomics), scans the buckets from the top and keeps the bucket
+      // where the running mass reaches the target; the keys above it are kept
+      // for sure.  The search starts at the highest bit in which the keys
+      // differ and ends when one candidate is left, or when all bits are
+      // fixed (equal keys: ties).  A row whose whole mass rounds below the
+      // target keeps every block.
+      unsigned long long vb = kmax;      // the boundary key
+      unsigned long long above = 0ull;   // packed mass of the keys above the candidates
+      bool single = true;
+      if (kmax == kmin) {
+        // all probabilities equal: ties from the first block on
+        unsigned long long tot = 0ull;
 #pragma unroll
         for (int i = 0; i < NJ; ++i)
-          if (lane + 32 * i < nb) keep |= 1u << i;
+          if (lane + 32 * i < nb) tot += packed_mass(srow[lane + 32 * i]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+        keep_all = (tot >> 11) < target;
+        single = false;
       } else {
-        // Radix select of the boundary probability vb: the smallest kept
-        // value, i.e. the largest v whose mass(A >= v) reaches the target.
-        // Keys are the bit patterns of the (non-negative) probabilities,
-        // ordered like the values.  Each round histograms one 8-bit digit of
-        // the candidates' keys (fixed-point mass and count per bucket), scans
-        // the buckets from the top and keeps the bucket where the running
-        // mass reaches the target; the keys above it are kept for sure.  The
-        // search starts at the highest bit in which the keys differ and ends
-        // when one candidate is left, or when all bits are fixed (ties).
-        unsigned long long kmax = 0ull, kmin = ~0ull;
+        int top = 63 - __clzll((long long)(kmax ^ kmin));   // highest bit in which keys differ (< 63)
+        unsigned long long pref = kmax >> (top + 1);         // the bits above it, common to all keys
+        int cnt = 0, s = 0;
+        bool first = true;
+        for (;;) {
+          const int w = min(8, top + 1);
+          s = top + 1 - w;
 #pragma unroll
-        for (int i = 0; i < NJ; ++i) {
-          const int J = lane + 32 * i;
-          if (J < nb) {
-            const unsigned long long key = key_of(J);
-            kmax = key > kmax ? key : kmax;
-            kmin = key < kmin ? key : kmin;
+          for (int k = 0; k < 8; ++k) my_hist[lane + 32 * k] = 0ull;
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < NJ; ++i) {
+            const int J = lane + 32 * i;
+            if (J < nb) {
+              const unsigned long long key = key_of(J);
+              if ((key >> (top + 1)) == pref)
+                atomicAdd(&my_hist[(key >> s) & ((1u << w) - 1u)], packed_mass(srow[J]));
+            }
           }
+          __syncwarp();
+          // lane L scans buckets 255 - 8 L down to 248 - 8 L
+          unsigned long long loc[8], lsum = 0ull;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            loc[e] = my_hist[255 - 8 * lane - e];
+            lsum += loc[e];
+          }
+          unsigned long long incl = lsum;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const unsigned long long t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+          }
+          if (first && (__shfl_sync(0xffffffffu, incl, 31) >> 11) < target) {
+            keep_all = true;             // the whole row's mass rounds below 1 - thr
+            break;
+          }
+          first = false;
+          unsigned long long cum = above + (incl - lsum), before = 0ull;
+          int found = -1;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const unsigned long long nc = cum + loc[e];
+            if (found < 0 && (nc >> 11) >= target) {
+              found = e;
+              before = cum;
+            }
+            cum = nc;
+          }
+          const uint32_t bal = __ballot_sync(0xffffffffu, found >= 0);
+          if (bal == 0u) {                // cannot happen: the candidates and `above` reach the target
+            keep_all = true;
+            break;
+          }
+          const int src_lane = __ffs(bal) - 1;
+          const int e_sel = __shfl_sync(0xffffffffu, found, src_lane);
+          above = __shfl_sync(0xffffffffu, before, src_lane);
+          const int d_sel = 255 - 8 * src_lane - e_sel;
+          cnt = (int)(my_hist[d_sel] & 2047ull);
+          pref = (pref << w) | (unsigned long long)d_sel;
+          __syncwarp();   // the histogram is cleared by the next round
+          if (cnt == 1 || s == 0) break;
+          top = s - 1;
         }
-        kmax = warp_max(kmax);
-        kmin = warp_min(kmin);
-        unsigned long long vb = kmax;      // the boundary key
-        unsigned long long above = 0ull;   // packed mass of the keys above the candidates
-        bool single = true;
-        if (kmax != kmin) {
-          int top = 63 - __clzll((long long)(kmax ^ kmin));   // highest bit in which keys differ (< 63)
-          unsigned long long pref = kmax >> (top + 1);         // the bits above it, common to all keys
-          int cnt = 0;
-          int s = 0;
-          for (;;) {
-            const int w = min(8, top + 1);
-            s = top + 1 - w;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) my_hist[lane + 32 * k] = 0ull;
-            __syncwarp();
-#pragma unroll
-            for (int i = 0; i < NJ; ++i) {
-              const int J = lane + 32 * i;
-              if (J < nb) {
-                const unsigned long long key = key_of(J);
-                if ((key >> (top + 1)) == pref)
-                  atomicAdd(&my_hist[(key >> s) & ((1u << w) - 1u)], packed_mass(srow[J]));
-              }
-            }
-            __syncwarp();
-            // lane L scans buckets 255 - 8 L down to 248 - 8 L
-            unsigned long long loc[8], lsum = 0ull;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              loc[e] = my_hist[255 - 8 * lane - e];
-              lsum += loc[e];
-            }
-            unsigned long long incl = lsum;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-              const unsigned long long t = __shfl_up_sync(0xffffffffu, incl, o);
-              if (lane >= o) incl += t;
-            }
-            unsigned long long cum = above + (incl - lsum), before = 0ull;
-            int found = -1;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const unsigned long long nc = cum + loc[e];
-              if (found < 0 && (nc >> 11) >= target) {
-                found = e;
-                before = cum;
-              }
-              cum = nc;
-            }
-            const uint32_t bal = __ballot_sync(0xffffffffu, found >= 0);
-            const int src = __ffs(bal) - 1;   // bal != 0: the candidates and `above` reach the target
-            const int e_sel = __shfl_sync(0xffffffffu, found, src);
-            above = __shfl_sync(0xffffffffu, before, src);
-            const int d_sel = 255 - 8 * src - e_sel;
-            cnt = (int)(my_hist[d_sel] & 2047ull);
-            pref = (pref << w) | (unsigned long long)d_sel;
-            __syncwarp();   // the histogram is cleared by the next round
-            if (cnt == 1 || s == 0) break;
-            top = s - 1;
-          }
+        if (!keep_all) {
           if (cnt == 1) {
             // the one key with these leading bits
             unsigned long long best = 0ull;
@@ -434,6 +423,8 @@ __global__ void __launch_bounds__(kMaskThreads, 2) mask_kernel(const double* __r
             single = false;
           }
         }
+      }
+      if (!keep_all) {
         // Every block above vb is kept.  With a single block at vb it is kept
         // too; equal keys at vb are added in ascending index order until the
         // mass reaches the target.
@@ -462,36 +453,40 @@ __global__ void __launch_bounds__(kMaskThreads, 2) mask_kernel(const double* __r
           }
         }
       }
-
-      if (sta_t >= 0) {
-        int ti, hi_, wi;
-        block_tile(I, g, ti, hi_, wi);
-#pragma unroll 1
-        for (int i = 0; i < NJ; ++i) {
-          const int J = lane + 32 * i;
-          if (J >= nb) break;
-          int tj, hj, wj;
-          block_tile(J, g, tj, hj, wj);
-          if (abs(ti - tj) <= sta_t && abs(hi_ - hj) <= sta_h && abs(wi - wj) <= sta_w) keep |= 1u << i;
-        }
-      }
-
-      const size_t row = bh * nb + I;
-      int base = 0;
-      const uint32_t lt = (1u << lane) - 1u;
+    }
+    if (keep_all) {
 #pragma unroll
+      for (int i = 0; i < NJ; ++i)
+        if (lane + 32 * i < nb) keep |= 1u << i;
+    }
+
+    if (sta_t >= 0) {
+      int ti, hi_, wi;
+      block_tile(I, g, ti, hi_, wi);
+#pragma unroll 1
       for (int i = 0; i < NJ; ++i) {
         const int J = lane + 32 * i;
-        const bool k = (keep >> i) & 1u;
-        const uint32_t bal = __ballot_sync(0xffffffffu, k);
-        if (k) kv_idx[row * nb + base + __popc(bal & lt)] = J;
-        if (mask != nullptr && J < nb) mask[row * nb + J] = k ? 1 : 0;
-        base += __popc(bal);
+        if (J >= nb) break;
+        int tj, hj, wj;
+        block_tile(J, g, tj, hj, wj);
+        if (abs(ti - tj) <= sta_t && abs(hi_ - hj) <= sta_h && abs(wi - wj) <= sta_w) keep |= 1u << i;
       }
-      if (lane == 0) kv_count[row] = base;
-    }  // rows of this warp
-    __syncthreads();   // qs and sc are rewritten by the next group
-  }  // groups
+    }
+
+    int base = 0;
+    const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+    for (int i = 0; i < NJ; ++i) {
+      const int J = lane + 32 * i;
+      const bool k = (keep >> i) & 1u;
+      const uint32_t bal = __ballot_sync(0xffffffffu, k);
+      if (k) kv_idx[row * nb + base + __popc(bal & lt)] = J;
+      if (mask != nullptr && J < nb) mask[row * nb + J] = k ? 1 : 0;
+      base += __popc(bal);
+    }
+    if (lane == 0) kv_count[row] = base;
+    __syncwarp();   // srow is rewritten by the warp's next row
+  }
 }
 
 }  // namespace
@@ -523,40 +518,49 @@ cudaError_t launch_pool(const Dims& g, const void* q, const void* k, double* qba
   return launch_pool_t<64, 128>(g, q, k, qbar, kbar, ctrl, seq, st);
 }
 
-template <int D, int NJ>
-cudaError_t launch_mask_t(const Dims& g, const double* qbar, const double* kbar, double thr, int sta_t, int sta_h,
-                          int sta_w, int32_t* kv_count, int32_t* kv_idx, uint8_t* mask, cudaStream_t st) {
-  constexpr int R = mask_rows<NJ>();
-  const size_t smem = (size_t)R * (g.d + g.nb) * sizeof(double) + (size_t)kMaskWarps * 256 * sizeof(uint64_t);
-  const double scale = 1.0 / std::sqrt((double)g.d);
-  cudaError_t e = cudaFuncSetAttribute(mask_kernel<D, NJ>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+size_t mask_scores_bytes(const Dims& g) { return (size_t)g.B * g.heads * g.nb * g.nb * sizeof(double); }
+
+template <int NJ>
+cudaError_t launch_select_t(const Dims& g, const double* scores, double thr, int sta_t, int sta_h, int sta_w,
+                            int32_t* kv_count, int32_t* kv_idx, uint8_t* mask, cudaStream_t st) {
+  const size_t smem = (size_t)kSelWarps * (NJ * 32 * sizeof(double) + 256 * sizeof(uint64_t));
+  cudaError_t e = cudaFuncSetAttribute(select_kernel<NJ>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0, per_sm = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, mask_kernel<D, NJ>, kMaskThreads, smem)) !=
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_kernel<NJ>, kSelThreads, smem)) !=
       cudaSuccess)
     return e;
-  const int total = (g.nb + R - 1) / R * g.B * g.heads;
-  const int grid = std::max(1, std::min(total, sms * std::max(1, per_sm)));
-  mask_kernel<D, NJ><<<grid, kMaskThreads, smem, st>>>(qbar, kbar, g, thr, scale, sta_t, sta_h, sta_w, kv_count,
-                                                       kv_idx, mask);
+  const size_t rows = (size_t)g.B * g.heads * g.nb;
+  const size_t need = (rows + kSelWarps - 1) / kSelWarps;
+  const int grid = (int)std::max<size_t>(1, std::min<size_t>(need, (size_t)sms * std::max(1, per_sm)));
+  select_kernel<NJ><<<grid, kSelThreads, smem, st>>>(scores, g, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask);
   return cudaGetLastError();
 }
 
 template <int D>
-cudaError_t launch_mask_d(const Dims& g, const double* qbar, const double* kbar, double thr, int sta_t, int sta_h,
-                          int sta_w, int32_t* kv_count, int32_t* kv_idx, uint8_t* mask, cudaStream_t st) {
-  if (g.nb <= 128) return launch_mask_t<D, 4>(g, qbar, kbar, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask, st);
-  if (g.nb <= 256) return launch_mask_t<D, 8>(g, qbar, kbar, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask, st);
-  if (g.nb <= 512) return launch_mask_t<D, 16>(g, qbar, kbar, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask, st);
-  return launch_mask_t<D, 32>(g, qbar, kbar, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask, st);
+cudaError_t launch_scores_t(const Dims& g, const double* qbar, const double* kbar, double* scores, cudaStream_t st) {
+  const size_t smem = (size_t)(kScoreRows * kAStride + D * kBStride) * sizeof(double);
+  cudaError_t e = cudaFuncSetAttribute(scores_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const size_t tiles = (size_t)((g.nb + kScoreRows - 1) / kScoreRows) * ((g.nb + kScoreCols - 1) / kScoreCols) *
+                       g.B * g.heads;
+  if (tiles > 0x7FFFFFFFull) return cudaErrorInvalidValue;
+  scores_kernel<D><<<(unsigned)tiles, kScoreThreads, smem, st>>>(qbar, kbar, g, 1.0 / std::sqrt((double)D), scores);
+  return cudaGetLastError();
 }
 
-cudaError_t launch_mask(const Dims& g, const double* qbar, const double* kbar, double thr, int sta_t, int sta_h,
-                        int sta_w, int32_t* kv_count, int32_t* kv_idx, uint8_t* mask, cudaStream_t st) {
-  if (g.d == 128) return launch_mask_d<128>(g, qbar, kbar, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask, st);
-  return launch_mask_d<64>(g, qbar, kbar, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask, st);
+cudaError_t launch_mask(const Dims& g, const double* qbar, const double* kbar, double* scores, double thr,
+                        int sta_t, int sta_h, int sta_w, int32_t* kv_count, int32_t* kv_idx, uint8_t* mask,
+                        cudaStream_t st) {
+  cudaError_t e = (g.d == 128) ? launch_scores_t<128>(g, qbar, kbar, scores, st)
+                               : launch_scores_t<64>(g, qbar, kbar, scores, st);
+  if (e != cudaSuccess) return e;
+  if (g.nb <= 128) return launch_select_t<4>(g, scores, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask, st);
+  if (g.nb <= 256) return launch_select_t<8>(g, scores, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask, st);
+  if (g.nb <= 512) return launch_select_t<16>(g, scores, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask, st);
+  return launch_select_t<32>(g, scores, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask, st);
 }
 
 }  // namespace bsa

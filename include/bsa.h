@@ -84,9 +84,10 @@ BSA_API int64_t bsa_num_blocks(const bsa_shape* s);
 
 /* Bytes of device workspace that bsa_build_block_mask and bsa_attn_fwd need
  * for this shape: a control block (device error word), the pooled block means
- * of Q and K (2 * B*heads*nb*d doubles) and the attention work plan (one int2
- * per 128-row query tile; with 64-token blocks also 64 bytes of pairing
- * weights and 4 bytes of counts per block row; a work counter).  0 for an
+ * of Q and K (2 * B*heads*nb*d doubles), the reduced scores (B*heads*nb*nb
+ * doubles) and the attention work plan (one int2 per 128-row query tile; with
+ * 64-token blocks also 64 bytes of pairing weights and 4 bytes of counts per
+ * block row; a work counter), each part rounded up to 256 bytes.  0 for an
  * invalid shape. */
 BSA_API size_t bsa_workspace_bytes(const bsa_shape* s);
 

@@ -301,6 +301,121 @@ def masked_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, keep: np.ndarr
     return O, lse
 
 
+# --------------------------------------- Hilbert-curve order, sub-block scoring
+
+def hilbert_index(coords: Sequence[int], bits: int) -> int:
+    """Index of a point along the n-dimensional Hilbert curve of side 2^bits.
+
+    DFSAttn explainer, section 1 ("El barajado de la Curva de Hilbert"): tokens
+    are ordered along a 3-D Hilbert curve so that neighbours in the sequence
+    are neighbours in space and time.  The page does not say which Hilbert
+    curve; this is J. Skilling's construction ("Programming the Hilbert
+    curve", AIP Conf. Proc. 707, 2004), written from its description: the
+    coordinates are turned into the curve's "transposed" index by undoing the
+    excess work of the reflected Gray code level by level (from the top bit
+    down, an axis with the current bit set flips the lower bits of axis 0,
+    otherwise axes 0 and i exchange their lower bits), Gray-encoding across
+    the axes, and a final fix-up; the index interleaves the transposed words
+    from the top bit down, axis 0 first.
+    """
+    x = [int(c) for c in coords]
+    n = len(x)
+    top = 1 << (bits - 1)
+    q = top
+    while q > 1:
+        low = q - 1
+        for i in range(n):
+            if x[i] & q:
+                x[0] ^= low
+            else:
+                t = (x[0] ^ x[i]) & low
+                x[0] ^= t
+                x[i] ^= t
+        q >>= 1
+    for i in range(1, n):
+        x[i] ^= x[i - 1]
+    t = 0
+    q = top
+    while q > 1:
+        if x[n - 1] & q:
+            t ^= q - 1
+        q >>= 1
+    for i in range(n):
+        x[i] ^= t
+    h = 0
+    for b in range(bits - 1, -1, -1):
+        for i in range(n):
+            h = (h << 1) | ((x[i] >> b) & 1)
+    return h
+
+
+def hilbert_bits(T: int, H: int, W: int) -> int:
+    """Bits per axis of the smallest power-of-two cube that holds the grid."""
+    return max(1, int(math.ceil(math.log2(max(T, H, W)))))
+
+
+def hilbert_order(T: int, H: int, W: int) -> np.ndarray:
+    """Position p -> original token n = t*H*W + h*W + w along the 3-D Hilbert
+    curve of the smallest power-of-two cube holding the T x H x W grid, axes
+    (t, h, w) in that order, points outside the grid skipped (the plainest
+    reading for grids that are not a power-of-two cube)."""
+    bits = hilbert_bits(T, H, W)
+    keys = []
+    for t in range(T):
+        for h in range(H):
+            for w in range(W):
+                keys.append(hilbert_index((t, h, w), bits))
+    return np.argsort(np.asarray(keys, dtype=np.int64), kind="stable").astype(np.int64)
+
+
+def reorder_by(x_bnhd: np.ndarray, order: np.ndarray, block: int) -> np.ndarray:
+    """[B, N, heads, d] -> [B, heads, Npad, d] with position p holding token
+    order[p], zero tail (the layout change of ``reorder`` for any order)."""
+    B, N, heads, d = x_bnhd.shape
+    y = np.zeros((B, heads, padded_len(N, block), d), dtype=np.float64)
+    for p in range(N):
+        y[:, :, p, :] = x_bnhd[:, order[p], :, :]
+    return y
+
+
+def subblock_scores(q_bhnd: np.ndarray, k_bhnd: np.ndarray, N: int, block: int, sub: int,
+                    scale: Optional[float] = None) -> np.ndarray:
+    """Hierarchical block importance from sub-block scores: [.., nb, nb], rows sum to 1.
+
+    DFSAttn explainer, section 2 ("La puntuacion de Sub-bloque"): instead of
+    judging a block by its average, blocks are split into smaller sub-blocks
+    and their finer scores are added up.  Reading: Q and K are mean-pooled over
+    sub-blocks of `sub` tokens (valid tokens only; `sub` divides the block
+    size), the reduced attention is taken at sub-block resolution (a row
+    softmax over all key sub-blocks), and block I's importance for block J is
+    the mass its query sub-blocks give to J's key sub-blocks, summed over J's
+    sub-blocks and averaged over I's valid query sub-blocks.  With sub ==
+    block this is NABLA's reduced map.
+    """
+    assert block % sub == 0
+    qs = block_means(q_bhnd, N, sub)           # [.., ns, d]
+    ks = block_means(k_bhnd, N, sub)
+    ns_valid = -(-N // sub)                    # sub-blocks holding at least one valid token
+    qs, ks = qs[..., :ns_valid, :], ks[..., :ns_valid, :]
+    A = reduced_attention(qs, ks, scale)       # [.., ns_valid, ns_valid]
+    per = block // sub
+    nb = padded_len(N, block) // block
+    out = np.zeros(A.shape[:-2] + (nb, nb), dtype=np.float64)
+    for I in range(nb):
+        a_rows = [a for a in range(I * per, (I + 1) * per) if a < ns_valid]
+        for J in range(nb):
+            b_cols = [b for b in range(J * per, (J + 1) * per) if b < ns_valid]
+            if b_cols:
+                out[..., I, J] = A[..., a_rows, :][..., :, b_cols].sum(axis=(-1, -2)) / len(a_rows)
+    return out
+
+
+def block_mask_subblock(q_bhnd: np.ndarray, k_bhnd: np.ndarray, N: int, block: int, sub: int, thr: float,
+                        scale: Optional[float] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """Sub-block importance -> the same CDF rule as NABLA.  Returns (keep, ambiguous)."""
+    return cdf_keep(subblock_scores(q_bhnd, k_bhnd, N, block, sub, scale), thr)
+
+
 # ------------------------------------------ block-sparse attention backward
 
 def masked_attention_backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, keep: np.ndarray, dO: np.ndarray,

@@ -42,11 +42,12 @@ def test_shape_arithmetic(bsa):
     assert bsa.seq_len(s) == 32760
     assert bsa.padded_len(s) == 32768
     assert bsa.num_blocks(s) == 512
-    # control block | q and k block means (double) | attention plan (one int2 per 128-row
-    # tile, then pairing weights of 32 neighbours (uint16) and a count (int32) per block
-    # row, then a 256-byte slot for the work counter of the attention kernel)
-    assert bsa.workspace_bytes(s) == (256 + 2 * 12 * 512 * 128 * 8 + 12 * 256 * 8 + 12 * 512 * 64 + 12 * 512 * 4
-                                      + 256)
+    # control block | q and k block means (double) | reduced scores (double) | attention
+    # plan (one int2 per 128-row tile, then pairing weights of 32 neighbours (uint16) and
+    # a count (int32) per block row, then a 256-byte slot for the work counter of the
+    # attention kernel)
+    assert bsa.workspace_bytes(s) == (256 + 2 * 12 * 512 * 128 * 8 + 12 * 512 * 512 * 8 + 12 * 256 * 8
+                                      + 12 * 512 * 64 + 12 * 512 * 4 + 256)
     s = bsa.make_shape(1, 33, 45, 80, 24, 128, 128, 8)
     assert (bsa.seq_len(s), bsa.padded_len(s), bsa.num_blocks(s)) == (118800, 118912, 929)
     assert bsa.validate_shape(s) == 0

@@ -55,6 +55,6 @@ def test_kernel_launch_count_per_step():
     sys.path.insert(0, ROOT)
     import bench
     from block_sparse_attention_fractal_b200 import synth
-    assert bench.kernel_launches_per_step(synth.WORKLOADS["wan480p"]) == 7
-    assert bench.kernel_launches_per_step(synth.WORKLOADS["hunyuan720p"]) == 6
+    assert bench.kernel_launches_per_step(synth.WORKLOADS["wan480p"]) == 8
+    assert bench.kernel_launches_per_step(synth.WORKLOADS["hunyuan720p"]) == 7
     assert bench.kernel_launches_per_step(synth.WORKLOADS["density_sweep"]) == 6

@@ -496,6 +496,105 @@ def test_pins_catch_a_backward_without_the_softmax_jacobian_term(monkeypatch):
         test_backward_equals_library_autograd(96, 32)
 
 
+# ------------------------------------------------- Hilbert order, sub-blocks
+
+def test_hilbert_2x2x2_matches_hand_derivation(golden_dir):
+    g = _read_golden(os.path.join(golden_dir, "hilbert_order_2x2x2.txt"))
+    assert oracle.hilbert_order(2, 2, 2).tolist() == g["order"]
+    assert [oracle.hilbert_index((n // 4, (n // 2) % 2, n % 2), 1) for n in range(8)] == g["index"]
+
+
+def _hilbert_curve_properties(bits):
+    """The cube's points in curve order, checked for the properties that
+    define a Hilbert curve: a bijection onto [0, 8^bits), consecutive points
+    one step apart, and every aligned sub-cube of side 2^k visited as one
+    contiguous run of 8^k points."""
+    side = 1 << bits
+    pts = [(t, h, w) for t in range(side) for h in range(side) for w in range(side)]
+    idx = [nabla.hilbert_index(p, bits) for p in pts]
+    if sorted(idx) != list(range(side ** 3)):
+        return False
+    path = [p for _, p in sorted(zip(idx, pts))]
+    if any(sum(abs(a - b) for a, b in zip(path[i], path[i + 1])) != 1 for i in range(len(path) - 1)):
+        return False
+    for k in range(1, bits):
+        runs = {}
+        for pos, p in enumerate(path):
+            runs.setdefault(tuple(c >> k for c in p), []).append(pos)
+        for positions in runs.values():
+            if positions != list(range(positions[0], positions[0] + 8 ** k)):
+                return False
+    return path[0] == (0, 0, 0)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_hilbert_curve_is_continuous_and_hierarchical(bits):
+    assert _hilbert_curve_properties(bits)
+
+
+def test_pins_catch_a_hilbert_curve_without_the_gray_encoding(monkeypatch):
+    def bad(coords, bits):          # interleaves the raw coordinate bits (a Z-order curve)
+        h = 0
+        for b in range(bits - 1, -1, -1):
+            for c in coords:
+                h = (h << 1) | ((int(c) >> b) & 1)
+        return h
+    monkeypatch.setattr(nabla, "hilbert_index", bad)
+    assert not _hilbert_curve_properties(2)
+
+
+def test_hilbert_order_of_a_ragged_grid_is_the_cube_order_restricted():
+    T, H, W = 3, 5, 6
+    o = oracle.hilbert_order(T, H, W)
+    assert sorted(o.tolist()) == list(range(T * H * W))
+    bits = oracle.hilbert_bits(T, H, W)
+    keys = [nabla.hilbert_index((n // (H * W), (n // W) % H, n % W), bits) for n in o]
+    assert keys == sorted(keys)
+    # a reorder by it is a bijection of the token rows, zero tail
+    x = np.random.default_rng(13).standard_normal((1, T * H * W, 2, 3))
+    y = nabla.reorder_by(x, o, 16)
+    assert np.all(y[:, :, T * H * W:] == 0)
+    assert np.array_equal(y[0, 1, 7], x[0, o[7], 1])
+
+
+def test_subblock_scores_with_one_subblock_per_block_is_the_reduced_map():
+    rng = np.random.default_rng(14)
+    N, bs, d = 100, 32, 8
+    q = rng.standard_normal((1, 2, nabla.padded_len(N, bs), d))
+    k = rng.standard_normal((1, 2, nabla.padded_len(N, bs), d))
+    q[:, :, N:] = 0
+    k[:, :, N:] = 0
+    want = oracle.reduced_attention(oracle.block_means(q, N, bs), oracle.block_means(k, N, bs))
+    assert np.allclose(oracle.subblock_scores(q, k, N, bs, bs), want, rtol=0, atol=1e-15)
+
+
+def test_subblock_scores_closed_forms():
+    rng = np.random.default_rng(15)
+    N, bs, sub, d = 100, 32, 8, 4       # 13 valid sub-blocks: 4 + 4 + 4 + 1
+    Npad = nabla.padded_len(N, bs)
+    q = rng.standard_normal((1, 1, Npad, d))
+    # identical key sub-blocks: every query sub-block spreads its mass evenly,
+    # so block J's importance is its share of the valid key sub-blocks
+    k = np.tile(rng.standard_normal((1, 1, 1, d)), (1, 1, Npad, 1))
+    M = oracle.subblock_scores(q, k, N, bs, sub)
+    assert np.allclose(M[0, 0], np.array([4, 4, 4, 1]) / 13.0, rtol=0, atol=1e-15)
+    # rows are distributions for any input
+    k = rng.standard_normal((1, 1, Npad, d)) * 3
+    M = oracle.subblock_scores(q, k, N, bs, sub)
+    assert np.all(M >= 0) and np.allclose(M.sum(-1), 1.0, atol=1e-12)
+
+
+def test_pins_catch_subblock_scores_that_average_instead_of_summing(monkeypatch):
+    orig = nabla.subblock_scores
+
+    def bad(q, k, N, block, sub, scale=None):
+        per = block // sub
+        return orig(q, k, N, block, sub, scale) / per
+    monkeypatch.setattr(oracle, "subblock_scores", bad)
+    with pytest.raises(AssertionError):
+        test_subblock_scores_closed_forms()
+
+
 def test_lists_roundtrip():
     rng = np.random.default_rng(9)
     keep = rng.random((2, 3, 7, 7)) < 0.4
