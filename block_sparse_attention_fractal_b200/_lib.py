@@ -60,6 +60,8 @@ def _load() -> ctypes.CDLL:
                                              P, P, P, P, ctypes.c_size_t, P]),
         "bsa_attn_fwd": (st, [S, P, P, P, P, P, ctypes.c_float, P, P, P, ctypes.c_size_t, P]),
         "bsa_attn_fwd_baseline": (st, [S, P, P, P, P, P, ctypes.c_float, P, P, P, ctypes.c_size_t, P]),
+        "bsa_attn_bwd_workspace_bytes": (ctypes.c_size_t, [S]),
+        "bsa_attn_bwd": (st, [S, P, P, P, P, P, P, P, P, ctypes.c_float, P, P, P, P, ctypes.c_size_t, P]),
         "bsa_check_device_status": (st, [P, P]),
         "bsa_status_string": (ctypes.c_char_p, [st]),
     }
@@ -185,6 +187,19 @@ def attn_fwd_baseline(s: Shape, q: torch.Tensor, k: torch.Tensor, v: torch.Tenso
                                      float(scale), _ptr(o), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(),
                                      _stream(q.device)),
            "bsa_attn_fwd_baseline")
+
+
+def attn_bwd_workspace_bytes(s: Shape) -> int:
+    return get_lib().bsa_attn_bwd_workspace_bytes(ctypes.byref(s))
+
+
+def attn_bwd(s: Shape, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, dO: torch.Tensor,
+             lse: torch.Tensor, kv_count: torch.Tensor, kv_idx: torch.Tensor, scale: float, dq: torch.Tensor,
+             dk: torch.Tensor, dv: torch.Tensor, ws: torch.Tensor) -> None:
+    _check(get_lib().bsa_attn_bwd(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse),
+                                  _ptr(kv_count), _ptr(kv_idx), float(scale), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
+                                  ws.numel() * ws.element_size(), _stream(q.device)),
+           "bsa_attn_bwd")
 
 
 def check_device_status(ws: torch.Tensor) -> int:

@@ -240,6 +240,87 @@ bsa_status bsa_attn_fwd_baseline(const bsa_shape* s, const void* q, const void* 
   return attn_common(s, q, k, v, kv_count, kv_idx, scale, o, lse_or_null, workspace, ws_bytes, stream, true);
 }
 
+}  // extern "C"
+
+namespace {
+
+// Backward workspace: control block | D | bit matrix | transposed counts |
+// transposed lists | planner region of the query tiles | of the KV tiles.
+struct BwdLayout {
+  size_t Dv, bits, q_count, q_idx, plan_q, plan_kv, total;
+};
+
+BwdLayout bwd_layout(const Dims& g) {
+  const size_t bh = (size_t)g.B * g.heads;
+  const size_t nw = (size_t)(g.nb + 31) / 32;
+  BwdLayout L;
+  L.Dv = sizeof(Ctrl);
+  L.bits = L.Dv + align256(bh * g.Npad * sizeof(float));
+  L.q_count = L.bits + align256(bh * g.nb * nw * sizeof(uint32_t));
+  L.q_idx = L.q_count + align256(bh * g.nb * sizeof(int32_t));
+  L.plan_q = L.q_idx + align256(bh * g.nb * g.nb * sizeof(int32_t));
+  L.plan_kv = L.plan_q + align256(bsa::plan_region_bytes(g));
+  L.total = L.plan_kv + align256(bsa::plan_region_bytes(g));
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t bsa_attn_bwd_workspace_bytes(const bsa_shape* s) {
+  Dims g;
+  return check_shape(s, &g) == BSA_OK ? bwd_layout(g).total : 0;
+}
+
+bsa_status bsa_attn_bwd(const bsa_shape* s, const void* q, const void* k, const void* v, const void* o,
+                        const void* dO, const float* lse, const int32_t* kv_count, const int32_t* kv_idx, float scale,
+                        void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, bsa_stream_t stream) {
+  Dims g;
+  bsa_status st = check_shape(s, &g);
+  if (st != BSA_OK) return st;
+  if (g.nb > BSA_MAX_BLOCKS) return BSA_ERR_UNSUPPORTED;
+  const void* ptrs[13] = {q, k, v, o, dO, lse, kv_count, kv_idx, dq, dk, dv, workspace, workspace};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return BSA_ERR_INVALID_ARG;
+  if (dq == dk || dq == dv || dk == dv) return BSA_ERR_INVALID_ARG;
+  const BwdLayout L = bwd_layout(g);
+  if (ws_bytes < L.total) return BSA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || scale < 0.0f) return BSA_ERR_INVALID_ARG;
+  if (scale == 0.0f) scale = (float)(1.0 / std::sqrt((double)g.d));
+  char* ws = (char*)workspace;
+  cudaStream_t cs = (cudaStream_t)stream;
+  bsa::BwdArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.dO = dO;
+  a.lse = lse;
+  a.Dv = (const float*)(ws + L.Dv);
+  a.kv_count = kv_count;
+  a.kv_idx = kv_idx;
+  a.q_count = (const int32_t*)(ws + L.q_count);
+  a.q_idx = (const int32_t*)(ws + L.q_idx);
+  int2* items_q = (int2*)(ws + L.plan_q);
+  int2* items_kv = (int2*)(ws + L.plan_kv);
+  a.items_q = items_q;
+  a.items_kv = items_kv;
+  a.work_q = bsa::plan_work_counter(g, items_q);
+  a.work_kv = bsa::plan_work_counter(g, items_kv);
+  a.scale = scale;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.ctrl = (Ctrl*)workspace;
+  a.seq = bsa::next_launch_seq();
+  cudaError_t e = bsa::launch_bwd_prep(g, o, dO, kv_count, kv_idx, (float*)(ws + L.Dv), (uint32_t*)(ws + L.bits),
+                                       (int32_t*)(ws + L.q_count), (int32_t*)(ws + L.q_idx), cs);
+  if (e != cudaSuccess) return BSA_ERR_CUDA;
+  if (bsa::launch_plan(g, kv_count, kv_idx, items_q, cs) != cudaSuccess) return BSA_ERR_CUDA;
+  if (bsa::launch_plan(g, a.q_count, a.q_idx, items_kv, cs) != cudaSuccess) return BSA_ERR_CUDA;
+  return from_cuda(bsa::launch_attn_bwd(g, a, cs));
+}
+
 bsa_status bsa_check_device_status(void* workspace, bsa_stream_t stream) {
   if (workspace == nullptr || !aligned16(workspace)) return BSA_ERR_INVALID_ARG;
   cudaStream_t cs = (cudaStream_t)stream;

@@ -60,4 +60,27 @@ cudaError_t launch_attn_tc2(const Dims& g, const void* q, const void* k, const v
                             const int32_t* kv_idx, const int2* items, int* work, float scale, void* o, float* lse,
                             Ctrl* ctrl, uint32_t seq, cudaStream_t st);
 
+// Backward pass (attn_bwd.cu).  Every pointer is device memory; the planner
+// regions (items_q / items_kv with their work counters) are filled by
+// launch_plan from the forward lists and from the transposed lists.
+struct BwdArgs {
+  const void *q, *k, *v, *dO;         // [B, heads, Npad, d] bf16, kernel order
+  const float* lse;                   // [B, heads, Npad] natural-log LSE of the forward pass
+  const float* Dv;                    // [B, heads, Npad] rowsum(dO * O) (launch_bwd_prep)
+  const int32_t *kv_count, *kv_idx;   // forward lists
+  const int32_t *q_count, *q_idx;     // transposed lists (launch_bwd_prep)
+  const int2 *items_q, *items_kv;     // planner tiles of query blocks / of KV blocks
+  int *work_q, *work_kv;              // their work counters
+  float scale;
+  void *dq, *dk, *dv;                 // [B, heads, Npad, d] bf16 outputs
+  Ctrl* ctrl;
+  uint32_t seq;
+};
+// D = rowsum(dO * O), the bit matrix of the forward lists (`bits`,
+// [B, heads, nb, ceil(nb / 32)] uint32) and the transposed lists.
+cudaError_t launch_bwd_prep(const Dims& g, const void* o, const void* dO, const int32_t* kv_count,
+                            const int32_t* kv_idx, float* Dv, uint32_t* bits, int32_t* q_count, int32_t* q_idx,
+                            cudaStream_t st);
+cudaError_t launch_attn_bwd(const Dims& g, const BwdArgs& a, cudaStream_t st);
+
 }  // namespace bsa

@@ -139,20 +139,36 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __nv_bfloat16*
 
 // scores_kernel: S[bh][I][J] = scale * qbar_I . kbar_J for one 32 x 64 tile of
 // one (b, head) per CTA, on the fp64 tensor cores (mma.sync m8n8k4, fp64
-// multiply-add).  The tile's qbar rows and kbar columns are staged in shared
-// memory first (rows padded so the fragment loads of a half-warp hit 16
-// different banks); each of the 4 warps computes 32 rows x 16 columns.
+// multiply-add).  The head dimension is walked in chunks of 32: each chunk's
+// qbar rows and kbar columns are copied to shared memory with cp.async (two
+// buffers, the next chunk in flight while the current one is multiplied),
+// with rows padded so the fragment loads of a half-warp hit 16 different
+// banks.  Each of the 4 warps computes 32 rows x 16 columns.
 constexpr int kScoreRows = 32, kScoreCols = 64, kScoreThreads = 128;
-constexpr int kAStride = 132;                 // doubles per staged qbar row (D = 128 + 4)
+constexpr int kKC = 32;                       // head-dimension chunk
+constexpr int kAStride = kKC + 4;             // doubles per staged qbar row
 constexpr int kBStride = kScoreCols + 4;      // doubles per staged kbar row
+constexpr int kStageDoubles = kScoreRows * kAStride + kKC * kBStride;
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+  const int n = valid ? 16 : 0;   // zero-fill when the source is outside the matrix
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(d), "l"(src), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async8(void* dst, const void* src, bool valid) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+  const int n = valid ? 8 : 0;
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;\n" ::"r"(d), "l"(src), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
 
 template <int D>
 __global__ void __launch_bounds__(kScoreThreads) scores_kernel(const double* __restrict__ qbar,
                                                                const double* __restrict__ kbar, Dims g,
                                                                double scale, double* __restrict__ scores) {
   extern __shared__ __align__(16) double sm[];
-  double* As = sm;                                  // [kScoreRows][kAStride]
-  double* Bs = sm + kScoreRows * kAStride;          // [D][kBStride]
   const int nb = g.nb;
   const int tiles_i = (nb + kScoreRows - 1) / kScoreRows, tiles_j = (nb + kScoreCols - 1) / kScoreCols;
   const int tj = blockIdx.x % tiles_j;
@@ -161,15 +177,25 @@ __global__ void __launch_bounds__(kScoreThreads) scores_kernel(const double* __r
   const int I0 = ti * kScoreRows, J0 = tj * kScoreCols;
   const double* qsrc = qbar + (bh * nb) * D;
   const double* ksrc = kbar + bh * D * (size_t)nb;
-  for (int i = threadIdx.x; i < kScoreRows * D; i += kScoreThreads) {
-    const int r = i / D, c = i % D;
-    As[r * kAStride + c] = (I0 + r < nb) ? qsrc[(size_t)(I0 + r) * D + c] : 0.0;
-  }
-  for (int i = threadIdx.x; i < D * kScoreCols; i += kScoreThreads) {
-    const int k = i / kScoreCols, c = i % kScoreCols;
-    Bs[k * kBStride + c] = (J0 + c < nb) ? ksrc[(size_t)k * nb + J0 + c] : 0.0;
-  }
-  __syncthreads();
+  // chunk kc into buffer buf: 32 x 32 of qbar (16-byte pieces), 32 x 64 of
+  // kbar (8-byte pieces); pieces past the matrix are zero-filled (their
+  // source address is clamped to the matrix start, never read)
+  auto stage = [&](int kc, int buf) {
+    double* As = sm + buf * kStageDoubles;
+    double* Bs = As + kScoreRows * kAStride;
+    for (int i = threadIdx.x; i < kScoreRows * kKC / 2; i += kScoreThreads) {
+      const int r = i / (kKC / 2), c2 = i % (kKC / 2);
+      const bool ok = I0 + r < nb;
+      cp_async16(As + r * kAStride + 2 * c2, ok ? qsrc + (size_t)(I0 + r) * D + kc * kKC + 2 * c2 : qsrc, ok);
+    }
+    // kbar rows are nb doubles long (nb may be odd): 8-byte pieces
+    for (int i = threadIdx.x; i < kKC * kScoreCols; i += kScoreThreads) {
+      const int k = i / kScoreCols, c = i % kScoreCols;
+      const bool ok = J0 + c < nb;
+      cp_async8(Bs + k * kBStride + c, ok ? ksrc + (size_t)(kc * kKC + k) * nb + J0 + c : ksrc, ok);
+    }
+    cp_async_commit();
+  };
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int gq = lane >> 2, tq = lane & 3;
   double acc[4][2][2];
@@ -177,20 +203,35 @@ __global__ void __launch_bounds__(kScoreThreads) scores_kernel(const double* __r
   for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
     for (int n = 0; n < 2; ++n) acc[mt][n][0] = acc[mt][n][1] = 0.0;
-#pragma unroll 4
-  for (int ks = 0; ks < D / 4; ++ks) {
-    double av[4], bv[2];
+  constexpr int NC = D / kKC;
+  stage(0, 0);
+#pragma unroll 1
+  for (int kc = 0; kc < NC; ++kc) {
+    if (kc + 1 < NC) {
+      stage(kc + 1, (kc + 1) & 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const double* As = sm + (kc & 1) * kStageDoubles;
+    const double* Bs = As + kScoreRows * kAStride;
 #pragma unroll
-    for (int mt = 0; mt < 4; ++mt) av[mt] = As[(mt * 8 + gq) * kAStride + 4 * ks + tq];
+    for (int ks = 0; ks < kKC / 4; ++ks) {
+      double av[4], bv[2];
 #pragma unroll
-    for (int n = 0; n < 2; ++n) bv[n] = Bs[(4 * ks + tq) * kBStride + wid * 16 + n * 8 + gq];
+      for (int mt = 0; mt < 4; ++mt) av[mt] = As[(mt * 8 + gq) * kAStride + 4 * ks + tq];
 #pragma unroll
-    for (int mt = 0; mt < 4; ++mt)
+      for (int n = 0; n < 2; ++n) bv[n] = Bs[(4 * ks + tq) * kBStride + wid * 16 + n * 8 + gq];
 #pragma unroll
-      for (int n = 0; n < 2; ++n)
-        asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};\n"
-                     : "+d"(acc[mt][n][0]), "+d"(acc[mt][n][1])
-                     : "d"(av[mt]), "d"(bv[n]));
+      for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+          asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};\n"
+                       : "+d"(acc[mt][n][0]), "+d"(acc[mt][n][1])
+                       : "d"(av[mt]), "d"(bv[n]));
+    }
+    __syncthreads();   // the buffer is refilled two chunks on
   }
   // accumulator element (row gq + 8 mt, column 2 tq + e) of each 8 x 8 tile
 #pragma unroll
@@ -215,6 +256,8 @@ __global__ void __launch_bounds__(kScoreThreads) scores_kernel(const double* __r
 
 constexpr int kSelThreads = 256;             // 8 warps, one row each at a time
 constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kHistSlots = 256 + 32;
+__device__ __forceinline__ int hslot(int b) { return b + (b >> 3); }
 
 __device__ __forceinline__ double warp_sum(double v) {
 #pragma unroll
@@ -266,8 +309,10 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __res
   const int nb = g.nb;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   double* srow = ssm + wid * (NJ * 32);                                     // this warp's row
+  // histogram of 256 buckets, bucket b at b + b / 8 (the scan's lanes read 8
+  // consecutive buckets each: the padding spreads them over the banks)
   unsigned long long* my_hist =
-      reinterpret_cast<unsigned long long*>(ssm + kSelWarps * NJ * 32) + wid * 256;
+      reinterpret_cast<unsigned long long*>(ssm + kSelWarps * NJ * 32) + wid * kHistSlots;
   const unsigned long long target = __double2ull_rn((1.0 - thr) * kMassScale);
   const size_t total_rows = (size_t)g.B * g.heads * nb;
 
@@ -352,7 +397,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __res
           const int w = min(8, top + 1);
           s = top + 1 - w;
 #pragma unroll
-          for (int k = 0; k < 8; ++k) my_hist[lane + 32 * k] = 0ull;
+          for (int k = 0; k < kHistSlots / 32; ++k) my_hist[lane + 32 * k] = 0ull;
           __syncwarp();
 #pragma unroll
           for (int i = 0; i < NJ; ++i) {
@@ -360,7 +405,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __res
             if (J < nb) {
               const unsigned long long key = key_of(J);
               if ((key >> (top + 1)) == pref)
-                atomicAdd(&my_hist[(key >> s) & ((1u << w) - 1u)], packed_mass(srow[J]));
+                atomicAdd(&my_hist[hslot((int)((key >> s) & ((1u << w) - 1u)))], packed_mass(srow[J]));
             }
           }
           __syncwarp();
@@ -368,7 +413,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __res
           unsigned long long loc[8], lsum = 0ull;
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            loc[e] = my_hist[255 - 8 * lane - e];
+            loc[e] = my_hist[hslot(255 - 8 * lane - e)];
             lsum += loc[e];
           }
           unsigned long long incl = lsum;
@@ -402,7 +447,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __res
           const int e_sel = __shfl_sync(0xffffffffu, found, src_lane);
           above = __shfl_sync(0xffffffffu, before, src_lane);
           const int d_sel = 255 - 8 * src_lane - e_sel;
-          cnt = (int)(my_hist[d_sel] & 2047ull);
+          cnt = (int)(my_hist[hslot(d_sel)] & 2047ull);
           pref = (pref << w) | (unsigned long long)d_sel;
           __syncwarp();   // the histogram is cleared by the next round
           if (cnt == 1 || s == 0) break;
@@ -523,7 +568,7 @@ size_t mask_scores_bytes(const Dims& g) { return (size_t)g.B * g.heads * g.nb * 
 template <int NJ>
 cudaError_t launch_select_t(const Dims& g, const double* scores, double thr, int sta_t, int sta_h, int sta_w,
                             int32_t* kv_count, int32_t* kv_idx, uint8_t* mask, cudaStream_t st) {
-  const size_t smem = (size_t)kSelWarps * (NJ * 32 * sizeof(double) + 256 * sizeof(uint64_t));
+  const size_t smem = (size_t)kSelWarps * (NJ * 32 * sizeof(double) + kHistSlots * sizeof(uint64_t));
   cudaError_t e = cudaFuncSetAttribute(select_kernel<NJ>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0, per_sm = 0;
@@ -541,7 +586,7 @@ cudaError_t launch_select_t(const Dims& g, const double* scores, double thr, int
 
 template <int D>
 cudaError_t launch_scores_t(const Dims& g, const double* qbar, const double* kbar, double* scores, cudaStream_t st) {
-  const size_t smem = (size_t)(kScoreRows * kAStride + D * kBStride) * sizeof(double);
+  const size_t smem = 2 * (size_t)kStageDoubles * sizeof(double);
   cudaError_t e = cudaFuncSetAttribute(scores_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const size_t tiles = (size_t)((g.nb + kScoreRows - 1) / kScoreRows) * ((g.nb + kScoreCols - 1) / kScoreCols) *

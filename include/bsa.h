@@ -179,6 +179,37 @@ BSA_API bsa_status bsa_attn_fwd(const bsa_shape* s, const void* q, const void* k
                         void* o, float* lse_or_null,
                         void* workspace, size_t ws_bytes, bsa_stream_t stream);
 
+/* Bytes of device workspace bsa_attn_bwd needs for this shape (0 for an
+ * invalid shape): a control block (device error word), D = rowsum(dO * O)
+ * (B*heads*Npad floats), a bit matrix of the block mask (B*heads*nb*
+ * ceil(nb/32) words), the transposed lists (B*heads*nb*(nb+1) int32) and two
+ * attention work plans, each part rounded up to 256 bytes.  Initialise the
+ * control block once with bsa_workspace_init. */
+BSA_API size_t bsa_attn_bwd_workspace_bytes(const bsa_shape* s);
+
+/* Block-sparse attention backward: the gradients of bsa_attn_fwd with respect
+ * to Q, K and V, following the same block mask.  NABLA summary, "Contribuciones
+ * Clave" ("Aceleracion de Doble Fase": the block-sparse attention also runs in
+ * pre-training and fine-tuning).  For every valid query row q of block I and
+ * the valid keys k of the blocks I keeps, with P = exp(scale Q.K - lse):
+ *   dV_k = sum_q P[q,k] dO_q,  dS = P (dO_q . V_k - dO_q . O_q),
+ *   dQ_q = scale sum_k dS[q,k] K_k,  dK_k = scale sum_q dS[q,k] Q_q.
+ * bf16 operands (P and dS rounded to bf16 for the products, as the forward
+ * rounds P), fp32 accumulation, bf16 outputs.
+ *   q, k, v, o, dO: device, [B, heads, Npad, d] bf16 in kernel order (o: the
+ *       forward output, dO: the gradient of the loss with respect to it).
+ *   lse: device, [B, heads, Npad] float32, the forward pass's lse_or_null.
+ *   kv_count, kv_idx: the lists the forward pass used.
+ *   scale: as for bsa_attn_fwd (0 selects 1/sqrt(d)).
+ *   dq, dk, dv: device, [B, heads, Npad, d] bf16, written (padded rows 0);
+ *       pairwise distinct.
+ *   workspace / ws_bytes: at least bsa_attn_bwd_workspace_bytes(s).
+ * Errors as for bsa_attn_fwd. */
+BSA_API bsa_status bsa_attn_bwd(const bsa_shape* s, const void* q, const void* k, const void* v, const void* o,
+                                const void* dO, const float* lse, const int32_t* kv_count, const int32_t* kv_idx,
+                                float scale, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
+                                bsa_stream_t stream);
+
 /* Same contract as bsa_attn_fwd, computed by the legacy warp-level
  * mma.sync tensor-core kernel instead of the tcgen05 one.  Kept as the measured
  * baseline the tcgen05 kernel is compared with. */
