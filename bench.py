@@ -437,6 +437,36 @@ def run_ours(args, w, rank, world, dist):
     if plan.status() != 0:
         raise RuntimeError("device status not OK after the timed steps")
 
+    # ---- the backward pass (not part of `value`): K steps of bsa_attn_bwd on
+    # the same lists, CUDA events on the launching stream, L2 flushed between
+    bwd = None
+    if args.bwd and not args.baseline_kernel:
+        g = torch.Generator().manual_seed(99)
+        dO = torch.randn(plan.o.shape, generator=g).to(torch.bfloat16).to(dev)
+        if plan.lse is None:
+            plan.lse = torch.empty(w.B, w.heads, plan.Npad, dtype=torch.float32, device=dev)
+        plan.attention_step()
+        dq, dk, dv = (torch.empty_like(plan.q) for _ in range(3))
+        bws = torch.zeros((bsa.attn_bwd_workspace_bytes(shape) + 15) // 16 * 16, dtype=torch.uint8, device=dev)
+        bsa.workspace_init(bws)
+        run_bwd = lambda: bsa.attn_bwd(shape, plan.q, plan.k, plan.v, plan.o, dO, plan.lse, plan.kv_count,
+                                       plan.kv_idx, 0.0, dq, dk, dv, bws)
+        for _ in range(args.warmup):
+            run_bwd()
+        torch.cuda.synchronize()
+        if bsa.check_device_status(bws) != 0:
+            raise RuntimeError("device status not OK after the backward warm-up")
+        bt = []
+        for _ in range(args.steps):
+            flush.fill_(1)
+            b0, b1 = ev(), ev()
+            b0.record(stream)
+            run_bwd()
+            b1.record(stream)
+            bt.append((b0, b1))
+        torch.cuda.synchronize()
+        bwd_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in bt) / args.steps, dist, dev)
+        bwd = {"ms": bwd_ms, "flops": 2.5 * flops_step}
     if rank != 0:
         return
     peaks, src = load_peaks()
@@ -507,6 +537,12 @@ def run_ours(args, w, rank, world, dist):
     }
     if cpu is not None:
         line["cpu_baseline"] = cpu
+    if bwd is not None:
+        bt_tf = bwd["flops"] / (bwd["ms"] * 1e-3) / 1e12
+        line["config"]["bwd"] = {"ms": bwd["ms"], "tflops": bt_tf, "pct_bf16_peak": 100.0 * bt_tf / peak_tf,
+                                 "flops": "2.5 x the forward's effective FLOPs (the five products of the "
+                                          "definition per kept tile pair)",
+                                 "launches_per_call": 3 + (4 if w.block == 64 else 2) + 2}
     print(json.dumps(line), flush=True)
 
 
@@ -519,6 +555,7 @@ def main(argv=None):
     ap.add_argument("--workload", default="wan480p")
     ap.add_argument("--density", type=float, default=None, help="density-sweep workload: kept fraction")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--no-bwd", dest="bwd", action="store_false", help="skip the backward-pass timing")
     ap.add_argument("--baseline-kernel", action="store_true",
                     help="time the legacy mma.sync attention kernel instead of the tcgen05 one")
     ap.add_argument("--cpu-budget", type=float, default=15.0)

@@ -123,6 +123,19 @@ def _task(args):
             if hi < (I + 1) * block:           # padded rows of the last block must be 0
                 pad_nonzero += int(np.count_nonzero(np.asarray(ogpu[b, h, hi:(I + 1) * block])))
         return mx, sm, n, lmx, pad_nonzero
+    if kind == "bwd_check":                    # ("bwd_check", b, h)
+        b, h = args[1], args[2]
+        keep = np.asarray(_mm("keep")[b, h], dtype=bool)[None, None]
+        dO = _bf16_bits_to_f64(np.asarray(_mm("dogpu")[b, h]))[None, None]
+        grads = oracle.masked_attention_backward(_head(0, b, h), _head(1, b, h), _head(2, b, h), keep, dO, N, block)
+        out = []
+        for i, name in enumerate(("dqgpu", "dkgpu", "dvgpu")):
+            got = _bf16_bits_to_f64(np.asarray(_mm(name)[b, h]))
+            want = grads[i][0, 0]
+            err = np.abs(got[:N] - want[:N])
+            out.append((float(err.max()), float(err.sum()), err.size, float(np.abs(want[:N]).max()),
+                        float(np.abs(want[:N]).sum()), int(np.count_nonzero(got[N:]))))
+        return out
     if kind == "inverse":                      # ("inverse", slot)
         slot = args[1]
         x = oracle.inverse_reorder(np.asarray(_mm("o64")[slot])[None, None], T, H, W, P)
@@ -154,6 +167,10 @@ class OraclePool:
             "o64": ("float64", (max(1, slots), w.Npad, w.d)),
             "ogpu": ("uint16", (w.B, w.heads, w.Npad, w.d)),
             "lsegpu": ("float32", (w.B, w.heads, w.Npad)),
+            "dogpu": ("uint16", (w.B, w.heads, w.Npad, w.d)),
+            "dqgpu": ("uint16", (w.B, w.heads, w.Npad, w.d)),
+            "dkgpu": ("uint16", (w.B, w.heads, w.Npad, w.d)),
+            "dvgpu": ("uint16", (w.B, w.heads, w.Npad, w.d)),
         }
         self.meta = {"dir": self.dir, "files": files, "T": w.T, "H": w.H, "W": w.W, "P": w.patch,
                      "block": w.block, "N": w.N, "Npad": w.Npad, "nb": w.nb, "thr": w.thr,
@@ -233,6 +250,26 @@ class OraclePool:
     def inverse(self, slot: int = 0) -> float:
         _, t = self._map([("inverse", slot)])
         return t
+
+    def check_backward(self, dO, dq, dk, dv, pairs: Iterable[Tuple[int, int]]):
+        """Element-by-element comparison of GPU gradients with the oracle's
+        (oracle.masked_attention_backward, one task per (b, head), under the
+        mask set by ``masks`` or ``set_keep``).  All tensors bf16 CPU
+        [B, heads, Npad, d].  Returns, per gradient name, (max-abs error,
+        mean-abs error, max |ref|, mean |ref|, nonzero padded elements)."""
+        import torch
+        for name, t in (("dogpu", dO), ("dqgpu", dq), ("dkgpu", dk), ("dvgpu", dv)):
+            mm = _open(self.meta, name)
+            mm[:] = t.contiguous().view(torch.int16).numpy().view(np.uint16)
+            mm.flush()
+        res, _ = self._map([("bwd_check", b, h) for (b, h) in pairs])
+        out = {}
+        for i, name in enumerate(("dq", "dk", "dv")):
+            rows = [r[i] for r in res]
+            n = sum(r[2] for r in rows)
+            out[name] = (max(r[0] for r in rows), sum(r[1] for r in rows) / max(1, n),
+                         max(r[3] for r in rows), sum(r[4] for r in rows) / max(1, n), sum(r[5] for r in rows))
+        return out
 
     def check_attention(self, o_gpu, lse_gpu, items: Iterable[Tuple[int, int, Sequence[int]]], chunk: int = 16):
         """Element-by-element comparison of the GPU output with the oracle's.

@@ -133,3 +133,33 @@ def test_density_sweep(bsa):
             pool.set_keep(keep)
             print(f"density {dens}:")
             _check_attention(pool, plan, _sampled_items(w, per_head=2, seed=100 + i, run=48))
+
+
+def test_full_size_backward_wan480p(bsa):
+    """The backward pass at the Wan-480p size: every element of dQ, dK and dV
+    of every head against the oracle's gradients (oracle mask of the GPU's
+    forward lists), within the bounds of tests/test_gpu_backward.py."""
+    from test_gpu_backward import MAX_REL, MEAN_REL
+    w = synth.WORKLOADS["wan480p"]
+    q, k, v = synth.make_qkv(w)
+    plan = _plan(bsa, w)
+    plan(q.cuda(), k.cuda(), v.cuda(), w.thr, w.sta)
+    g = torch.Generator().manual_seed(17)
+    dO = torch.randn(plan.o.shape, generator=g).to(torch.bfloat16)
+    dO[:, :, w.N:] = 0
+    dOd = dO.cuda()
+    dq, dk, dv = (torch.full_like(plan.q, float("nan")) for _ in range(3))
+    ws = torch.zeros((bsa.attn_bwd_workspace_bytes(plan.shape) + 15) // 16 * 16, dtype=torch.uint8, device="cuda")
+    bsa.attn_bwd(plan.shape, plan.q, plan.k, plan.v, plan.o, dOd, plan.lse, plan.kv_count, plan.kv_idx, 0.0,
+                 dq, dk, dv, ws)
+    torch.cuda.synchronize()
+    assert bsa.check_device_status(ws) == 0 and plan.status() == 0
+    keep = lists_to_keep(plan.kv_count, plan.kv_idx, plan.nb)
+    with OraclePool(w, q, k, v) as pool:
+        pool.reorder(pool.pairs())
+        pool.set_keep(keep)
+        rep = pool.check_backward(dO, dq.cpu(), dk.cpu(), dv.cpu(), pool.pairs())
+    for name, (mx, mean, refmax, refmean, pad) in rep.items():
+        print(f"  {name}: max-abs {mx:.3e} (ref max {refmax:.3e}), mean-abs {mean:.3e} (ref mean {refmean:.3e})")
+        assert pad == 0, name
+        assert mx <= MAX_REL * refmax and mean <= MEAN_REL * refmean, name

@@ -46,3 +46,15 @@ def test_pool_equals_the_serial_oracle():
         assert pool.check_attention(o_pad, lse32, items)[4] == 1
         # the attention and inverse stages run and time themselves
         assert pool.attention(0, 1, range(w.nb)) > 0 and pool.inverse() > 0
+        # backward: the serial oracle's gradients, rounded to bf16, pass; a planted error is found
+        f64 = lambda t: t.to(torch.float64).numpy()
+        yq, yk, yv = (oracle.reorder(f64(x), w.T, w.H, w.W, w.patch, w.block) for x in (q, k, v))
+        dO = torch.randn(o_bf.shape, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
+        dO[:, :, w.N:] = 0
+        grads = oracle.masked_attention_backward(yq, yk, yv, keep_s, f64(dO), w.N, w.block)
+        gb = [torch.from_numpy(g).to(torch.bfloat16) for g in grads]
+        rep = pool.check_backward(dO, *gb, pool.pairs())
+        for name, (mx_, mean_, refmax, refmean, pad_) in rep.items():
+            assert mx_ <= 2.0 ** -8 * refmax and pad_ == 0, name
+        gb[1][1, 0, 5, 3] += 1.0
+        assert pool.check_backward(dO, *gb, pool.pairs())["dk"][0] > 0.9
