@@ -60,6 +60,14 @@ def _load() -> ctypes.CDLL:
                                              P, P, P, P, ctypes.c_size_t, P]),
         "bsa_attn_fwd": (st, [S, P, P, P, P, P, ctypes.c_float, P, P, P, ctypes.c_size_t, P]),
         "bsa_attn_fwd_baseline": (st, [S, P, P, P, P, P, ctypes.c_float, P, P, P, ctypes.c_size_t, P]),
+        "bsa_hilbert_workspace_bytes": (ctypes.c_size_t, [S]),
+        "bsa_hilbert_order": (st, [S, P, P, ctypes.c_size_t, P]),
+        "bsa_reorder_perm": (st, [S, P, P, P, P]),
+        "bsa_inverse_reorder_perm": (st, [S, P, P, P, P]),
+        "bsa_reorder_qk_pooled_perm": (st, [S, P, P, P, P, P, P, ctypes.c_size_t, P]),
+        "bsa_subblock_workspace_bytes": (ctypes.c_size_t, [S, ctypes.c_int32]),
+        "bsa_build_block_mask_subblock": (st, [S, P, P, ctypes.c_int32, ctypes.c_float, P, P, P, P, ctypes.c_size_t,
+                                               P]),
         "bsa_attn_bwd_workspace_bytes": (ctypes.c_size_t, [S]),
         "bsa_attn_bwd": (st, [S, P, P, P, P, P, P, P, P, ctypes.c_float, P, P, P, P, ctypes.c_size_t, P]),
         "bsa_check_device_status": (st, [P, P]),
@@ -187,6 +195,45 @@ def attn_fwd_baseline(s: Shape, q: torch.Tensor, k: torch.Tensor, v: torch.Tenso
                                      float(scale), _ptr(o), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(),
                                      _stream(q.device)),
            "bsa_attn_fwd_baseline")
+
+
+def hilbert_workspace_bytes(s: Shape) -> int:
+    return get_lib().bsa_hilbert_workspace_bytes(ctypes.byref(s))
+
+
+def hilbert_order(s: Shape, order: torch.Tensor, ws: torch.Tensor) -> None:
+    _check(get_lib().bsa_hilbert_order(ctypes.byref(s), _ptr(order), _ptr(ws), ws.numel() * ws.element_size(),
+                                       _stream(order.device)), "bsa_hilbert_order")
+
+
+def reorder_perm(s: Shape, order: torch.Tensor, x_bnhd: torch.Tensor, y_bhnd: torch.Tensor) -> None:
+    _check(get_lib().bsa_reorder_perm(ctypes.byref(s), _ptr(order), _ptr(x_bnhd), _ptr(y_bhnd),
+                                      _stream(x_bnhd.device)), "bsa_reorder_perm")
+
+
+def inverse_reorder_perm(s: Shape, order: torch.Tensor, y_bhnd: torch.Tensor, x_bnhd: torch.Tensor) -> None:
+    _check(get_lib().bsa_inverse_reorder_perm(ctypes.byref(s), _ptr(order), _ptr(y_bhnd), _ptr(x_bnhd),
+                                              _stream(y_bhnd.device)), "bsa_inverse_reorder_perm")
+
+
+def reorder_qk_pooled_perm(s: Shape, order: torch.Tensor, q_bnhd: torch.Tensor, k_bnhd: torch.Tensor,
+                           q_bhnd: torch.Tensor, k_bhnd: torch.Tensor, ws: torch.Tensor) -> None:
+    _check(get_lib().bsa_reorder_qk_pooled_perm(ctypes.byref(s), _ptr(order), _ptr(q_bnhd), _ptr(k_bnhd),
+                                                _ptr(q_bhnd), _ptr(k_bhnd), _ptr(ws), ws.numel() * ws.element_size(),
+                                                _stream(q_bnhd.device)), "bsa_reorder_qk_pooled_perm")
+
+
+def subblock_workspace_bytes(s: Shape, sub: int) -> int:
+    return get_lib().bsa_subblock_workspace_bytes(ctypes.byref(s), int(sub))
+
+
+def build_block_mask_subblock(s: Shape, q_bhnd: torch.Tensor, k_bhnd: torch.Tensor, sub: int, thr: float,
+                              kv_count: torch.Tensor, kv_idx: torch.Tensor, mask: Optional[torch.Tensor],
+                              ws: torch.Tensor) -> None:
+    _check(get_lib().bsa_build_block_mask_subblock(ctypes.byref(s), _ptr(q_bhnd), _ptr(k_bhnd), int(sub), float(thr),
+                                                   _ptr(kv_count), _ptr(kv_idx), _ptr(mask), _ptr(ws),
+                                                   ws.numel() * ws.element_size(), _stream(q_bhnd.device)),
+           "bsa_build_block_mask_subblock")
 
 
 def attn_bwd_workspace_bytes(s: Shape) -> int:

@@ -78,6 +78,14 @@ size_t workspace_bytes(const Dims& g) { return plan_offset(g) + align256(bsa::pl
 
 bsa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_CUDA; }
 
+// Hilbert order: cubes up to side 2^9 (bitmap of 2^27 bits, 16 MiB).
+constexpr int kMaxHilbertBits = 9;
+
+// Sub-block size: 16 or 32 tokens, dividing the block, or the block itself.
+bool subblock_ok(const Dims& g, int sub) {
+  return (sub == 16 || sub == 32 || sub == g.bs) && sub <= g.bs && g.bs % sub == 0;
+}
+
 }  // namespace
 
 extern "C" {
@@ -319,6 +327,89 @@ bsa_status bsa_attn_bwd(const bsa_shape* s, const void* q, const void* k, const 
   if (bsa::launch_plan(g, kv_count, kv_idx, items_q, cs) != cudaSuccess) return BSA_ERR_CUDA;
   if (bsa::launch_plan(g, a.q_count, a.q_idx, items_kv, cs) != cudaSuccess) return BSA_ERR_CUDA;
   return from_cuda(bsa::launch_attn_bwd(g, a, cs));
+}
+
+size_t bsa_hilbert_workspace_bytes(const bsa_shape* s) {
+  Dims g;
+  if (check_shape(s, &g) != BSA_OK || bsa::hilbert_bits(g) > kMaxHilbertBits) return 0;
+  return bsa::hilbert_layout(g).total;
+}
+
+bsa_status bsa_hilbert_order(const bsa_shape* s, int32_t* order, void* workspace, size_t ws_bytes,
+                             bsa_stream_t stream) {
+  Dims g;
+  bsa_status st = check_shape(s, &g);
+  if (st != BSA_OK) return st;
+  if (bsa::hilbert_bits(g) > kMaxHilbertBits) return BSA_ERR_UNSUPPORTED;
+  if (order == nullptr || workspace == nullptr || !aligned16(order) || !aligned16(workspace))
+    return BSA_ERR_INVALID_ARG;
+  if (ws_bytes < bsa::hilbert_layout(g).total) return BSA_ERR_INVALID_ARG;
+  return from_cuda(bsa::launch_hilbert_order(g, order, workspace, (cudaStream_t)stream));
+}
+
+bsa_status bsa_reorder_perm(const bsa_shape* s, const int32_t* order, const void* x_bnhd, void* y_bhnd,
+                            bsa_stream_t stream) {
+  Dims g;
+  bsa_status st = check_shape(s, &g);
+  if (st != BSA_OK) return st;
+  if (order == nullptr || x_bnhd == nullptr || y_bhnd == nullptr || !aligned16(x_bnhd) || !aligned16(y_bhnd) ||
+      x_bnhd == y_bhnd)
+    return BSA_ERR_INVALID_ARG;
+  return from_cuda(bsa::launch_reorder_perm(g, order, x_bnhd, y_bhnd, (cudaStream_t)stream));
+}
+
+bsa_status bsa_inverse_reorder_perm(const bsa_shape* s, const int32_t* order, const void* y_bhnd, void* x_bnhd,
+                                    bsa_stream_t stream) {
+  Dims g;
+  bsa_status st = check_shape(s, &g);
+  if (st != BSA_OK) return st;
+  if (order == nullptr || x_bnhd == nullptr || y_bhnd == nullptr || !aligned16(x_bnhd) || !aligned16(y_bhnd) ||
+      x_bnhd == y_bhnd)
+    return BSA_ERR_INVALID_ARG;
+  return from_cuda(bsa::launch_inverse_reorder_perm(g, order, y_bhnd, x_bnhd, (cudaStream_t)stream));
+}
+
+bsa_status bsa_reorder_qk_pooled_perm(const bsa_shape* s, const int32_t* order, const void* q_bnhd,
+                                      const void* k_bnhd, void* q_bhnd, void* k_bhnd, void* workspace,
+                                      size_t ws_bytes, bsa_stream_t stream) {
+  Dims g;
+  bsa_status st = check_shape(s, &g);
+  if (st != BSA_OK) return st;
+  if (order == nullptr) return BSA_ERR_INVALID_ARG;
+  const void* ptrs[5] = {q_bnhd, k_bnhd, q_bhnd, k_bhnd, workspace};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return BSA_ERR_INVALID_ARG;
+  if (q_bnhd == q_bhnd || k_bnhd == k_bhnd || q_bhnd == k_bhnd) return BSA_ERR_INVALID_ARG;
+  if (ws_bytes < workspace_bytes(g)) return BSA_ERR_INVALID_ARG;
+  double* qbar = (double*)((char*)workspace + sizeof(Ctrl));
+  double* kbar = qbar + pooled_bytes(g) / sizeof(double);
+  return from_cuda(bsa::launch_reorder_qk_pool_perm(g, order, q_bnhd, k_bnhd, q_bhnd, k_bhnd, qbar, kbar,
+                                                    (cudaStream_t)stream));
+}
+
+size_t bsa_subblock_workspace_bytes(const bsa_shape* s, int32_t sub) {
+  Dims g;
+  if (check_shape(s, &g) != BSA_OK || !subblock_ok(g, sub)) return 0;
+  return bsa::subblock_layout(g, sub).total;
+}
+
+bsa_status bsa_build_block_mask_subblock(const bsa_shape* s, const void* q_bhnd, const void* k_bhnd, int32_t sub,
+                                         float thr, int32_t* kv_count, int32_t* kv_idx, uint8_t* mask_or_null,
+                                         void* workspace, size_t ws_bytes, bsa_stream_t stream) {
+  Dims g;
+  bsa_status st = check_shape(s, &g);
+  if (st != BSA_OK) return st;
+  if (g.nb > BSA_MAX_BLOCKS) return BSA_ERR_UNSUPPORTED;
+  if (!subblock_ok(g, sub)) return BSA_ERR_INVALID_ARG;
+  if (!(thr >= 0.0f && thr < 1.0f)) return BSA_ERR_INVALID_ARG;
+  if (q_bhnd == nullptr || k_bhnd == nullptr || kv_count == nullptr || kv_idx == nullptr || workspace == nullptr)
+    return BSA_ERR_INVALID_ARG;
+  if (!aligned16(q_bhnd) || !aligned16(k_bhnd) || !aligned16(kv_count) || !aligned16(kv_idx) ||
+      !aligned16(workspace))
+    return BSA_ERR_INVALID_ARG;
+  if (ws_bytes < bsa::subblock_layout(g, sub).total) return BSA_ERR_INVALID_ARG;
+  return from_cuda(bsa::launch_mask_subblock(g, sub, q_bhnd, k_bhnd, (double)thr, kv_count, kv_idx, mask_or_null,
+                                             workspace, bsa::next_launch_seq(), (cudaStream_t)stream));
 }
 
 bsa_status bsa_check_device_status(void* workspace, bsa_stream_t stream) {

@@ -60,6 +60,39 @@ cudaError_t launch_attn_tc2(const Dims& g, const void* q, const void* k, const v
                             const int32_t* kv_idx, const int2* items, int* work, float scale, void* o, float* lse,
                             Ctrl* ctrl, uint32_t seq, cudaStream_t st);
 
+// Hilbert-curve token order (order.cu): order[p] = the token at position p.
+// Scratch: the tokens' curve indices, a bitmap over the enclosing cube and
+// the prefix counts of its 64-word blocks.
+struct HilbertLayout {
+  int bits;                        // bits per axis of the cube
+  size_t words, blocks;            // bitmap words, 64-word blocks
+  size_t keys, bitmap, block_sums, total;   // byte offsets in the scratch, total bytes
+};
+int hilbert_bits(const Dims& g);
+HilbertLayout hilbert_layout(const Dims& g);
+cudaError_t launch_hilbert_order(const Dims& g, int32_t* order, void* scratch, cudaStream_t st);
+
+// Reorders with an explicit position -> token table instead of the fractal order.
+cudaError_t launch_reorder_perm(const Dims& g, const int32_t* order, const void* x_bnhd, void* y_bhnd,
+                                cudaStream_t st);
+cudaError_t launch_inverse_reorder_perm(const Dims& g, const int32_t* order, const void* y_bhnd, void* x_bnhd,
+                                        cudaStream_t st);
+cudaError_t launch_reorder_qk_pool_perm(const Dims& g, const int32_t* order, const void* q_bnhd,
+                                        const void* k_bnhd, void* q_bhnd, void* k_bhnd, double* qbar, double* kbar,
+                                        cudaStream_t st);
+
+// Sub-block scoring (mask.cu): block importance from the reduced attention
+// of `sub`-token sub-blocks, then the CDF selection.  Workspace: control
+// block | sub-block means of Q and K | sub-block scores | block importance.
+struct SubblockLayout {
+  int ns;                                  // sub-blocks holding a valid token
+  size_t qbar, kbar, scores, M, total;     // byte offsets, total bytes
+};
+SubblockLayout subblock_layout(const Dims& g, int sub);
+cudaError_t launch_mask_subblock(const Dims& g, int sub, const void* q, const void* k, double thr,
+                                 int32_t* kv_count, int32_t* kv_idx, uint8_t* mask, void* workspace, uint32_t seq,
+                                 cudaStream_t st);
+
 // Backward pass (attn_bwd.cu).  Every pointer is device memory; the planner
 // regions (items_q / items_kv with their work counters) are filled by
 // launch_plan from the forward lists and from the transposed lists.

@@ -299,7 +299,7 @@ __device__ __forceinline__ void block_tile(int I, const Dims& g, int& t, int& th
 // shared memory, turned into probabilities in place (fp64 softmax), and the
 // CDF threshold picks the kept blocks (radix select below); the optional STA
 // union is added and the ascending KV list written.  Lane L owns J = L + 32 i.
-template <int NJ>
+template <int NJ, bool kProbs>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __restrict__ scores, Dims g, double thr,
                                                              int sta_t, int sta_h, int sta_w,
                                                              int32_t* __restrict__ kv_count,
@@ -319,7 +319,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __res
   for (size_t row = (size_t)blockIdx.x * kSelWarps + wid; row < total_rows; row += (size_t)gridDim.x * kSelWarps) {
     const int I = (int)(row % nb);
     const double* src = scores + row * nb;
-    // the row into shared memory, its largest and smallest score on the way
+    // the row into shared memory, its largest and smallest value on the way
+    // (scores, or with kProbs the probabilities themselves)
     double mx = -DBL_MAX, mn = DBL_MAX;
 #pragma unroll
     for (int i = 0; i < NJ; ++i) {
@@ -336,28 +337,34 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __res
       mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       mn = fmin(mn, __shfl_xor_sync(0xffffffffu, mn, o));
     }
-    double z = 0.0;
+    unsigned long long kmax, kmin;
+    if (kProbs) {
+      kmax = (unsigned long long)__double_as_longlong(mx);
+      kmin = (unsigned long long)__double_as_longlong(mn);
+    } else {
+      double z = 0.0;
 #pragma unroll
-    for (int i = 0; i < NJ; ++i) {
-      const int J = lane + 32 * i;
-      if (J < nb) {
-        const double e = exp(srow[J] - mx);
-        srow[J] = e;
-        z += e;
+      for (int i = 0; i < NJ; ++i) {
+        const int J = lane + 32 * i;
+        if (J < nb) {
+          const double e = exp(srow[J] - mx);
+          srow[J] = e;
+          z += e;
+        }
       }
-    }
-    z = warp_sum(z);
-    const double rz = 1.0 / z;
+      z = warp_sum(z);
+      const double rz = 1.0 / z;
 #pragma unroll
-    for (int i = 0; i < NJ; ++i) {
-      const int J = lane + 32 * i;
-      if (J < nb) srow[J] *= rz;        // A = e / sum(e)
+      for (int i = 0; i < NJ; ++i) {
+        const int J = lane + 32 * i;
+        if (J < nb) srow[J] *= rz;        // A = e / sum(e)
+      }
+      // The largest and smallest probabilities, by the same arithmetic as the
+      // row's own entries (exp(0) = 1 exactly): their bit patterns bound the
+      // keys of the radix select.
+      kmax = (unsigned long long)__double_as_longlong(1.0 * rz);
+      kmin = (unsigned long long)__double_as_longlong(exp(mn - mx) * rz);
     }
-    // The largest and smallest probabilities, by the same arithmetic as the
-    // row's own entries (exp(0) = 1 exactly): their bit patterns bound the
-    // keys of the radix select.
-    const unsigned long long kmax = (unsigned long long)__double_as_longlong(1.0 * rz);
-    const unsigned long long kmin = (unsigned long long)__double_as_longlong(exp(mn - mx) * rz);
     auto key_of = [&](int J) { return (unsigned long long)__double_as_longlong(srow[J]); };
 
     // keep bits: bit i of `keep` <-> J = lane + 32 i
@@ -534,6 +541,56 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const double* __res
   }
 }
 
+// ----------------------------------------------------- sub-block scoring
+
+// subblock_reduce_kernel: block importance from sub-block scores (DFSAttn
+// explainer, section 2).  One warp per (b, head, query block I): for each of
+// I's valid query sub-blocks a, the softmax over all valid key sub-blocks b of
+// the scores S[a][b] (fp64), and the mass that falls on each key block J
+// (the sum over J's sub-blocks); the masses are averaged over I's valid query
+// sub-blocks.  M[bh][I][J] is written as a row of probabilities (it sums to 1)
+// for the selection kernel.  `gs` describes the sub-block grid (nb = the
+// number of valid sub-blocks), `g` the block grid; per = block / sub
+// consecutive sub-blocks make a block.
+template <int PER>
+__global__ void __launch_bounds__(256) subblock_reduce_kernel(const double* __restrict__ S, Dims g, int ns,
+                                                              double* __restrict__ M) {
+  extern __shared__ __align__(16) double macc[];     // [8 warps][nb]
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int nb = g.nb;
+  const size_t unit = (size_t)blockIdx.x * 8 + wid;  // bh * nb + I
+  if (unit >= (size_t)g.B * g.heads * nb) return;
+  const size_t bh = unit / nb;
+  const int I = (int)(unit % nb);
+  double* acc = macc + wid * nb;
+  for (int J = lane; J < nb; J += 32) acc[J] = 0.0;
+  __syncwarp();
+  const int a0 = I * PER, a1 = min(a0 + PER, ns);
+  for (int a = a0; a < a1; ++a) {
+    const double* row = S + (bh * ns + a) * (size_t)ns;
+    double mx = -DBL_MAX;
+    for (int b = lane; b < ns; b += 32) mx = fmax(mx, row[b]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    double z = 0.0;
+    for (int b = lane; b < ns; b += 32) z += exp(row[b] - mx);
+    z = warp_sum(z);
+    const double rz = 1.0 / z;
+    // per key block: the PER consecutive sub-blocks of a block sit in PER
+    // consecutive lanes of one 32-wide slice (PER divides 32)
+    for (int b0 = 0; b0 < ns; b0 += 32) {
+      const int b = b0 + lane;
+      double p = (b < ns) ? exp(row[b] - mx) * rz : 0.0;
+#pragma unroll
+      for (int o = PER / 2; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
+      if ((lane % PER) == 0 && b < ns) acc[b / PER] += p;
+    }
+    __syncwarp();
+  }
+  const double inv = 1.0 / (double)(a1 - a0);
+  for (int J = lane; J < nb; J += 32) M[unit * nb + J] = acc[J] * inv;
+}
+
 }  // namespace
 
 template <int D, int BS>
@@ -557,6 +614,10 @@ cudaError_t launch_pool_t(const Dims& g, const void* q, const void* k, double* q
 
 cudaError_t launch_pool(const Dims& g, const void* q, const void* k, double* qbar, double* kbar, Ctrl* ctrl,
                         uint32_t seq, cudaStream_t st) {
+  if (g.d == 128 && g.bs == 16) return launch_pool_t<128, 16>(g, q, k, qbar, kbar, ctrl, seq, st);
+  if (g.d == 128 && g.bs == 32) return launch_pool_t<128, 32>(g, q, k, qbar, kbar, ctrl, seq, st);
+  if (g.d == 64 && g.bs == 16) return launch_pool_t<64, 16>(g, q, k, qbar, kbar, ctrl, seq, st);
+  if (g.d == 64 && g.bs == 32) return launch_pool_t<64, 32>(g, q, k, qbar, kbar, ctrl, seq, st);
   if (g.d == 128 && g.bs == 64) return launch_pool_t<128, 64>(g, q, k, qbar, kbar, ctrl, seq, st);
   if (g.d == 128 && g.bs == 128) return launch_pool_t<128, 128>(g, q, k, qbar, kbar, ctrl, seq, st);
   if (g.d == 64 && g.bs == 64) return launch_pool_t<64, 64>(g, q, k, qbar, kbar, ctrl, seq, st);
@@ -565,23 +626,33 @@ cudaError_t launch_pool(const Dims& g, const void* q, const void* k, double* qba
 
 size_t mask_scores_bytes(const Dims& g) { return (size_t)g.B * g.heads * g.nb * g.nb * sizeof(double); }
 
-template <int NJ>
+template <int NJ, bool kProbs>
 cudaError_t launch_select_t(const Dims& g, const double* scores, double thr, int sta_t, int sta_h, int sta_w,
                             int32_t* kv_count, int32_t* kv_idx, uint8_t* mask, cudaStream_t st) {
   const size_t smem = (size_t)kSelWarps * (NJ * 32 * sizeof(double) + kHistSlots * sizeof(uint64_t));
-  cudaError_t e = cudaFuncSetAttribute(select_kernel<NJ>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(select_kernel<NJ, kProbs>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0, per_sm = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_kernel<NJ>, kSelThreads, smem)) !=
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_kernel<NJ, kProbs>, kSelThreads, smem)) !=
       cudaSuccess)
     return e;
   const size_t rows = (size_t)g.B * g.heads * g.nb;
   const size_t need = (rows + kSelWarps - 1) / kSelWarps;
   const int grid = (int)std::max<size_t>(1, std::min<size_t>(need, (size_t)sms * std::max(1, per_sm)));
-  select_kernel<NJ><<<grid, kSelThreads, smem, st>>>(scores, g, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask);
+  select_kernel<NJ, kProbs><<<grid, kSelThreads, smem, st>>>(scores, g, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask);
   return cudaGetLastError();
+}
+
+template <bool kProbs>
+cudaError_t launch_select(const Dims& g, const double* scores, double thr, int sta_t, int sta_h, int sta_w,
+                          int32_t* kv_count, int32_t* kv_idx, uint8_t* mask, cudaStream_t st) {
+  if (g.nb <= 128) return launch_select_t<4, kProbs>(g, scores, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask, st);
+  if (g.nb <= 256) return launch_select_t<8, kProbs>(g, scores, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask, st);
+  if (g.nb <= 512)
+    return launch_select_t<16, kProbs>(g, scores, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask, st);
+  return launch_select_t<32, kProbs>(g, scores, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask, st);
 }
 
 template <int D>
@@ -602,10 +673,57 @@ cudaError_t launch_mask(const Dims& g, const double* qbar, const double* kbar, d
   cudaError_t e = (g.d == 128) ? launch_scores_t<128>(g, qbar, kbar, scores, st)
                                : launch_scores_t<64>(g, qbar, kbar, scores, st);
   if (e != cudaSuccess) return e;
-  if (g.nb <= 128) return launch_select_t<4>(g, scores, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask, st);
-  if (g.nb <= 256) return launch_select_t<8>(g, scores, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask, st);
-  if (g.nb <= 512) return launch_select_t<16>(g, scores, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask, st);
-  return launch_select_t<32>(g, scores, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask, st);
+  return launch_select<false>(g, scores, thr, sta_t, sta_h, sta_w, kv_count, kv_idx, mask, st);
+}
+
+SubblockLayout subblock_layout(const Dims& g, int sub) {
+  auto a256 = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  SubblockLayout L;
+  L.ns = (g.N + sub - 1) / sub;
+  const size_t bh = (size_t)g.B * g.heads;
+  L.qbar = sizeof(Ctrl);
+  L.kbar = L.qbar + a256(bh * L.ns * g.d * sizeof(double));
+  L.scores = L.kbar + a256(bh * L.ns * g.d * sizeof(double));
+  L.M = L.scores + a256(bh * L.ns * (size_t)L.ns * sizeof(double));
+  L.total = L.M + a256(bh * g.nb * (size_t)g.nb * sizeof(double));
+  return L;
+}
+
+cudaError_t launch_mask_subblock(const Dims& g, int sub, const void* q, const void* k, double thr,
+                                 int32_t* kv_count, int32_t* kv_idx, uint8_t* mask, void* workspace, uint32_t seq,
+                                 cudaStream_t st) {
+  const SubblockLayout L = subblock_layout(g, sub);
+  char* ws = (char*)workspace;
+  double* qbar = (double*)(ws + L.qbar);
+  double* kbar = (double*)(ws + L.kbar);
+  double* S = (double*)(ws + L.scores);
+  double* M = (double*)(ws + L.M);
+  // the sub-block grid: `sub` tokens per block, only the sub-blocks holding a valid token
+  Dims gs = g;
+  gs.bs = sub;
+  gs.nb = L.ns;
+  cudaError_t e = launch_pool(gs, q, k, qbar, kbar, (Ctrl*)workspace, seq, st);
+  if (e != cudaSuccess) return e;
+  e = (g.d == 128) ? launch_scores_t<128>(gs, qbar, kbar, S, st) : launch_scores_t<64>(gs, qbar, kbar, S, st);
+  if (e != cudaSuccess) return e;
+  const size_t units = (size_t)g.B * g.heads * g.nb;
+  const size_t smem = 8 * (size_t)g.nb * sizeof(double);
+  const unsigned grid = (unsigned)((units + 7) / 8);
+  auto run = [&](auto kernel) -> cudaError_t {
+    cudaError_t r = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (r != cudaSuccess) return r;
+    kernel<<<grid, 256, smem, st>>>(S, g, L.ns, M);
+    return cudaGetLastError();
+  };
+  switch (g.bs / sub) {
+    case 1: e = run(subblock_reduce_kernel<1>); break;
+    case 2: e = run(subblock_reduce_kernel<2>); break;
+    case 4: e = run(subblock_reduce_kernel<4>); break;
+    case 8: e = run(subblock_reduce_kernel<8>); break;
+    default: return cudaErrorInvalidValue;
+  }
+  if (e != cudaSuccess) return e;
+  return launch_select<true>(g, M, thr, -1, -1, -1, kv_count, kv_idx, mask, st);
 }
 
 }  // namespace bsa

@@ -14,6 +14,10 @@
 // fastest: the CTAs that run together move the same positions of every head,
 // i.e. the neighbouring rows of the same model-order tokens.
 //
+// Any other order of the tokens (a position -> token table, e.g. the Hilbert
+// curve of order.cu) runs through the same kernels in place of the fractal
+// formula.
+//
 // The pooled variant also sums each column of the block's valid rows in
 // double (exact for bf16 inputs: no rounding unless a block mixes values more
 // than 2^38 apart) and writes the block mean: qbar [bh][I][d] row-major for
@@ -32,6 +36,7 @@ struct Tensors {
   uint4* dst[2];
   double* mean[2];   // block means (pooled variant): [0] row-major, [1] transposed
   int n;             // tensors in this launch (1 or 2)
+  const int32_t* order;   // position -> token table, or null for the fractal order
 };
 
 template <int D, int BS, bool kInverse, bool kPool>
@@ -61,7 +66,7 @@ __global__ void __launch_bounds__(kThreads) reorder_kernel(Tensors a, Dims g) {
   __shared__ int tok[BS];
   if (threadIdx.x < BS) {
     const int p = I * BS + threadIdx.x;
-    tok[threadIdx.x] = (p < g.N) ? fractal_token(p, g.H, g.W, g.P) : -1;
+    tok[threadIdx.x] = (p >= g.N) ? -1 : (a.order != nullptr ? a.order[p] : fractal_token(p, g.H, g.W, g.P));
   }
   __syncthreads();
 
@@ -143,18 +148,35 @@ cudaError_t launch(const Tensors& a, const Dims& g, cudaStream_t st) {
 }  // namespace
 
 cudaError_t launch_reorder(const Dims& g, const void* x_bnhd, void* y_bhnd, cudaStream_t st) {
-  Tensors a = {{(const uint4*)x_bnhd, nullptr}, {(uint4*)y_bhnd, nullptr}, {nullptr, nullptr}, 1};
-  return launch<false, false>(a, g, st);
+  return launch_reorder_perm(g, nullptr, x_bnhd, y_bhnd, st);
 }
 
 cudaError_t launch_inverse_reorder(const Dims& g, const void* y_bhnd, void* x_bnhd, cudaStream_t st) {
-  Tensors a = {{(const uint4*)y_bhnd, nullptr}, {(uint4*)x_bnhd, nullptr}, {nullptr, nullptr}, 1};
-  return launch<true, false>(a, g, st);
+  return launch_inverse_reorder_perm(g, nullptr, y_bhnd, x_bnhd, st);
 }
 
 cudaError_t launch_reorder_qk_pool(const Dims& g, const void* q_bnhd, const void* k_bnhd, void* q_bhnd,
                                    void* k_bhnd, double* qbar, double* kbar, cudaStream_t st) {
-  Tensors a = {{(const uint4*)q_bnhd, (const uint4*)k_bnhd}, {(uint4*)q_bhnd, (uint4*)k_bhnd}, {qbar, kbar}, 2};
+  return launch_reorder_qk_pool_perm(g, nullptr, q_bnhd, k_bnhd, q_bhnd, k_bhnd, qbar, kbar, st);
+}
+
+cudaError_t launch_reorder_perm(const Dims& g, const int32_t* order, const void* x_bnhd, void* y_bhnd,
+                                cudaStream_t st) {
+  Tensors a = {{(const uint4*)x_bnhd, nullptr}, {(uint4*)y_bhnd, nullptr}, {nullptr, nullptr}, 1, order};
+  return launch<false, false>(a, g, st);
+}
+
+cudaError_t launch_inverse_reorder_perm(const Dims& g, const int32_t* order, const void* y_bhnd, void* x_bnhd,
+                                        cudaStream_t st) {
+  Tensors a = {{(const uint4*)y_bhnd, nullptr}, {(uint4*)x_bnhd, nullptr}, {nullptr, nullptr}, 1, order};
+  return launch<true, false>(a, g, st);
+}
+
+cudaError_t launch_reorder_qk_pool_perm(const Dims& g, const int32_t* order, const void* q_bnhd,
+                                        const void* k_bnhd, void* q_bhnd, void* k_bhnd, double* qbar, double* kbar,
+                                        cudaStream_t st) {
+  Tensors a = {{(const uint4*)q_bnhd, (const uint4*)k_bnhd}, {(uint4*)q_bhnd, (uint4*)k_bhnd}, {qbar, kbar}, 2,
+               order};
   return launch<false, true>(a, g, st);
 }
 

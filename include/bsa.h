@@ -179,6 +179,64 @@ BSA_API bsa_status bsa_attn_fwd(const bsa_shape* s, const void* q, const void* k
                         void* o, float* lse_or_null,
                         void* workspace, size_t ws_bytes, bsa_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * Alternative token order and block estimator (DFSAttn explainer,
+ * gist.science/es/paper/2605.23445, sections 1 and 2): a 3-D Hilbert-curve
+ * order of the tokens, and block importance from finer sub-block scores,
+ * feeding the same CDF threshold.
+ * ------------------------------------------------------------------------- */
+
+/* Scratch bytes of bsa_hilbert_order (0 for an invalid shape or a grid whose
+ * largest side exceeds 512). */
+BSA_API size_t bsa_hilbert_workspace_bytes(const bsa_shape* s);
+
+/* The 3-D Hilbert-curve order of the T x H x W tokens, DFSAttn explainer,
+ * section 1 ("El barajado de la Curva de Hilbert"): order[p] = the token
+ * n = t*H*W + h*W + w at position p, for p < N.  The curve is J. Skilling's
+ * construction ("Programming the Hilbert curve", 2004) over the smallest
+ * power-of-two cube holding the grid, axes (t, h, w); grid points keep the
+ * cube's order, points outside the grid are skipped.
+ *   order: device, [N] int32, written.
+ *   workspace / ws_bytes: scratch of at least bsa_hilbert_workspace_bytes(s). */
+BSA_API bsa_status bsa_hilbert_order(const bsa_shape* s, int32_t* order, void* workspace, size_t ws_bytes,
+                                     bsa_stream_t stream);
+
+/* bsa_reorder, bsa_inverse_reorder and bsa_reorder_qk_pooled with the token
+ * order given as a table (e.g. from bsa_hilbert_order) instead of the fractal
+ * order: y[b, h, p, :] = x[b, order[p], h, :] for p < N, zero tail.  `order`
+ * (device, [N] int32) must be a permutation of 0..N-1.  The STA union of the
+ * block-mask calls places blocks by the fractal order and does not apply to
+ * other orders. */
+BSA_API bsa_status bsa_reorder_perm(const bsa_shape* s, const int32_t* order, const void* x_bnhd, void* y_bhnd,
+                                    bsa_stream_t stream);
+BSA_API bsa_status bsa_inverse_reorder_perm(const bsa_shape* s, const int32_t* order, const void* y_bhnd,
+                                            void* x_bnhd, bsa_stream_t stream);
+BSA_API bsa_status bsa_reorder_qk_pooled_perm(const bsa_shape* s, const int32_t* order, const void* q_bnhd,
+                                              const void* k_bnhd, void* q_bhnd, void* k_bhnd, void* workspace,
+                                              size_t ws_bytes, bsa_stream_t stream);
+
+/* Workspace bytes of bsa_build_block_mask_subblock (0 for an invalid shape or
+ * sub-block size): a control block, the sub-block means of Q and K
+ * (2 * B*heads*ns*d doubles, ns = ceil(N / sub)), the sub-block scores
+ * (B*heads*ns*ns doubles) and the block importance (B*heads*nb*nb doubles). */
+BSA_API size_t bsa_subblock_workspace_bytes(const bsa_shape* s, int32_t sub);
+
+/* Block mask from sub-block scores, DFSAttn explainer, section 2 ("La
+ * puntuacion de Sub-bloque"), with NABLA's CDF rule (bsa_build_block_mask):
+ * Q and K are mean-pooled over sub-blocks of `sub` tokens (valid tokens only),
+ * each query sub-block's softmax over all key sub-blocks (scale 1/sqrt(d)) is
+ * summed over each key block's sub-blocks, and block I's importance for block
+ * J is that mass averaged over I's query sub-blocks (rows sum to 1); the CDF
+ * threshold then keeps the shortest most-important prefix of mass >= 1 - thr.
+ * With sub == block this is NABLA's reduced map.  Double precision throughout.
+ *   sub: 16 or 32 (dividing the block size), or the block size.
+ *   Other arguments as for bsa_build_block_mask (no STA union);
+ *   workspace / ws_bytes: at least bsa_subblock_workspace_bytes(s, sub). */
+BSA_API bsa_status bsa_build_block_mask_subblock(const bsa_shape* s, const void* q_bhnd, const void* k_bhnd,
+                                                 int32_t sub, float thr, int32_t* kv_count, int32_t* kv_idx,
+                                                 uint8_t* mask_or_null, void* workspace, size_t ws_bytes,
+                                                 bsa_stream_t stream);
+
 /* Bytes of device workspace bsa_attn_bwd needs for this shape (0 for an
  * invalid shape): a control block (device error word), D = rowsum(dO * O)
  * (B*heads*Npad floats), a bit matrix of the block mask (B*heads*nb*
