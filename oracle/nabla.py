@@ -416,6 +416,93 @@ def block_mask_subblock(q_bhnd: np.ndarray, k_bhnd: np.ndarray, N: int, block: i
     return cdf_keep(subblock_scores(q_bhnd, k_bhnd, N, block, sub, scale), thr)
 
 
+# ------------------------------------------------------ token-radius masks
+
+def attention_entropy(q: np.ndarray, k: np.ndarray, N: int, scale: Optional[float] = None) -> np.ndarray:
+    """Entropy (nats) of each query row of the dense attention: [B, heads, Npad] (0 for padded rows).
+
+    TRA summary, section 2 ("Entropia-a-Presupuesto"): in a dense warm-up pass
+    the entropy of each query's attention distribution is computed,
+    H_i = -sum_j p_ij ln p_ij with p_i = softmax_j(scale q_i . k_j) over the
+    valid keys.
+    """
+    B, heads, Npad, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    H = np.zeros((B, heads, Npad), dtype=np.float64)
+    for b in range(B):
+        for h in range(heads):
+            s = (q[b, h, :N] @ k[b, h, :N].T) * scale
+            s = s - s.max(axis=1, keepdims=True)
+            e = np.exp(s)
+            p = e / e.sum(axis=1, keepdims=True)
+            H[b, h, :N] = -(p * np.log(p, where=p > 0, out=np.zeros_like(p))).sum(axis=1)
+    return H
+
+
+def token_radius(H: np.ndarray, t_of: np.ndarray, T: int, tau: float, gamma: float, N: int) -> np.ndarray:
+    """Base radius of each query token from its entropy: [.., Npad] (0 for padded rows).
+
+    TRA summary, section 2 ("Entropia-a-Presupuesto", "Presupuesto-a-Radio"):
+    the token budget is tau * exp(H_i) keys (clamped to [1, N]); the support
+    of the query in frame t is a 2-D disk of radius r_i * phi(|t - t_i|), with
+    phi(delta) = exp(-gamma * delta), and r_i makes the disks' total area the
+    budget: sum_t pi (r_i phi(|t - t_i|))^2 = budget.  `t_of`: the frame of the
+    token at each position.
+    """
+    out = np.zeros(H.shape, dtype=np.float64)
+    for p in range(N):
+        ti = int(t_of[p])
+        area = sum(math.pi * math.exp(-2.0 * gamma * abs(t - ti)) for t in range(T))
+        budget = np.clip(tau * np.exp(H[..., p]), 1.0, float(N))
+        out[..., p] = np.sqrt(budget / area)
+    return out
+
+
+def radius_block_mask(r: np.ndarray, T: int, H: int, W: int, P: int, block: int, gamma: float,
+                      vote: int = 1) -> np.ndarray:
+    """Block mask from token-radius supports: [B, heads, nb, nb] bool.
+
+    TRA summary, section 2 ("Ejecucion Eficiente"): tokens in the tile-major
+    (here: the fractal P x P) order; key token j is in query token i's support
+    when (h_j - h_i)^2 + (w_j - w_i)^2 <= (r_i phi(|t_j - t_i|))^2; a query
+    token votes for a key block when the block holds a key of its support, and
+    block I keeps block J when at least `vote` of I's valid query tokens vote
+    for J (the token-level masks made into regular block masks).
+    `r`: [B, heads, Npad] base radii by position.
+    """
+    N = T * H * W
+    order = fractal_order(T, H, W, P)
+    nb = num_blocks(N, block)
+    t = order // (H * W)
+    hh = (order % (H * W)) // W
+    ww = order % W
+    lead = r.shape[:-1]
+    keep = np.zeros(lead + (nb, nb), dtype=bool)
+    for idx in np.ndindex(*lead):
+        for I in range(nb):
+            qs = range(I * block, min((I + 1) * block, N))
+            votes = np.zeros(nb, dtype=np.int64)
+            for i in qs:
+                rad = r[idx + (i,)] * np.exp(-gamma * np.abs(t - t[i]))
+                inside = (hh - hh[i]) ** 2 + (ww - ww[i]) ** 2 <= rad ** 2
+                hit = np.zeros(nb, dtype=bool)
+                hit[np.nonzero(inside)[0] // block] = True
+                votes += hit
+            keep[idx + (I,)] = votes >= vote
+    return keep
+
+
+def radius_mask_from_qk(q: np.ndarray, k: np.ndarray, T: int, H: int, W: int, P: int, block: int, tau: float,
+                        gamma: float, vote: int = 1, scale: Optional[float] = None) -> np.ndarray:
+    """The whole chain on reordered Q, K: entropy -> budget -> radius -> block mask."""
+    N = T * H * W
+    Hn = attention_entropy(q, k, N, scale)
+    t_of = fractal_order(T, H, W, P) // (H * W)
+    r = token_radius(Hn, t_of, T, tau, gamma, N)
+    return radius_block_mask(r, T, H, W, P, block, gamma, vote)
+
+
 # ------------------------------------------ block-sparse attention backward
 
 def masked_attention_backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, keep: np.ndarray, dO: np.ndarray,

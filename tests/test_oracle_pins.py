@@ -595,6 +595,96 @@ def test_pins_catch_subblock_scores_that_average_instead_of_summing(monkeypatch)
         test_subblock_scores_closed_forms()
 
 
+# ------------------------------------------------------------ radius masks
+
+def test_attention_entropy_against_library_and_closed_forms():
+    rng = np.random.default_rng(21)
+    N, bs, d = 50, 16, 8
+    Npad = nabla.padded_len(N, bs)
+    q = rng.standard_normal((1, 2, Npad, d)) * 2
+    k = rng.standard_normal((1, 2, Npad, d)) * 2
+    H = oracle.attention_entropy(q, k, N)
+    for h in range(2):
+        logits = torch.from_numpy(q[0, h, :N] @ k[0, h, :N].T / math.sqrt(d))
+        ref = torch.distributions.Categorical(logits=logits).entropy().numpy()
+        assert np.allclose(H[0, h, :N], ref, rtol=1e-12, atol=1e-12)
+    assert np.all(H[:, :, N:] == 0)
+    # identical keys: a uniform distribution over the N valid keys
+    k_eq = np.tile(k[:, :, :1], (1, 1, Npad, 1))
+    assert np.allclose(oracle.attention_entropy(q, k_eq, N)[:, :, :N], math.log(N), atol=1e-12)
+
+
+def test_token_radius_closed_form():
+    T, N = 3, 30
+    t_of = np.repeat(np.arange(T), N // T)
+    H = np.full((1, 1, N), math.log(12.0))
+    r = oracle.token_radius(H, t_of, T, 2.0, 0.5, N)
+    # budget 2 * 12 = 24 tokens; a query in frame 0 has disks of area pi r^2 (1 + e^-1 + e^-2)
+    assert abs(r[0, 0, 0] - math.sqrt(24.0 / (math.pi * (1 + math.exp(-1) + math.exp(-2))))) < 1e-12
+    # frame 1 (middle): 1 + 2 e^-1
+    assert abs(r[0, 0, 10] - math.sqrt(24.0 / (math.pi * (1 + 2 * math.exp(-1))))) < 1e-12
+    # the budget is clamped to [1, N]
+    r = oracle.token_radius(np.full((1, 1, N), 50.0), t_of, 1, 1.0, 0.0, N)
+    assert abs(r[0, 0, 0] - math.sqrt(N / math.pi)) < 1e-12
+
+
+def _radius_mask_brute(r_tok, T, H, W, P, bs, gamma, vote):
+    """Token-level support by explicit loops over original (t, h, w)
+    coordinates, blocks through the inverse of the fractal order."""
+    N = T * H * W
+    pos = np.empty(N, dtype=np.int64)
+    pos[oracle.fractal_order(T, H, W, P)] = np.arange(N)       # token -> position
+    nb = nabla.num_blocks(N, bs)
+    votes = np.zeros((nb, nb), dtype=np.int64)
+    for ti in range(T):
+        for hi in range(H):
+            for wi in range(W):
+                i = ti * H * W + hi * W + wi
+                hit = set()
+                for tj in range(T):
+                    rad = r_tok[i] * math.exp(-gamma * abs(tj - ti))
+                    for hj in range(H):
+                        for wj in range(W):
+                            if (hj - hi) ** 2 + (wj - wi) ** 2 <= rad * rad:
+                                hit.add(pos[tj * H * W + hj * W + wj] // bs)
+                for J in hit:
+                    votes[pos[i] // bs, J] += 1
+    return votes >= vote
+
+
+@pytest.mark.parametrize("gamma,vote", [(0.0, 1), (0.7, 1), (0.7, 3)])
+def test_radius_block_mask_by_brute_force(gamma, vote):
+    rng = np.random.default_rng(22)
+    T, H, W, P, bs = 3, 5, 7, 4, 8
+    N = T * H * W
+    r_tok = rng.uniform(0.0, 2.5, N)                      # radius per token (model order)
+    order = oracle.fractal_order(T, H, W, P)
+    r_pos = np.zeros((1, 1, nabla.padded_len(N, bs)))
+    r_pos[0, 0, :N] = r_tok[order]
+    got = oracle.radius_block_mask(r_pos, T, H, W, P, bs, gamma, vote)[0, 0]
+    assert np.array_equal(got, _radius_mask_brute(r_tok, T, H, W, P, bs, gamma, vote))
+
+
+def test_radius_zero_is_the_same_position_in_every_frame():
+    """r = 0, no decay: a query's support is its own (h, w) in every frame; on
+    an aligned grid (blocks = patches) that is the STA window (T, 0, 0)."""
+    T, H, W, P = 3, 16, 16, 8
+    bs = P * P
+    r = np.zeros((1, 1, T * H * W))
+    keep = oracle.radius_block_mask(r, T, H, W, P, bs, 0.0, 1)[0, 0]
+    assert np.array_equal(keep, oracle.sta_mask(T, H, W, P, bs, (T, 0, 0)))
+
+
+def test_pins_catch_a_radius_mask_without_temporal_decay(monkeypatch):
+    orig = nabla.radius_block_mask
+
+    def bad(r, T, H, W, P, block, gamma, vote=1):
+        return orig(r, T, H, W, P, block, 0.0, vote)
+    monkeypatch.setattr(oracle, "radius_block_mask", bad)
+    with pytest.raises(AssertionError):
+        test_radius_block_mask_by_brute_force(0.7, 1)
+
+
 def test_lists_roundtrip():
     rng = np.random.default_rng(9)
     keep = rng.random((2, 3, 7, 7)) < 0.4
