@@ -60,6 +60,9 @@ def _load() -> ctypes.CDLL:
                                              P, P, P, P, ctypes.c_size_t, P]),
         "bsa_attn_fwd": (st, [S, P, P, P, P, P, ctypes.c_float, P, P, P, ctypes.c_size_t, P]),
         "bsa_attn_fwd_baseline": (st, [S, P, P, P, P, P, ctypes.c_float, P, P, P, ctypes.c_size_t, P]),
+        "bsa_attn_fwd_entropy": (st, [S, P, P, P, P, P, ctypes.c_float, P, P, P, P, ctypes.c_size_t, P]),
+        "bsa_dense_lists": (st, [S, P, P, P]),
+        "bsa_build_block_mask_radius": (st, [S, P, ctypes.c_float, ctypes.c_float, ctypes.c_int32, P, P, P, P]),
         "bsa_hilbert_workspace_bytes": (ctypes.c_size_t, [S]),
         "bsa_hilbert_order": (st, [S, P, P, ctypes.c_size_t, P]),
         "bsa_reorder_perm": (st, [S, P, P, P, P]),
@@ -195,6 +198,27 @@ def attn_fwd_baseline(s: Shape, q: torch.Tensor, k: torch.Tensor, v: torch.Tenso
                                      float(scale), _ptr(o), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(),
                                      _stream(q.device)),
            "bsa_attn_fwd_baseline")
+
+
+def attn_fwd_entropy(s: Shape, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, kv_count: torch.Tensor,
+                     kv_idx: torch.Tensor, scale: float, o: torch.Tensor, lse: torch.Tensor, entropy: torch.Tensor,
+                     ws: torch.Tensor) -> None:
+    _check(get_lib().bsa_attn_fwd_entropy(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(kv_count), _ptr(kv_idx),
+                                          float(scale), _ptr(o), _ptr(lse), _ptr(entropy), _ptr(ws),
+                                          ws.numel() * ws.element_size(), _stream(q.device)),
+           "bsa_attn_fwd_entropy")
+
+
+def dense_lists(s: Shape, kv_count: torch.Tensor, kv_idx: torch.Tensor) -> None:
+    _check(get_lib().bsa_dense_lists(ctypes.byref(s), _ptr(kv_count), _ptr(kv_idx), _stream(kv_count.device)),
+           "bsa_dense_lists")
+
+
+def build_block_mask_radius(s: Shape, entropy: torch.Tensor, tau: float, gamma: float, vote: int,
+                            kv_count: torch.Tensor, kv_idx: torch.Tensor, mask: Optional[torch.Tensor]) -> None:
+    _check(get_lib().bsa_build_block_mask_radius(ctypes.byref(s), _ptr(entropy), float(tau), float(gamma), int(vote),
+                                                 _ptr(kv_count), _ptr(kv_idx), _ptr(mask), _stream(entropy.device)),
+           "bsa_build_block_mask_radius")
 
 
 def hilbert_workspace_bytes(s: Shape) -> int:

@@ -1,6 +1,6 @@
-// Block-sparse attention forward on the sm_100a tensor cores: persistent,
-// one CTA per SM.  NABLA summary, Metodologia 2 "Expansion": only the listed
-// N x N tiles are computed.
+// Block-sparse attention forward on the sm_100a tensor cores, with P in
+// tensor memory: persistent, one CTA per SM.  NABLA summary, Metodologia 2
+// "Expansion": only the listed N x N tiles are computed.
 //
 // Work: the plan's 128-row query tiles (one block of 128, or two blocks of 64,
 // rows 0-63 and 64-127), fetched one at a time from a work counter in the
@@ -13,25 +13,34 @@
 //                  masks keys its row's block does not keep (and padding),
 //                  keeps a running base-2 max (O_w rescaled only when it grows
 //                  by more than 8) and writes P = 2^(s - m) as bf16 into the
-//                  group's P tile in shared memory
-//   O_w += P V     tcgen05.mma with A = P and B = V (MN-major) from shared
-//                  memory, O_w in TMEM
-// TMEM holds S_0, S_1, O_0, O_1 (4 x 128 columns).  Because P does not live in
-// the S buffer, the S of the group's next tile is issued as soon as the group
-// has read its current S, and a softmax waits only for its own S; the P.V
-// products run beside it.  The epilogue merges the two groups' partial results
+//                  first 64 columns of the same TMEM buffer (tcgen05.st)
+//   O_w += P V     tcgen05.mma with A = P from TMEM and B = V (MN-major) from
+//                  shared memory, O_w in TMEM
+// Shared memory then carries only the TMA tiles and the MMA reads of Q, K and
+// V: about 160 KB per KV tile against 1024 cycles of tensor work, where
+// staging P in shared memory as well (written by the softmax, read by the
+// MMA) costs another 64 KB per tile of its 128 bytes per clock.
+//
+// One thread issues every MMA of the CTA, in this order: S(0), S(1), then for
+// each j: O_w += P(j) V(j), S(j + 2) into the same buffer w.  tcgen05.mma
+// operations of one thread execute in issue order, so S(j + 2) overwrites the
+// P(j) columns only after the P.V product has read them; and the commit that
+// reports S(j + 2) complete covers every earlier MMA of the thread, so a
+// softmax that has seen its S knows that its group's previous P.V product is
+// done (O_w can be rescaled, P can be rewritten).  TMEM holds S_0, S_1, O_0,
+// O_1 (4 x 128 columns).  The epilogue merges the two groups' partial results
 // of each row exactly.  K and V have two stages in shared memory, each loaded
 // by its own producer warp.  O is normalised by the sum of the bf16-rounded
 // weights the P.V product uses (an exact convex combination of V rows up to
 // accumulation rounding); the LSE uses the fp32 sum of the unrounded ones.
 //
-// Roles: warps 0 and 2 issue TMA loads (Q and K; V), warp 3 issues the S
-// MMAs and warp 1 the P.V MMAs (one elected thread each), warps 4-11 run the
-// softmax and the epilogue (warp w reads TMEM lanes 32 (w mod 4) .. +31).
-// Every mbarrier wait is bounded; on expiry the CTA records BSA_ERR_TIMEOUT in
-// the workspace error word, tells the launch's other CTAs to give up (its own
-// launch sequence number in the control block), waits (bounded) for the
-// copies and MMAs it has already issued, frees its TMEM and leaves.
+// Roles: warps 0 and 2 issue TMA loads (Q and K; V), warp 1 issues the MMAs
+// (one elected thread), warps 4-11 run the softmax and the epilogue (warp w
+// reads TMEM lanes 32 (w mod 4) .. +31).  Every mbarrier wait is bounded; on
+// expiry the CTA records BSA_ERR_TIMEOUT in the workspace error word, tells
+// the launch's other CTAs to give up (its own launch sequence number in the
+// control block), waits (bounded) for the copies and MMAs it has already
+// issued, frees its TMEM and leaves.
 #include <cmath>
 #include <cstdlib>
 
@@ -54,13 +63,12 @@ constexpr uint32_t kGroupThreads = 128;   // threads of one softmax group
 constexpr uint64_t kWaitNs = 250ull * 1000ull * 1000ull;  // 250 ms: far beyond any legitimate wait
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 256;     // O_0 at 256, O_1 at 384; S_0 at 0, S_1 at 128
-constexpr uint32_t kPTile = 128u * 128u * 2u;  // bf16 P of one 128 x 128 tile in shared memory
 
 struct Ctl {
   uint64_t q_full;
   uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
-  uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];   // per softmax group
-  uint64_t drain[2];   // final commit of each MMA issuer (S, P.V) before TMEM is freed
+  uint64_t s_full[2], p_full[2], pv_done[2];   // per softmax group
+  uint64_t drain;      // final commit of the MMA issuer before TMEM is freed
   uint32_t tmem_base;
   int n_ent;
   int item;
@@ -109,17 +117,22 @@ __device__ __forceinline__ bool pair_sync(int q4, bool ok) {
   return r != 0u;
 }
 
-template <int D, int BS, bool WITH_LSE>
-__global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_constant__ CUtensorMap mq,
+// MODE 0: O only; 1: O and the LSE; 2: O, the LSE and the entropy of each
+// row's attention distribution.
+template <int D, int BS, int MODE>
+__global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ CUtensorMap mq,
                                                                const __grid_constant__ CUtensorMap mk,
                                                                const __grid_constant__ CUtensorMap mv,
                                                                const int32_t* __restrict__ kv_count,
                                                                const int32_t* __restrict__ kv_idx,
                                                                const int2* __restrict__ items, int* work,
                                                                float scale_log2, __nv_bfloat16* __restrict__ o,
-                                                               float* __restrict__ lse, Ctrl* ctrl, Dims g,
+                                                               float* __restrict__ lse, float* __restrict__ ent,
+                                                               Ctrl* ctrl, Dims g,
                                                                int items_per_bh, int n_items, uint32_t seq,
                                                                int force_timeout) {
+  constexpr bool WITH_LSE = MODE >= 1;
+  constexpr bool WITH_ENT = MODE == 2;
   constexpr int QB = 128 / BS;          // query blocks per tile
   constexpr int E = 128 / BS;           // list entries per KV tile
   constexpr int CH = D / 64;            // 64-column (128-byte) chunks of a row
@@ -136,8 +149,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
   uint8_t* sQ = smem_raw;
   uint8_t* sK = sQ + kTile;            // two stages
   uint8_t* sV = sQ + 3 * kTile;        // two stages
-  uint8_t* sP = sQ + 5 * kTile;        // P of each softmax group
-  Ctl& c = *reinterpret_cast<Ctl*>(sP + 2 * kPTile);
+  Ctl& c = *reinterpret_cast<Ctl*>(sQ + 5 * kTile);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -157,11 +169,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(&c.s_full[w], 1);
-      mbar_init(&c.s_free[w], kGroupThreads);
       mbar_init(&c.p_full[w], kGroupThreads);
       mbar_init(&c.pv_done[w], 1);
-      mbar_init(&c.drain[w], 1);
     }
+    mbar_init(&c.drain, 1);
     c.abort = 0;
     fence_mbar_init();
   }
@@ -320,65 +331,56 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
           }
         }
       }
-    } else if (warp == 3) {
-      // ---------------------------------------------------------- S issuer
-      // KV tile j of the item belongs to softmax group w = j mod 2: its S goes
-      // to S buffer w as soon as the group has read its previous S (P lives
-      // in shared memory, so the S does not wait for any P.V product).
-      // Issued by its own thread, so an S never queues behind a wait for a P.
+    } else if (warp == 1) {
+      // ---------------------------------------------------------- MMA issuer
+      // S(0), S(1), then for each KV tile j: O_w += P(j) V(j) once group w
+      // has written P(j) and V(j) has landed, followed by S(j + 2) into the
+      // same TMEM buffer (in issue order: it overwrites P(j) only after the
+      // P.V product has read it).
       if (lane == 0 && n_tiles > 0) {
         constexpr uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);
+        constexpr uint32_t idO = idesc_bf16_f32(128, D, 0, 1);
         const uint64_t dQ = smem_desc_sw128(smem_addr(sQ), 16, 1024);
-        const uint32_t aK = smem_addr(sK);
+        const uint32_t aK = smem_addr(sK), aV = smem_addr(sV);
+        // S(jj) into buffer jj mod 2; false on a timeout
+        auto issue_s = [&](int jj) -> bool {
+          const uint32_t jg = jbase + jj, ks = jg & 1;
+          const int w = jj & 1;
+          if (!wait(&c.k_full[ks], (jg >> 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 21); return false; }
+          tc_fence_after();
+          // descriptors built once per tile: two adds per MMA
+          const uint64_t dK = smem_desc_sw128(aK + ks * kTile, 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
+            mma_ss(tmem + 128 * w, smem_desc_add(dQ, off), smem_desc_add(dK, off), idS, kk > 0);
+          }
+          mma_commit(&c.s_full[w]);
+          mma_commit(&c.k_empty[ks]);
+          return true;
+        };
+        bool go = true;
         if (!wait(&c.q_full, nq & 1, ctrl, seq)) {
           timeout(ctrl, c, seq, 20);
-        } else {
-          for (int j = 0; j < n_tiles; ++j) {
-            const uint32_t jg = jbase + j, ks = jg & 1;
-            const int w = j & 1;
-            const uint32_t gw = gbase[w] + (j >> 1);   // this group's tile count
-            if (!wait(&c.k_full[ks], (jg >> 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 21); break; }
-            if (gw >= 1 && !wait(&c.s_free[w], (gw - 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 22); break; }
-            tc_fence_after();
-            // descriptors built once per tile: the issuing thread shares its
-            // sub-partition with two softmax warps, so each MMA costs it only
-            // the two descriptor adds
-            const uint64_t dK = smem_desc_sw128(aK + ks * kTile, 16, 1024);
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
-              mma_ss(tmem + 128 * w, smem_desc_add(dQ, off), smem_desc_add(dK, off), idS, kk > 0);
-            }
-            mma_commit(&c.s_full[w]);
-            mma_commit(&c.k_empty[ks]);
-          }
+          go = false;
         }
-      }
-    } else if (warp == 1) {
-      // ---------------------------------------------------------- P.V issuer
-      // O_w += P V for KV tile j (group w = j mod 2) once the group's softmax
-      // has written P to shared memory and V has landed.
-      if (lane == 0 && n_tiles > 0) {
-        constexpr uint32_t idO = idesc_bf16_f32(128, D, 0, 1);
-        const uint32_t aV = smem_addr(sV), aP = smem_addr(sP);
-        for (int j = 0; j < n_tiles; ++j) {
+        for (int jj = 0; go && jj < 2 && jj < n_tiles; ++jj) go = issue_s(jj);
+        for (int j = 0; go && j < n_tiles; ++j) {
           const uint32_t jg = jbase + j, vs = jg & 1;
           const int w = j & 1;
           const uint32_t gw = gbase[w] + (j >> 1);
           if (!wait(&c.p_full[w], gw & 1, ctrl, seq)) { timeout(ctrl, c, seq, 23); break; }
           if (!wait(&c.v_full[vs], (jg >> 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 24); break; }
           tc_fence_after();
-          const uint64_t dP = smem_desc_sw128(aP + w * kPTile, 16, 1024);
           const uint64_t dV = smem_desc_sw128(aV + vs * kTile, kChunk, 1024);
           const uint32_t acc0 = (j >= 2) ? 1u : 0u;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
-            mma_ss(tmem + kTmemO + 128 * w, smem_desc_add(dP, off), smem_desc_add(dV, kk * 2048), idO,
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + kTmemO + 128 * w, tmem + 128 * w + 8 * kk, smem_desc_add(dV, kk * 2048), idO,
                    kk > 0 ? 1u : acc0);
-          }
           mma_commit(&c.pv_done[w]);
           mma_commit(&c.v_empty[vs]);
+          if (j + 2 < n_tiles) go = issue_s(j + 2);
         }
       }
     } else if (warp >= kSoftmaxWarp0) {
@@ -391,6 +393,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
       const uint32_t tS = trow + 128 * w, tOw = trow + kTmemO + 128 * w;
       float m = -INFINITY;
       float l = 0.f, lx = 0.f;
+      // entropy: vx = sum of p (y - m) over the row's weights p = 2^(y - m),
+      // y the base-2 logits, relative to the current running max m
+      float vx = 0.f;
       bool ok = true;
       int mine = 0;   // KV tiles this group ran in this item
       for (int j = w; j < n_tiles; j += 2, ++mine) {
@@ -409,6 +414,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
           }
           lim[h] = kept ? max(0, min(64, g.N - key0)) : 0;
         }
+        // S(j) complete: the commit behind it also covers this group's
+        // previous P.V product, so O_w and the P columns are free as well
         if (!wait_warp(&c.s_full[w], gw & 1, ctrl, seq)) { timeout(ctrl, c, seq, 30); ok = false; break; }
         tc_fence_after();
         // Pass 1: row max of the raw scores over the kept, real keys (scale > 0
@@ -440,10 +447,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
             mh[h] = mm;
           }
         }
-        // O_w and P buffer w are free once the group's previous P.V product
-        // has completed (normally long before: it was issued a tile ago).
-        if (gw >= 1 && !wait_warp(&c.pv_done[w], (gw - 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 32); ok = false; break; }
-        tc_fence_after();
         const float mnew = fmaxf(m, fmaxf(mh[0], mh[1]) * scale_log2);
         // The running max moves only when it grows by more than 8 (a factor
         // 256 in p), or when it is set for the first time.  The O rescale uses
@@ -463,6 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
             tmem_st32(tOw + cc, ov);
           }
           tmem_wait_st();
+          if (WITH_ENT && grow && m != -INFINITY) vx = alpha * (vx + (m - mnew) * lx);
           l *= alpha;
           lx *= alpha;
         }
@@ -475,12 +479,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
         // unrounded ones.  Halves the row's query block does not keep cost
         // nothing.
         // Pass 2, 32 keys at a time (the next chunk's load in flight): their
-        // bf16 weights go to row r of the group's P tile in shared memory
-        // (K-major, 128-byte swizzle: 16-byte unit u of a row at u ^ (r mod 8)).
-        // S buffer w is released as soon as its last chunk has been read.
-        uint8_t* prow = sP + w * kPTile + r * 128;
+        // bf16 weights, two per 32-bit column, go to columns [16 c, 16 c + 16)
+        // of the same TMEM buffer -- columns whose scores this pass has
+        // already read into registers.
         float rs[2] = {0.f, 0.f};
-        float rx = 0.f;
+        float rx = 0.f, ry = 0.f;
         const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(nm, nm);
         uint32_t sc[2][32];
         tmem_ld32(tS, sc[0]);
@@ -488,12 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
         for (int cch = 0; cch < 4; ++cch) {
           const int h = cch >> 1;
           tmem_wait_ld();
-          if (cch < 3) {
-            tmem_ld32(tS + 32 * (cch + 1), sc[(cch + 1) & 1]);
-          } else {
-            tc_fence_before();
-            mbar_arrive(&c.s_free[w]);
-          }
+          if (cch < 3) tmem_ld32(tS + 32 * (cch + 1), sc[(cch + 1) & 1]);
           const float* x = reinterpret_cast<const float*>(sc[cch & 1]);
           uint32_t pk[16];
           if (lim[h] > 0) {
@@ -513,22 +511,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
               pk[i] = pack_bf16(p.x, p.y);
               rs[i & 1] = add_bf16x2(rs[i & 1], pk[i]);
               if (WITH_LSE) rx += p.x + p.y;
+              if (WITH_ENT) ry = fmaf(p.x, y0, fmaf(p.y, y1, ry));
             }
           } else {
 #pragma unroll
             for (int i = 0; i < 16; ++i) pk[i] = 0u;
           }
-          uint8_t* pc = prow + (cch >> 1) * kChunk;
-#pragma unroll
-          for (int u4 = 0; u4 < 4; ++u4) {
-            const int u = (cch & 1) * 4 + u4;
-            *reinterpret_cast<uint4*>(pc + ((u ^ (r & 7)) << 4)) =
-                make_uint4(pk[4 * u4], pk[4 * u4 + 1], pk[4 * u4 + 2], pk[4 * u4 + 3]);
-          }
+          tmem_st16(tS + 16 * cch, pk);
         }
         l += rs[0] + rs[1];
         if (WITH_LSE) lx += rx;
-        fence_proxy_async_smem();   // the P stores, visible to the tensor core
+        if (WITH_ENT) vx += ry;
+        tmem_wait_st();             // the P stores, complete before the tensor core reads them
+        tc_fence_before();
         mbar_arrive(&c.p_full[w]);
       }
 
@@ -549,9 +544,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
       // (its softmax ran) and the next item's K loads start after the item.
       float* xm = reinterpret_cast<float*>(sK);   // [group][row]: running max
       float* xl = xm + 2 * 128;                   // [group][sum kind][row]: row sums
+      float* xv = xl + 4 * 128;                   // [group][row]: entropy sums
       xm[w * 128 + r] = (mine > 0) ? m : -INFINITY;
       xl[(2 * w + 0) * 128 + r] = l;
       xl[(2 * w + 1) * 128 + r] = lx;
+      if (WITH_ENT) xv[w * 128 + r] = vx;
       tc_fence_before();
       ok = pair_sync(q4, ok);
       tc_fence_after();
@@ -600,6 +597,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
       }
       if (WITH_LSE && w == 0 && store)
         lse[(size_t)bh * g.Npad + grow] = real ? (mt + __log2f(lxt)) * 0.69314718055994531f : 0.f;
+      if (WITH_ENT && w == 0 && store) {
+        // H = -sum p ln p with p = 2^(y - mt) / lxt: ln 2 (log2 lxt - sum 2^(y - mt) (y - mt) / lxt)
+        float vt = 0.f;
+        if (has0 && m0 != -INFINITY) vt += a0 * (xv[r] + (m0 - mt) * xl[128 + r]);
+        if (has1 && m1 != -INFINITY) vt += a1 * (xv[128 + r] + (m1 - mt) * xl[3 * 128 + r]);
+        ent[(size_t)bh * g.Npad + grow] = real ? (__log2f(lxt) - vt / lxt) * 0.69314718055994531f : 0.f;
+      }
       fence_proxy_async_smem();   // the merge's accesses, ordered before the next K loads
     }
 
@@ -622,10 +626,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc2_kernel(const __grid_cons
       mbar_drain_ring(c.k_full, 2, armed, kWaitNs);
     } else if (warp == 2) {
       mbar_drain_ring(c.v_full, 2, armed, kWaitNs);
-    } else if (warp == 3 || warp == 1) {
-      uint64_t* d = &c.drain[warp == 3 ? 0 : 1];
-      mma_commit(d);
-      mbar_wait_ns(d, 0, kWaitNs, nullptr, 0u);
+    } else if (warp == 1) {
+      mma_commit(&c.drain);
+      mbar_wait_ns(&c.drain, 0, kWaitNs, nullptr, 0u);
     }
   }
   tc_fence_before();
@@ -651,10 +654,10 @@ int num_sms() {
   return n;
 }
 
-template <int D, int BS, bool WITH_LSE>
-cudaError_t launch_tc2(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
+template <int D, int BS, int MODE>
+cudaError_t launch_fwd(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
                        const int32_t* kv_idx, const int2* items, int* work, float scale, void* o, float* lse,
-                       Ctrl* ctrl, uint32_t seq, cudaStream_t st) {
+                       float* ent, Ctrl* ctrl, uint32_t seq, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
   const uint64_t rows = (uint64_t)g.Npad, bhs = (uint64_t)g.B * g.heads;
   if (!make_map_bf16_3d(&mq, q, D, rows, bhs, 64, 64) || !make_map_bf16_3d(&mk, k, D, rows, bhs, 64, 64) ||
@@ -662,40 +665,42 @@ cudaError_t launch_tc2(const Dims& g, const void* q, const void* k, const void* 
     return cudaErrorInvalidValue;
   const int items_per_bh = (BS == 64) ? (g.nb + 1) / 2 : g.nb;
   const int n_items = (int)(bhs * items_per_bh);
-  const size_t smem = 5u * 128u * D * 2u + 2u * kPTile + sizeof(Ctl);
-  static_assert(5u * 128u * 128u * 2u + 2u * kPTile + sizeof(Ctl) <= 227u * 1024u, "shared memory layout");
+  const size_t smem = 5u * 128u * D * 2u + sizeof(Ctl);
+  static_assert(5u * 128u * 128u * 2u + sizeof(Ctl) <= 227u * 1024u, "shared memory layout");
   cudaError_t e =
-      cudaFuncSetAttribute(attn_tc2_kernel<D, BS, WITH_LSE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      cudaFuncSetAttribute(attn_fwd_kernel<D, BS, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int grid = n_items < num_sms() ? n_items : num_sms();
-  attn_tc2_kernel<D, BS, WITH_LSE><<<grid, kThreads, smem, st>>>(mq, mk, mv, kv_count, kv_idx, items, work,
+  attn_fwd_kernel<D, BS, MODE><<<grid, kThreads, smem, st>>>(mq, mk, mv, kv_count, kv_idx, items, work,
                                                                  scale * 1.4426950408889634f, (__nv_bfloat16*)o, lse,
-                                                                 ctrl, g, items_per_bh, n_items, seq,
+                                                                 ent, ctrl, g, items_per_bh, n_items, seq,
                                                                  force_timeout_requested());
   return cudaGetLastError();
 }
 
 template <int D, int BS>
-cudaError_t launch_tc2_lse(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
+cudaError_t launch_fwd_mode(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
                            const int32_t* kv_idx, const int2* items, int* work, float scale, void* o, float* lse,
-                           Ctrl* ctrl, uint32_t seq, cudaStream_t st) {
+                           float* ent, Ctrl* ctrl, uint32_t seq, cudaStream_t st) {
+  if (ent != nullptr)
+    return launch_fwd<D, BS, 2>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ent, ctrl, seq, st);
   if (lse != nullptr)
-    return launch_tc2<D, BS, true>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, seq, st);
-  return launch_tc2<D, BS, false>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, seq, st);
+    return launch_fwd<D, BS, 1>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ent, ctrl, seq, st);
+  return launch_fwd<D, BS, 0>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ent, ctrl, seq, st);
 }
 
 }  // namespace
 
-cudaError_t launch_attn_tc2(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
-                            const int32_t* kv_idx, const int2* items, int* work, float scale, void* o, float* lse,
-                            Ctrl* ctrl, uint32_t seq, cudaStream_t st) {
+cudaError_t launch_attn(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
+                        const int32_t* kv_idx, const int2* items, int* work, float scale, void* o, float* lse,
+                        float* ent, Ctrl* ctrl, uint32_t seq, cudaStream_t st) {
   if (g.d == 128 && g.bs == 64)
-    return launch_tc2_lse<128, 64>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, seq, st);
+    return launch_fwd_mode<128, 64>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ent, ctrl, seq, st);
   if (g.d == 128 && g.bs == 128)
-    return launch_tc2_lse<128, 128>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, seq, st);
+    return launch_fwd_mode<128, 128>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ent, ctrl, seq, st);
   if (g.d == 64 && g.bs == 64)
-    return launch_tc2_lse<64, 64>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, seq, st);
-  return launch_tc2_lse<64, 128>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, seq, st);
+    return launch_fwd_mode<64, 64>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ent, ctrl, seq, st);
+  return launch_fwd_mode<64, 128>(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ent, ctrl, seq, st);
 }
 
 }  // namespace bsa

@@ -15,15 +15,6 @@ using bsa::Dims;
 
 namespace bsa {
 
-cudaError_t launch_attn(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
-                        const int32_t* kv_idx, const int2* items, int* work, float scale, void* o, float* lse,
-                        Ctrl* ctrl, uint32_t seq, cudaStream_t st) {
-  const char* pick = std::getenv("BSA_ATTN_KERNEL");
-  if (pick != nullptr && std::strcmp(pick, "tc2") == 0)
-    return launch_attn_tc2(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, seq, st);
-  return launch_attn_tc3(g, q, k, v, kv_count, kv_idx, items, work, scale, o, lse, ctrl, seq, st);
-}
-
 uint32_t next_launch_seq() {
   static std::atomic<uint32_t> counter{0};
   uint32_t s;
@@ -206,8 +197,8 @@ bsa_status bsa_build_block_mask(const bsa_shape* s, const void* q_bhnd, const vo
 namespace {
 
 bsa_status attn_common(const bsa_shape* s, const void* q, const void* k, const void* v, const int32_t* kv_count,
-                       const int32_t* kv_idx, float scale, void* o, float* lse_or_null, void* workspace,
-                       size_t ws_bytes, bsa_stream_t stream, bool baseline) {
+                       const int32_t* kv_idx, float scale, void* o, float* lse_or_null, float* ent_or_null,
+                       void* workspace, size_t ws_bytes, bsa_stream_t stream, bool baseline) {
   Dims g;
   bsa_status st = check_shape(s, &g);
   if (st != BSA_OK) return st;
@@ -216,7 +207,8 @@ bsa_status attn_common(const bsa_shape* s, const void* q, const void* k, const v
       workspace == nullptr)
     return BSA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(kv_count) ||
-      !aligned16(kv_idx) || !aligned16(workspace) || (lse_or_null != nullptr && !aligned16(lse_or_null)))
+      !aligned16(kv_idx) || !aligned16(workspace) || (lse_or_null != nullptr && !aligned16(lse_or_null)) ||
+      (ent_or_null != nullptr && !aligned16(ent_or_null)))
     return BSA_ERR_INVALID_ARG;
   if (ws_bytes < workspace_bytes(g)) return BSA_ERR_INVALID_ARG;
   if (!std::isfinite(scale) || scale < 0.0f) return BSA_ERR_INVALID_ARG;
@@ -229,7 +221,7 @@ bsa_status attn_common(const bsa_shape* s, const void* q, const void* k, const v
   cudaError_t e = bsa::launch_plan(g, kv_count, kv_idx, items, (cudaStream_t)stream);
   if (e != cudaSuccess) return BSA_ERR_CUDA;
   return from_cuda(bsa::launch_attn(g, q, k, v, kv_count, kv_idx, items, bsa::plan_work_counter(g, items), scale, o,
-                                   lse_or_null, ctrl, bsa::next_launch_seq(), (cudaStream_t)stream));
+                                   lse_or_null, ent_or_null, ctrl, bsa::next_launch_seq(), (cudaStream_t)stream));
 }
 
 }  // namespace
@@ -239,13 +231,32 @@ extern "C" {
 bsa_status bsa_attn_fwd(const bsa_shape* s, const void* q, const void* k, const void* v, const int32_t* kv_count,
                         const int32_t* kv_idx, float scale, void* o, float* lse_or_null, void* workspace,
                         size_t ws_bytes, bsa_stream_t stream) {
-  return attn_common(s, q, k, v, kv_count, kv_idx, scale, o, lse_or_null, workspace, ws_bytes, stream, false);
+  return attn_common(s, q, k, v, kv_count, kv_idx, scale, o, lse_or_null, nullptr, workspace, ws_bytes, stream,
+                     false);
+}
+
+bsa_status bsa_attn_fwd_entropy(const bsa_shape* s, const void* q, const void* k, const void* v,
+                                const int32_t* kv_count, const int32_t* kv_idx, float scale, void* o, float* lse,
+                                float* entropy, void* workspace, size_t ws_bytes, bsa_stream_t stream) {
+  if (lse == nullptr || entropy == nullptr) return BSA_ERR_INVALID_ARG;
+  return attn_common(s, q, k, v, kv_count, kv_idx, scale, o, lse, entropy, workspace, ws_bytes, stream, false);
+}
+
+bsa_status bsa_dense_lists(const bsa_shape* s, int32_t* kv_count, int32_t* kv_idx, bsa_stream_t stream) {
+  Dims g;
+  bsa_status st = check_shape(s, &g);
+  if (st != BSA_OK) return st;
+  if (g.nb > BSA_MAX_BLOCKS) return BSA_ERR_UNSUPPORTED;
+  if (kv_count == nullptr || kv_idx == nullptr || !aligned16(kv_count) || !aligned16(kv_idx))
+    return BSA_ERR_INVALID_ARG;
+  return from_cuda(bsa::launch_dense_lists(g, kv_count, kv_idx, (cudaStream_t)stream));
 }
 
 bsa_status bsa_attn_fwd_baseline(const bsa_shape* s, const void* q, const void* k, const void* v,
                                  const int32_t* kv_count, const int32_t* kv_idx, float scale, void* o,
                                  float* lse_or_null, void* workspace, size_t ws_bytes, bsa_stream_t stream) {
-  return attn_common(s, q, k, v, kv_count, kv_idx, scale, o, lse_or_null, workspace, ws_bytes, stream, true);
+  return attn_common(s, q, k, v, kv_count, kv_idx, scale, o, lse_or_null, nullptr, workspace, ws_bytes, stream,
+                     true);
 }
 
 }  // extern "C"
@@ -327,6 +338,22 @@ bsa_status bsa_attn_bwd(const bsa_shape* s, const void* q, const void* k, const 
   if (bsa::launch_plan(g, kv_count, kv_idx, items_q, cs) != cudaSuccess) return BSA_ERR_CUDA;
   if (bsa::launch_plan(g, a.q_count, a.q_idx, items_kv, cs) != cudaSuccess) return BSA_ERR_CUDA;
   return from_cuda(bsa::launch_attn_bwd(g, a, cs));
+}
+
+bsa_status bsa_build_block_mask_radius(const bsa_shape* s, const float* entropy, float tau, float gamma,
+                                       int32_t vote, int32_t* kv_count, int32_t* kv_idx, uint8_t* mask_or_null,
+                                       bsa_stream_t stream) {
+  Dims g;
+  bsa_status st = check_shape(s, &g);
+  if (st != BSA_OK) return st;
+  if (g.nb > BSA_MAX_BLOCKS || g.T > 1024) return BSA_ERR_UNSUPPORTED;
+  if (!(tau > 0.0f) || !std::isfinite(tau) || !(gamma >= 0.0f) || !std::isfinite(gamma) || vote < 1)
+    return BSA_ERR_INVALID_ARG;
+  if (entropy == nullptr || kv_count == nullptr || kv_idx == nullptr || !aligned16(entropy) || !aligned16(kv_count) ||
+      !aligned16(kv_idx))
+    return BSA_ERR_INVALID_ARG;
+  return from_cuda(bsa::launch_radius_mask(g, entropy, (double)tau, (double)gamma, vote, kv_count, kv_idx,
+                                           mask_or_null, (cudaStream_t)stream));
 }
 
 size_t bsa_hilbert_workspace_bytes(const bsa_shape* s) {

@@ -46,19 +46,13 @@ int* plan_work_counter(const Dims& g, int2* items);
 cudaError_t launch_plan(const Dims& g, const int32_t* kv_count, const int32_t* kv_idx, int2* items, cudaStream_t st);
 
 // Block-sparse attention on the tcgen05 tensor cores (TMEM accumulators,
-// TMA-staged tiles): persistent, one CTA per SM, two softmax groups on
-// alternating KV tiles, query tiles fetched from the plan's work counter.
-// tc2 stages P in shared memory, tc3 in tensor memory; launch_attn picks the
-// kernel the entry points use.
+// TMA-staged tiles, P in TMEM): persistent, one CTA per SM, two softmax
+// groups on alternating KV tiles, query tiles fetched from the plan's work
+// counter.  `lse` and `ent` (the entropy of each row's attention
+// distribution, nats) are optional outputs.
 cudaError_t launch_attn(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
                         const int32_t* kv_idx, const int2* items, int* work, float scale, void* o, float* lse,
-                        Ctrl* ctrl, uint32_t seq, cudaStream_t st);
-cudaError_t launch_attn_tc3(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
-                            const int32_t* kv_idx, const int2* items, int* work, float scale, void* o, float* lse,
-                            Ctrl* ctrl, uint32_t seq, cudaStream_t st);
-cudaError_t launch_attn_tc2(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
-                            const int32_t* kv_idx, const int2* items, int* work, float scale, void* o, float* lse,
-                            Ctrl* ctrl, uint32_t seq, cudaStream_t st);
+                        float* ent, Ctrl* ctrl, uint32_t seq, cudaStream_t st);
 
 // Hilbert-curve token order (order.cu): order[p] = the token at position p.
 // Scratch: the tokens' curve indices, a bitmap over the enclosing cube and
@@ -92,6 +86,12 @@ SubblockLayout subblock_layout(const Dims& g, int sub);
 cudaError_t launch_mask_subblock(const Dims& g, int sub, const void* q, const void* k, double thr,
                                  int32_t* kv_count, int32_t* kv_idx, uint8_t* mask, void* workspace, uint32_t seq,
                                  cudaStream_t st);
+
+// Token-radius block masks (radius.cu): dense lists for the warm-up pass, and
+// the mask from per-token entropies [B, heads, Npad].
+cudaError_t launch_dense_lists(const Dims& g, int32_t* kv_count, int32_t* kv_idx, cudaStream_t st);
+cudaError_t launch_radius_mask(const Dims& g, const float* entropy, double tau, double gamma, int vote,
+                               int32_t* kv_count, int32_t* kv_idx, uint8_t* mask, cudaStream_t st);
 
 // Backward pass (attn_bwd.cu).  Every pointer is device memory; the planner
 // regions (items_q / items_kv with their work counters) are filled by

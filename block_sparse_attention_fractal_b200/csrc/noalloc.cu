@@ -131,7 +131,7 @@ bsa_status bsa_attn_fwd_noalloc(const bsa_shape* s, const void* q, const void* k
   if (cudaMemsetAsync(ctrl, 0, sizeof(Ctrl), cs) != cudaSuccess) return BSA_ERR_CUDA;
   if (bsa::launch_plan(g, kv_count, kv_idx, items, cs) != cudaSuccess) return BSA_ERR_CUDA;
   if (bsa::launch_attn(g, q, k, v, kv_count, kv_idx, items, bsa::plan_work_counter(g, items), scale, o, lse_or_null,
-                       ctrl, bsa::next_launch_seq(), cs) != cudaSuccess)
+                       nullptr, ctrl, bsa::next_launch_seq(), cs) != cudaSuccess)
     return BSA_ERR_CUDA;
   if (error_word_or_null != nullptr &&
       cudaMemcpyAsync(error_word_or_null, &ctrl->error, sizeof(uint32_t), cudaMemcpyDeviceToDevice, cs) !=

@@ -180,6 +180,45 @@ BSA_API bsa_status bsa_attn_fwd(const bsa_shape* s, const void* q, const void* k
                         void* workspace, size_t ws_bytes, bsa_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Token-radius masks (TRA summary, gist.science/es/paper/2608.02504, section
+ * 2): entropy -> budget -> radius -> block mask, in the same list format.
+ * ------------------------------------------------------------------------- */
+
+/* bsa_attn_fwd that also writes, for every valid query row, the entropy (in
+ * nats) of its attention distribution over the listed keys,
+ * H = -sum_k p_k ln p_k, and its LSE (both required).  TRA summary, section 2
+ * ("Entropia-a-Presupuesto"): the dense warm-up pass that measures each
+ * query's entropy (with dense lists, see bsa_dense_lists).
+ *   lse, entropy: device, [B, heads, Npad] float32, written (0 for padded rows).
+ *   Other arguments and errors as for bsa_attn_fwd. */
+BSA_API bsa_status bsa_attn_fwd_entropy(const bsa_shape* s, const void* q, const void* k, const void* v,
+                                        const int32_t* kv_count, const int32_t* kv_idx, float scale, void* o,
+                                        float* lse, float* entropy, void* workspace, size_t ws_bytes,
+                                        bsa_stream_t stream);
+
+/* Lists that keep every block (kv_count = nb, kv_idx[b, h, I, J] = J): the
+ * dense attention of a warm-up pass. */
+BSA_API bsa_status bsa_dense_lists(const bsa_shape* s, int32_t* kv_count, int32_t* kv_idx, bsa_stream_t stream);
+
+/* Block mask from token radii, TRA summary, section 2 ("Presupuesto-a-Radio",
+ * "Ejecucion Eficiente").  Per valid query token i at (t_i, h_i, w_i), with
+ * phi(d) = exp(-gamma d):
+ *   budget_i = clamp(tau * exp(entropy_i), 1, N) keys;
+ *   r_i = sqrt(budget_i / (pi * sum_t phi(|t - t_i|)^2)) (the disks of radius
+ *         r_i phi(|t - t_i|) in every frame hold the budget in area);
+ *   key j is in i's support when (h_j-h_i)^2 + (w_j-w_i)^2 <= (r_i phi(|t_j-t_i|))^2;
+ * query token i votes for key block J when J holds a key of its support, and
+ * block I keeps J when at least `vote` of I's valid tokens vote for J.  Tokens
+ * are in the fractal order (the tile-major layout the summary asks for).
+ * Radii and comparisons in double precision.
+ *   entropy: device, [B, heads, Npad] float32 (bsa_attn_fwd_entropy).
+ *   tau > 0, gamma >= 0, vote >= 1; T <= 1024.
+ *   kv_count, kv_idx, mask_or_null: as written by bsa_build_block_mask. */
+BSA_API bsa_status bsa_build_block_mask_radius(const bsa_shape* s, const float* entropy, float tau, float gamma,
+                                               int32_t vote, int32_t* kv_count, int32_t* kv_idx,
+                                               uint8_t* mask_or_null, bsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Alternative token order and block estimator (DFSAttn explainer,
  * gist.science/es/paper/2605.23445, sections 1 and 2): a 3-D Hilbert-curve
  * order of the tokens, and block importance from finer sub-block scores,

@@ -117,7 +117,8 @@ def block_means(y_bhnd: np.ndarray, N: int, block: int) -> np.ndarray:
     for I in range(nb):
         lo = I * block
         hi = min((I + 1) * block, N)
-        out[:, :, I, :] = y_bhnd[:, :, lo:hi, :].sum(axis=2) / float(hi - lo)
+        if hi > lo:                       # a block past the last token has no mean (left 0)
+            out[:, :, I, :] = y_bhnd[:, :, lo:hi, :].sum(axis=2) / float(hi - lo)
     return out
 
 
