@@ -63,16 +63,6 @@ constexpr uint32_t kGroupThreads = 128;   // threads of one softmax group
 constexpr uint64_t kWaitNs = 250ull * 1000ull * 1000ull;  // 250 ms: far beyond any legitimate wait
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 256;     // O_0 at 256, O_1 at 384; S_0 at 0, S_1 at 128
-// Softmax variants (tuning knobs): one pass per tile once a row's max is set,
-// and one pair of scores in kPolyEvery through the FMA-pipe exp2 (0 = none).
-#ifndef BSA_SOFTMAX_ONEPASS
-#define BSA_SOFTMAX_ONEPASS 0
-#endif
-#ifndef BSA_POLY_EVERY
-#define BSA_POLY_EVERY 0
-#endif
-constexpr bool kOnePass = BSA_SOFTMAX_ONEPASS != 0;
-constexpr int kPolyEvery = BSA_POLY_EVERY;
 
 struct Ctl {
   uint64_t q_full;
@@ -428,147 +418,110 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         // previous P.V product, so O_w and the P columns are free as well
         if (!wait_warp(&c.s_full[w], gw & 1, ctrl, seq)) { timeout(ctrl, c, seq, 30); ok = false; break; }
         tc_fence_after();
-        // The exp pass, 32 keys at a time (the next chunk's load in flight):
-        // p = 2^(s * scale_log2 - m) with one packed FMA for two arguments,
-        // MUFU ex2 for most pairs and the FMA-pipe polynomial for one pair in
-        // kPolyEvery; the bf16 weights, two per 32-bit column, go to columns
-        // [16 c, 16 c + 16) of the same TMEM buffer (columns whose scores
-        // this pass has already read).  Returns the sums over the bf16
-        // weights (O is normalised by the weights the P.V product uses: an
-        // exact convex combination of V rows up to accumulation rounding),
-        // over the fp32 weights (LSE) and of p * (y - m) (entropy), and, when
-        // asked, the largest y - m of the kept keys.  Halves the row's query
-        // block does not keep cost nothing.
-        auto exp_pass = [&](float nm, bool track, float& s_l, float& s_x, float& s_y, float& ymax) {
-          float rs[2] = {0.f, 0.f};
-          float rx = 0.f, ry = 0.f, ym = -INFINITY;
-          const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(nm, nm);
-          uint32_t sc[2][32];
-          tmem_ld32(tS, sc[0]);
+        // Pass 1: row max of the raw scores over the kept, real keys (scale > 0
+        // keeps the order), 64 columns at a time.
+        float mh[2];
 #pragma unroll
-          for (int cch = 0; cch < 4; ++cch) {
-            const int h = cch >> 1;
-            tmem_wait_ld();
-            if (cch < 3) tmem_ld32(tS + 32 * (cch + 1), sc[(cch + 1) & 1]);
-            const float* x = reinterpret_cast<const float*>(sc[cch & 1]);
-            uint32_t pk[16];
+        for (int h = 0; h < 2; ++h) {
+          uint32_t sr[64];
+          tmem_ld32(tS + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+          tmem_ld32(tS + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+          tmem_wait_ld();
+          const float* xh = reinterpret_cast<const float*>(sr);
+          if (lim[h] == 64) {
+            float m0 = xh[0], m1 = xh[1], m2 = xh[2], m3 = xh[3];
+#pragma unroll
+            for (int i = 4; i < 64; i += 8) {
+              m0 = fmax3(m0, xh[i], xh[i + 1]);
+              m1 = fmax3(m1, xh[i + 2], xh[i + 3]);
+              m2 = fmax3(m2, xh[i + 4], xh[i + 5]);
+              m3 = fmax3(m3, xh[i + 6], xh[i + 7]);
+            }
+            mh[h] = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+          } else {
+            float mm = -INFINITY;
             if (lim[h] > 0) {
 #pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const float2 yy = ffma2(make_float2(x[2 * i], x[2 * i + 1]), sc2, nm2);
-                float2 p;
-                if (kPolyEvery > 0 && (i % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
-                  p = exp2_fma2(yy);
-                } else {
-                  p.x = ex2f(yy.x);
-                  p.y = ex2f(yy.y);
-                }
-                if (lim[h] < 64) {
-                  const int kc = (cch & 1) * 32 + 2 * i;   // key within the half
-                  const bool k0 = kc < lim[h], k1 = kc + 1 < lim[h];
-                  p.x = k0 ? p.x : 0.f;
-                  p.y = k1 ? p.y : 0.f;
-                  if (track) ym = fmax3(ym, k0 ? yy.x : -INFINITY, k1 ? yy.y : -INFINITY);
-                } else if (track) {
-                  ym = fmax3(ym, yy.x, yy.y);
-                }
-                pk[i] = pack_bf16(p.x, p.y);
-                rs[i & 1] = add_bf16x2(rs[i & 1], pk[i]);
-                if (WITH_LSE) rx += p.x + p.y;
-                if (WITH_ENT) ry = fmaf(p.x, yy.x, fmaf(p.y, yy.y, ry));
-              }
-            } else {
-#pragma unroll
-              for (int i = 0; i < 16; ++i) pk[i] = 0u;
+              for (int i = 0; i < 64; ++i) mm = (i < lim[h]) ? fmaxf(mm, xh[i]) : mm;
             }
-            tmem_st16(tS + 16 * cch, pk);
+            mh[h] = mm;
           }
-          s_l = rs[0] + rs[1];
-          s_x = rx;
-          s_y = ry;
-          ymax = ym;
-        };
-        // The running max m moves only when the row's scores grow by more
-        // than 8 past it (a factor 256 in p), or when it is set for the first
-        // time.  The O rescale uses warp-collective TMEM accesses, so the
-        // whole warp takes it when any lane needs it (lanes whose max did not
-        // move use alpha = 1).  O_w is stable: its last P.V product has
-        // completed (the commit behind S(j) covers it).
-        auto rescale_to = [&](float mnew, bool grow) {
-          if (__any_sync(0xffffffffu, grow && m != -INFINITY)) {
-            const float alpha = (grow && m != -INFINITY) ? ex2f(m - mnew) : 1.0f;
+        }
+        const float mnew = fmaxf(m, fmaxf(mh[0], mh[1]) * scale_log2);
+        // The running max moves only when it grows by more than 8 (a factor
+        // 256 in p), or when it is set for the first time.  The O rescale uses
+        // warp-collective TMEM accesses, so the whole warp takes it when any
+        // lane needs it (lanes whose max did not move use alpha = 1).  O_w is
+        // stable: its last P.V product has completed (waited above).
+        const bool grow = mnew > m + 8.0f;
+        if (__any_sync(0xffffffffu, grow && m != -INFINITY)) {
+          const float alpha = (grow && m != -INFINITY) ? ex2f(m - mnew) : 1.0f;
 #pragma unroll 1
-            for (int cc = 0; cc < D; cc += 32) {
-              uint32_t ov[32];
-              tmem_ld32(tOw + cc, ov);
-              tmem_wait_ld();
+          for (int cc = 0; cc < D; cc += 32) {
+            uint32_t ov[32];
+            tmem_ld32(tOw + cc, ov);
+            tmem_wait_ld();
 #pragma unroll
-              for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-              tmem_st32(tOw + cc, ov);
-            }
-            tmem_wait_st();
-            if (WITH_ENT && grow && m != -INFINITY) vx = alpha * (vx + (m - mnew) * lx);
-            l *= alpha;
-            lx *= alpha;
+            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+            tmem_st32(tOw + cc, ov);
           }
-          if (grow) m = mnew;
-        };
-        float t_l, t_x, t_y, t_ym;
-        // One pass when every lane with kept keys has its max already: the
-        // weights use the running max, and the tile is redone (after the
-        // rescale) only if some row's scores outgrow it by more than 8.
-        const bool need_max = __any_sync(0xffffffffu, m == -INFINITY && (lim[0] > 0 || lim[1] > 0));
-        bool done = false;
-        if (kOnePass && !need_max) {
-          exp_pass(-m, true, t_l, t_x, t_y, t_ym);
-          const bool grow = t_ym > 8.0f;
-          if (!__any_sync(0xffffffffu, grow)) {
-            done = true;
-          } else {
-            rescale_to(m + t_ym, grow);
-          }
+          tmem_wait_st();
+          if (WITH_ENT && grow && m != -INFINITY) vx = alpha * (vx + (m - mnew) * lx);
+          l *= alpha;
+          lx *= alpha;
         }
-        if (!done) {
-          if (kOnePass && !need_max) {
-            exp_pass((m == -INFINITY) ? 0.f : -m, false, t_l, t_x, t_y, t_ym);
-          } else {
-            // Pass 1: row max of the raw scores over the kept, real keys
-            // (scale > 0 keeps the order), 64 columns at a time; then the exp pass.
-            float mh[2];
+        if (grow) m = mnew;
+        const float nm = (m == -INFINITY) ? 0.f : -m;
+        // p = 2^(s * scale_log2 - m): one FFMA and one MUFU ex2 per score.  O is
+        // normalised by the sum of the bf16-rounded weights the P.V product
+        // uses (an exact convex combination of V rows up to accumulation
+        // rounding); the LSE, when asked for, uses the fp32 sum of the
+        // unrounded ones.  Halves the row's query block does not keep cost
+        // nothing.
+        // Pass 2, 32 keys at a time (the next chunk's load in flight): their
+        // bf16 weights, two per 32-bit column, go to columns [16 c, 16 c + 16)
+        // of the same TMEM buffer -- columns whose scores this pass has
+        // already read into registers.
+        float rs[2] = {0.f, 0.f};
+        float rx = 0.f, ry = 0.f;
+        const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(nm, nm);
+        uint32_t sc[2][32];
+        tmem_ld32(tS, sc[0]);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              uint32_t sr[64];
-              tmem_ld32(tS + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-              tmem_ld32(tS + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-              tmem_wait_ld();
-              const float* xh = reinterpret_cast<const float*>(sr);
-              if (lim[h] == 64) {
-                float m0 = xh[0], m1 = xh[1], m2 = xh[2], m3 = xh[3];
+        for (int cch = 0; cch < 4; ++cch) {
+          const int h = cch >> 1;
+          tmem_wait_ld();
+          if (cch < 3) tmem_ld32(tS + 32 * (cch + 1), sc[(cch + 1) & 1]);
+          const float* x = reinterpret_cast<const float*>(sc[cch & 1]);
+          uint32_t pk[16];
+          if (lim[h] > 0) {
 #pragma unroll
-                for (int i = 4; i < 64; i += 8) {
-                  m0 = fmax3(m0, xh[i], xh[i + 1]);
-                  m1 = fmax3(m1, xh[i + 2], xh[i + 3]);
-                  m2 = fmax3(m2, xh[i + 4], xh[i + 5]);
-                  m3 = fmax3(m3, xh[i + 6], xh[i + 7]);
-                }
-                mh[h] = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
-              } else {
-                float mm = -INFINITY;
-                if (lim[h] > 0) {
-#pragma unroll
-                  for (int i = 0; i < 64; ++i) mm = (i < lim[h]) ? fmaxf(mm, xh[i]) : mm;
-                }
-                mh[h] = mm;
+            for (int i = 0; i < 16; ++i) {
+              // both arguments in one fma.rn.f32x2 (half the issue slots)
+              const float2 yy = ffma2(make_float2(x[2 * i], x[2 * i + 1]), sc2, nm2);
+              const float y0 = yy.x, y1 = yy.y;
+              float2 p;
+              p.x = ex2f(y0);
+              p.y = ex2f(y1);
+              if (lim[h] < 64) {
+                const int kc = (cch & 1) * 32 + 2 * i;   // key within the half
+                p.x = (kc < lim[h]) ? p.x : 0.f;
+                p.y = (kc + 1 < lim[h]) ? p.y : 0.f;
               }
+              pk[i] = pack_bf16(p.x, p.y);
+              rs[i & 1] = add_bf16x2(rs[i & 1], pk[i]);
+              if (WITH_LSE) rx += p.x + p.y;
+              if (WITH_ENT) ry = fmaf(p.x, y0, fmaf(p.y, y1, ry));
             }
-            const float mnew = fmaxf(m, fmaxf(mh[0], mh[1]) * scale_log2);
-            rescale_to(mnew, mnew > m + 8.0f);
-            exp_pass((m == -INFINITY) ? 0.f : -m, false, t_l, t_x, t_y, t_ym);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[i] = 0u;
           }
+          tmem_st16(tS + 16 * cch, pk);
         }
-        l += t_l;
-        if (WITH_LSE) lx += t_x;
-        if (WITH_ENT) vx += t_y;
+        l += rs[0] + rs[1];
+        if (WITH_LSE) lx += rx;
+        if (WITH_ENT) vx += ry;
         tmem_wait_st();             // the P stores, complete before the tensor core reads them
         tc_fence_before();
         mbar_arrive(&c.p_full[w]);
