@@ -685,6 +685,75 @@ def test_pins_catch_a_radius_mask_without_temporal_decay(monkeypatch):
         test_radius_block_mask_by_brute_force(0.7, 1)
 
 
+# ----------------------------------------------- fine-grained KV selection
+
+def _fine_lists(keep_blocks, per):
+    """CSR lists of 4-token blocks covering the kept 64-token blocks (nq x nb bool)."""
+    off, idx = [0], []
+    for row in keep_blocks:
+        for J in np.nonzero(row)[0]:
+            idx.extend(range(J * per, (J + 1) * per))
+        off.append(len(idx))
+    return np.asarray(off), np.asarray(idx)
+
+
+def test_fine_attention_with_whole_blocks_is_block_sparse_attention():
+    rng = np.random.default_rng(31)
+    N, qb, d = 250, 128, 16
+    Npad = nabla.padded_len(N, qb)
+    q, k, v = (rng.standard_normal((1, 1, Npad, d)) for _ in range(3))
+    keep = rng.random((1, 1, Npad // qb, Npad // qb)) < 0.6
+    keep[..., np.arange(Npad // qb), np.arange(Npad // qb)] = True
+    off, idx = _fine_lists(keep[0, 0], qb // 4)
+    O, lse = oracle.fine_attention(q, k, v, off, idx, None, N)
+    O_ref, lse_ref = oracle.masked_attention(q, k, v, keep, N, qb)
+    assert np.allclose(O, O_ref, atol=1e-13) and np.allclose(lse, lse_ref, atol=1e-13)
+
+
+def test_fine_attention_weights_against_library_attention():
+    """Weights as an additive log mask in torch SDPA (float64); a uniform
+    weight changes nothing (the softmax is shift invariant); a weight of 3 on a
+    block acts as three copies of it."""
+    rng = np.random.default_rng(32)
+    N, d = 100, 8
+    Npad = nabla.padded_len(N, 128)
+    q, k, v = (rng.standard_normal((1, 1, Npad, d)) for _ in range(3))
+    idx = np.sort(rng.choice(N // 4, size=9, replace=False))
+    w = rng.uniform(1.0, 6.0, idx.size)
+    off = np.array([0, idx.size])
+    O, _ = oracle.fine_attention(q, k, v, off, idx, w, N)
+    cols = np.concatenate([np.arange(4 * b, 4 * b + 4) for b in idx])
+    bias = torch.from_numpy(np.repeat(np.log(w), 4))[None, :].expand(N, -1).contiguous()
+    ref = F.scaled_dot_product_attention(torch.from_numpy(q[0, 0, :N])[None, None],
+                                         torch.from_numpy(k[0, 0, cols])[None, None],
+                                         torch.from_numpy(v[0, 0, cols])[None, None],
+                                         attn_mask=bias[None, None], scale=1 / math.sqrt(d))[0, 0].numpy()
+    assert np.allclose(O[0, 0, :N], ref, rtol=1e-12, atol=1e-12)
+    O1, _ = oracle.fine_attention(q, k, v, off, idx, np.full(idx.size, 2.5), N)
+    O0, _ = oracle.fine_attention(q, k, v, off, idx, None, N)
+    assert np.allclose(O1, O0, atol=1e-13)
+    # weight 3 on block idx[0] == that block listed three times with weight 1
+    w3 = np.ones(idx.size)
+    w3[0] = 3.0
+    O3, _ = oracle.fine_attention(q, k, v, off, idx, w3, N)
+    idx_rep = np.concatenate([[idx[0], idx[0]], idx])
+    Orep, _ = oracle.fine_attention(q, k, v, np.array([0, idx_rep.size]), idx_rep, None, N)
+    assert np.allclose(O3, Orep, atol=1e-13)
+
+
+def test_pins_catch_weights_applied_to_the_numerator_only(monkeypatch):
+    orig = nabla.fine_attention
+
+    def bad(q, k, v, off, idx, w, N, qblock=128, kblock=4, scale=None):
+        O, lse = orig(q, k, v, off, idx, None, N, qblock, kblock, scale)
+        if w is None:
+            return O, lse
+        return O * float(np.mean(w)), lse
+    monkeypatch.setattr(oracle, "fine_attention", bad)
+    with pytest.raises(AssertionError):
+        test_fine_attention_weights_against_library_attention()
+
+
 def test_lists_roundtrip():
     rng = np.random.default_rng(9)
     keep = rng.random((2, 3, 7, 7)) < 0.4
