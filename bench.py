@@ -39,6 +39,9 @@ sys.path.insert(0, ROOT)
 
 METRIC = "block-sparse attn fwd ms & effective TFLOPS (% bf16 peak), Wan-480p shape"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# Fine-selection timing: fraction of the 4-token KV blocks each query block
+# keeps (the budget the AB-Attention article quotes for ideal top-k, 10.8 %).
+FINE_FRAC = 0.108
 
 
 def kernel_launches_per_step(w) -> int:
@@ -467,6 +470,47 @@ def run_ours(args, w, rank, world, dist):
         torch.cuda.synchronize()
         bwd_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in bt) / args.steps, dist, dev)
         bwd = {"ms": bwd_ms, "flops": 2.5 * flops_step}
+    # ---- fine-grained KV selection (not part of `value`): K calls of
+    # bsa_attn_fwd_fine on the same Q, K, V (kernel order) with lists of
+    # 4-token blocks covering 10.8 % of the keys per 128-row query block,
+    # weighted, L2 flushed between calls
+    fine = None
+    if args.fine and not args.baseline_kernel:
+        fshape = bsa.make_shape(w.B, w.T, w.H, w.W, w.heads, w.d, 128, w.patch)
+        fNpad = bsa.padded_len(fshape)
+        nq, nkb = fNpad // 128, -(-w.N // 4)
+        fq, fk, fv = (torch.zeros(w.B, w.heads, fNpad, w.d, dtype=torch.bfloat16, device=dev) for _ in range(3))
+        for dst, src_t in ((fq, plan.q), (fk, plan.k), (fv, plan.v)):
+            dst[:, :, :w.N].copy_(src_t[:, :, :w.N])
+        off, idx, wt = synth.random_fine_lists(w.B, w.heads, nq, nkb, FINE_FRAC, w.seed + 1000 * rank)
+        keys = torch.clamp(w.N - 4 * idx.to(torch.int64), max=4)
+        rows_valid = torch.clamp(w.N - 128 * (torch.arange(off.numel() - 1) % nq), max=128)
+        per_row = torch.zeros(off.numel() - 1, dtype=torch.int64)
+        per_row.index_add_(0, torch.repeat_interleave(torch.arange(off.numel() - 1), off[1:] - off[:-1]), keys)
+        fine_flops = 4.0 * w.d * float((per_row * rows_valid).sum())
+        offd, idxd, wtd = off.to(dev), idx.to(dev), wt.to(dev)
+        fo = torch.empty_like(fq)
+        flse = torch.empty(w.B, w.heads, fNpad, dtype=torch.float32, device=dev)
+        fws = torch.zeros(bsa.attn_fine_workspace_bytes(fshape), dtype=torch.uint8, device=dev)
+        run_fine = lambda: bsa.attn_fwd_fine(fshape, fq, fk, fv, offd, idxd, wtd, 0.0, fo, flse, fws)
+        for _ in range(args.warmup):
+            run_fine()
+        torch.cuda.synchronize()
+        if bsa.check_device_status(fws) != 0:
+            raise RuntimeError("device status not OK after the fine-selection warm-up")
+        ft = []
+        for _ in range(args.steps):
+            flush.fill_(1)
+            f0, f1 = ev(), ev()
+            f0.record(stream)
+            run_fine()
+            f1.record(stream)
+            ft.append((f0, f1))
+        torch.cuda.synchronize()
+        if bsa.check_device_status(fws) != 0:
+            raise RuntimeError("device status not OK after the fine-selection calls")
+        fine_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ft) / args.steps, dist, dev)
+        fine = {"ms": fine_ms, "flops": fine_flops, "entries_per_block": int(off[1] - off[0]), "nkb": nkb}
     if rank != 0:
         return
     peaks, src = load_peaks()
@@ -543,6 +587,13 @@ def run_ours(args, w, rank, world, dist):
                                  "flops": "2.5 x the forward's effective FLOPs (the five products of the "
                                           "definition per kept tile pair)",
                                  "launches_per_call": 3 + (4 if w.block == 64 else 2) + 2}
+    if fine is not None:
+        ft_tf = fine["flops"] / (fine["ms"] * 1e-3) / 1e12
+        line["config"]["fine"] = {"ms": fine["ms"], "tflops": ft_tf, "pct_bf16_peak": 100.0 * ft_tf / peak_tf,
+                                  "query_block": 128, "key_block": 4, "key_frac": FINE_FRAC,
+                                  "entries_per_block": fine["entries_per_block"], "weighted": True,
+                                  "flops": "4 d x valid query rows x valid selected keys",
+                                  "launches_per_call": 1}
     print(json.dumps(line), flush=True)
 
 
@@ -556,6 +607,7 @@ def main(argv=None):
     ap.add_argument("--density", type=float, default=None, help="density-sweep workload: kept fraction")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-bwd", dest="bwd", action="store_false", help="skip the backward-pass timing")
+    ap.add_argument("--no-fine", dest="fine", action="store_false", help="skip the fine-selection timing")
     ap.add_argument("--baseline-kernel", action="store_true",
                     help="time the legacy mma.sync attention kernel instead of the tcgen05 one")
     ap.add_argument("--cpu-budget", type=float, default=15.0)

@@ -73,6 +73,8 @@ def _load() -> ctypes.CDLL:
                                                P]),
         "bsa_attn_bwd_workspace_bytes": (ctypes.c_size_t, [S]),
         "bsa_attn_bwd": (st, [S, P, P, P, P, P, P, P, P, ctypes.c_float, P, P, P, P, ctypes.c_size_t, P]),
+        "bsa_attn_fine_workspace_bytes": (ctypes.c_size_t, [S]),
+        "bsa_attn_fwd_fine": (st, [S, P, P, P, P, P, P, ctypes.c_int64, ctypes.c_float, P, P, P, ctypes.c_size_t, P]),
         "bsa_check_device_status": (st, [P, P]),
         "bsa_status_string": (ctypes.c_char_p, [st]),
     }
@@ -271,6 +273,27 @@ def attn_bwd(s: Shape, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: tor
                                   _ptr(kv_count), _ptr(kv_idx), float(scale), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
                                   ws.numel() * ws.element_size(), _stream(q.device)),
            "bsa_attn_bwd")
+
+
+def attn_fine_workspace_bytes(s: Shape) -> int:
+    return get_lib().bsa_attn_fine_workspace_bytes(ctypes.byref(s))
+
+
+def attn_fwd_fine(s: Shape, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, sel_offsets: torch.Tensor,
+                  sel_idx: torch.Tensor, sel_w: Optional[torch.Tensor], scale: float, o: torch.Tensor,
+                  lse: Optional[torch.Tensor], ws: torch.Tensor) -> None:
+    """Attention over per-query-block lists of 4-token KV blocks (int64 CSR
+    offsets, int32 block indices, optional float32 inclusion weights)."""
+    if sel_offsets.dtype != torch.int64 or sel_idx.dtype != torch.int32:
+        raise TypeError("sel_offsets must be int64 and sel_idx int32")
+    if sel_w is not None and (sel_w.dtype != torch.float32 or sel_w.numel() != sel_idx.numel()):
+        raise TypeError("sel_w must be float32 with one weight per entry")
+    n_sel = sel_idx.numel()
+    _check(get_lib().bsa_attn_fwd_fine(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(sel_offsets),
+                                       _ptr(sel_idx) if n_sel else None, _ptr(sel_w) if n_sel else None, n_sel,
+                                       float(scale), _ptr(o), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(),
+                                       _stream(q.device)),
+           "bsa_attn_fwd_fine")
 
 
 def check_device_status(ws: torch.Tensor) -> int:

@@ -553,13 +553,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kernel(
   }
 }
 
-int num_sms() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
-  return n;
-}
-
 template <int D, int BS, bool DKDV>
 cudaError_t launch_pass(const Dims& g, const void* fix0, const void* fix1, const void* tile0, const void* tile1,
                         const int32_t* l_count, const int32_t* l_idx, const int2* items, int* work,

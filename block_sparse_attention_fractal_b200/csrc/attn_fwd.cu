@@ -640,20 +640,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   }
 }
 
-// BSA_TEST_FORCE_TIMEOUT=1 in the environment makes the attention kernel take
-// its bounded-wait failure path (tests of the device error word).
-int force_timeout_requested() {
-  const char* v = std::getenv("BSA_TEST_FORCE_TIMEOUT");
-  return (v != nullptr && v[0] == '1') ? 1 : 0;
-}
-
-int num_sms() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
-  return n;
-}
-
 template <int D, int BS, int MODE>
 cudaError_t launch_fwd(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
                        const int32_t* kv_idx, const int2* items, int* work, float scale, void* o, float* lse,
@@ -690,6 +676,18 @@ cudaError_t launch_fwd_mode(const Dims& g, const void* q, const void* k, const v
 }
 
 }  // namespace
+
+int force_timeout_requested() {
+  const char* v = std::getenv("BSA_TEST_FORCE_TIMEOUT");
+  return (v != nullptr && v[0] == '1') ? 1 : 0;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
 
 cudaError_t launch_attn(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
                         const int32_t* kv_idx, const int2* items, int* work, float scale, void* o, float* lse,

@@ -439,6 +439,36 @@ bsa_status bsa_build_block_mask_subblock(const bsa_shape* s, const void* q_bhnd,
                                              workspace, bsa::next_launch_seq(), (cudaStream_t)stream));
 }
 
+size_t bsa_attn_fine_workspace_bytes(const bsa_shape* s) {
+  Dims g;
+  if (check_shape(s, &g) != BSA_OK || g.bs != 128) return 0;
+  return sizeof(Ctrl) + 256;
+}
+
+bsa_status bsa_attn_fwd_fine(const bsa_shape* s, const void* q, const void* k, const void* v,
+                             const int64_t* sel_offsets, const int32_t* sel_idx, const float* sel_w_or_null,
+                             int64_t n_sel, float scale, void* o, float* lse_or_null, void* workspace,
+                             size_t ws_bytes, bsa_stream_t stream) {
+  Dims g;
+  bsa_status st = check_shape(s, &g);
+  if (st != BSA_OK) return st;
+  if (g.bs != 128) return BSA_ERR_UNSUPPORTED;
+  const void* ptrs[6] = {q, k, v, o, sel_offsets, workspace};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return BSA_ERR_INVALID_ARG;
+  if (n_sel < 0 || (n_sel > 0 && sel_idx == nullptr)) return BSA_ERR_INVALID_ARG;
+  if ((sel_idx != nullptr && ((uintptr_t)sel_idx & 3u)) || (sel_w_or_null != nullptr && ((uintptr_t)sel_w_or_null & 3u)))
+    return BSA_ERR_INVALID_ARG;
+  if (lse_or_null != nullptr && !aligned16(lse_or_null)) return BSA_ERR_INVALID_ARG;
+  if (ws_bytes < sizeof(Ctrl) + 256) return BSA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || scale < 0.0f) return BSA_ERR_INVALID_ARG;
+  if (scale == 0.0f) scale = (float)(1.0 / std::sqrt((double)g.d));
+  int* work = (int*)((char*)workspace + sizeof(Ctrl));
+  return from_cuda(bsa::launch_attn_fine(g, q, k, v, sel_offsets, sel_idx, sel_w_or_null, n_sel, scale, o,
+                                         lse_or_null, (Ctrl*)workspace, work, bsa::next_launch_seq(),
+                                         (cudaStream_t)stream));
+}
+
 bsa_status bsa_check_device_status(void* workspace, bsa_stream_t stream) {
   if (workspace == nullptr || !aligned16(workspace)) return BSA_ERR_INVALID_ARG;
   cudaStream_t cs = (cudaStream_t)stream;
@@ -450,7 +480,7 @@ bsa_status bsa_check_device_status(void* workspace, bsa_stream_t stream) {
   }
   if (word & bsa::kErrLayout) return BSA_ERR_CUDA;
   if (word & bsa::kErrTimeout) return BSA_ERR_TIMEOUT;
-  if (word & (bsa::kErrIndex | bsa::kErrCount)) return BSA_ERR_DEVICE_INDEX;
+  if (word & (bsa::kErrIndex | bsa::kErrCount | bsa::kErrWeight)) return BSA_ERR_DEVICE_INDEX;
   return BSA_OK;
 }
 

@@ -16,6 +16,7 @@ enum : uint32_t {
   kErrCount = 2u,    // a KV count outside [1, nb]
   kErrTimeout = 4u,  // a bounded wait expired
   kErrLayout = 8u,   // shared memory not aligned as the kernel's layout needs
+  kErrWeight = 16u,  // an inclusion weight that is not positive and finite
 };
 
 // Control block at the start of every workspace.

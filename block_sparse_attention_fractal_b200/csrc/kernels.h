@@ -11,6 +11,14 @@ namespace bsa {
 // with bounded waits compare it with Ctrl::abort_seq.
 uint32_t next_launch_seq();
 
+// Multiprocessors of the current device (148 when the query fails).
+int num_sms();
+
+// 1 when BSA_TEST_FORCE_TIMEOUT=1 is set in the environment: the tcgen05
+// attention kernels then take their bounded-wait failure path (tests of the
+// device error word).
+int force_timeout_requested();
+
 cudaError_t launch_reorder(const Dims& g, const void* x_bnhd, void* y_bhnd, cudaStream_t st);
 cudaError_t launch_inverse_reorder(const Dims& g, const void* y_bhnd, void* x_bnhd, cudaStream_t st);
 // Q and K reordered in one launch, their block means written on the way:
@@ -53,6 +61,13 @@ cudaError_t launch_plan(const Dims& g, const int32_t* kv_count, const int32_t* k
 cudaError_t launch_attn(const Dims& g, const void* q, const void* k, const void* v, const int32_t* kv_count,
                         const int32_t* kv_idx, const int2* items, int* work, float scale, void* o, float* lse,
                         float* ent, Ctrl* ctrl, uint32_t seq, cudaStream_t st);
+
+// Attention over per-query-block lists of 4-token KV blocks with optional
+// inclusion weights (attn_fine.cu); 128-row query blocks (g.bs == 128).
+// `work` is a device int the launch zeroes and uses as its work counter.
+cudaError_t launch_attn_fine(const Dims& g, const void* q, const void* k, const void* v, const int64_t* sel_offsets,
+                             const int32_t* sel_idx, const float* sel_w, int64_t n_sel, float scale, void* o,
+                             float* lse, Ctrl* ctrl, int* work, uint32_t seq, cudaStream_t st);
 
 // Hilbert-curve token order (order.cu): order[p] = the token at position p.
 // Scratch: the tokens' curve indices, a bitmap over the enclosing cube and

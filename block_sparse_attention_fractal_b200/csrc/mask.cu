@@ -23,6 +23,11 @@ namespace bsa {
 
 namespace {
 
+using sm100::cp_async16;
+using sm100::cp_async8;
+using sm100::cp_async_commit;
+using sm100::cp_async_wait;
+
 // ---------------------------------------------------------------- pooling
 
 constexpr int kPoolThreads = 256;
@@ -149,20 +154,6 @@ constexpr int kKC = 32;                       // head-dimension chunk
 constexpr int kAStride = kKC + 4;             // doubles per staged qbar row
 constexpr int kBStride = kScoreCols + 4;      // doubles per staged kbar row
 constexpr int kStageDoubles = kScoreRows * kAStride + kKC * kBStride;
-
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
-  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
-  const int n = valid ? 16 : 0;   // zero-fill when the source is outside the matrix
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(d), "l"(src), "r"(n) : "memory");
-}
-__device__ __forceinline__ void cp_async8(void* dst, const void* src, bool valid) {
-  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
-  const int n = valid ? 8 : 0;
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;\n" ::"r"(d), "l"(src), "r"(n) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
 
 template <int D>
 __global__ void __launch_bounds__(kScoreThreads) scores_kernel(const double* __restrict__ qbar,

@@ -22,6 +22,13 @@ measure on):
   ``k = max(1, round(rho * nb))`` blocks: the diagonal block I plus ``k - 1``
   others drawn uniformly without replacement.
 
+* Fine selections (AB-Attention): for every (b, head, query block of 128)
+  a list of ``k`` distinct 4-token KV blocks drawn uniformly without
+  replacement (``k = round(frac * nkb)``, or, for ragged lists, ``k`` drawn
+  uniformly from ``[0, 2 * round(frac * nkb)]``), in ascending order; the
+  weights are 1 for half of the entries (blocks always taken) and ``1 / pi``
+  with ``pi ~ U(0.05, 1)`` for the others.
+
 Random numbers come from ``torch.Generator`` (CPU, Mersenne twister) in fixed
 chunks of ``_CHUNK`` elements, each chunk seeded from (seed, stream, chunk
 index); chunks are drawn on a thread pool, so the values do not depend on the
@@ -170,3 +177,35 @@ def random_block_lists(B: int, heads: int, nb: int, density: float, seed: int):
     kv_idx[..., :k] = chosen.to(torch.int32)
     kv_count = torch.full((B, heads, nb), k, dtype=torch.int32)
     return kv_count, kv_idx
+
+
+def random_fine_lists(B: int, heads: int, nq: int, nkb: int, frac: float, seed: int, ragged: bool = False):
+    """Seeded fine selections as CSR lists.
+
+    Returns ``(sel_offsets [B*heads*nq + 1] int64, sel_idx [n_sel] int32,
+    sel_w [n_sel] float32)``: row r = (b*heads + h)*nq + I holds entries
+    ``sel_offsets[r] .. sel_offsets[r+1]`` (see the module docstring for the
+    draw).
+    """
+    rows = B * heads * nq
+    k0 = max(1, min(nkb, int(round(frac * nkb))))
+    g = torch.Generator().manual_seed(_mix(seed, 0xF1E5, int(round(frac * 1e6)), int(ragged)))
+    if ragged:
+        counts = torch.randint(0, min(nkb, 2 * k0) + 1, (rows,), generator=g)
+    else:
+        counts = torch.full((rows,), k0, dtype=torch.int64)
+    offsets = torch.zeros(rows + 1, dtype=torch.int64)
+    offsets[1:] = torch.cumsum(counts, 0)
+    idx = torch.empty(int(offsets[-1]), dtype=torch.int32)
+    step = max(1, (1 << 24) // max(1, nkb))          # rows per batch of draws
+    for r0 in range(0, rows, step):
+        r1 = min(rows, r0 + step)
+        order = torch.argsort(torch.rand(r1 - r0, nkb, generator=g), dim=1)
+        for r in range(r0, r1):
+            c = int(counts[r])
+            if c:
+                idx[int(offsets[r]):int(offsets[r]) + c] = torch.sort(order[r - r0, :c]).values.to(torch.int32)
+    always = torch.rand(idx.numel(), generator=g) < 0.5
+    pi = 0.05 + 0.95 * torch.rand(idx.numel(), generator=g)
+    w = torch.where(always, torch.ones_like(pi), 1.0 / pi).to(torch.float32)
+    return offsets, idx, w

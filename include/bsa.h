@@ -55,7 +55,7 @@ typedef enum bsa_status {
   BSA_ERR_INVALID_ARG = 1,   /* bad shape, pointer, alignment, threshold or workspace size   */
   BSA_ERR_UNSUPPORTED = 2,   /* valid but outside what the kernels implement (e.g. nb > max) */
   BSA_ERR_CUDA = 3,          /* a CUDA runtime call or kernel launch failed                   */
-  BSA_ERR_DEVICE_INDEX = 4,  /* device saw a KV index outside [0, nb) or a count outside [1, nb] */
+  BSA_ERR_DEVICE_INDEX = 4,  /* device saw an invalid list: index, count, offsets or weight   */
   BSA_ERR_TIMEOUT = 5        /* a bounded device-side wait expired                           */
 } bsa_status;
 
@@ -306,6 +306,50 @@ BSA_API bsa_status bsa_attn_bwd(const bsa_shape* s, const void* q, const void* k
                                 const void* dO, const float* lse, const int32_t* kv_count, const int32_t* kv_idx,
                                 float scale, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
                                 bsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Fine-grained KV selection (AB-Attention article, news.hamidun.com/es/news/
+ * 14960, "Los tres recursos de AB-Attention": the fine selection on coarse
+ * hardware, and SIP's inclusion-probability weights).
+ * ------------------------------------------------------------------------- */
+
+/* Bytes of device workspace bsa_attn_fwd_fine needs (a control block and a
+ * work counter); 0 for an invalid shape or one whose block is not 128. */
+BSA_API size_t bsa_attn_fine_workspace_bytes(const bsa_shape* s);
+
+/* Attention of each 128-row query block over its own list of KV blocks of 4
+ * tokens, each optionally weighted by the inverse w of its inclusion
+ * probability (the Horvitz-Thompson estimate of both the softmax numerator
+ * and its normalisation, as a logit shift ln w):
+ *   O[q] = sum_k w_b(k) exp(scale Q[q].K[k]) V[k] / sum_k w_b(k) exp(scale Q[q].K[k])
+ * over the valid keys k < N of the listed blocks b (block b holds keys
+ * 4b .. 4b + 3).  The chosen blocks are gathered by index into full 128-key
+ * tiles of the tcgen05 tensor cores; fp32 softmax and accumulation, bf16
+ * output.
+ *   s: shape with block = 128 (the query block); BSA_ERR_UNSUPPORTED otherwise.
+ *   q, k, v: device, [B, heads, Npad, d] bf16 (any token order: the lists
+ *       index rows of k and v as given).
+ *   sel_offsets: device, int64 [B * heads * Npad / 128 + 1], CSR offsets: the
+ *       list of query block I of (b, h) is entries sel_offsets[r] ..
+ *       sel_offsets[r + 1] - 1 of sel_idx, r = (b * heads + h) * (Npad / 128) + I.
+ *   sel_idx: device, int32 [n_sel], 4-token block indices in [0, ceil(N / 4)),
+ *       in any order (a repeated entry counts again); NULL when n_sel = 0.
+ *   sel_w_or_null: device, float32 [n_sel] positive finite weights, or NULL
+ *       (every weight 1: plain attention over the selected keys).
+ *   n_sel: entries of sel_idx (and sel_w).
+ *   scale: >= 0; 0 selects 1/sqrt(d).
+ *   o: device, [B, heads, Npad, d] bf16, written; rows >= N, and rows whose
+ *       list holds no valid key, are 0.
+ *   lse_or_null: device, [B, heads, Npad] float32 natural-log sum of
+ *       w exp(scale s) per row (0 where o is 0), or NULL.
+ *   workspace / ws_bytes: at least bsa_attn_fine_workspace_bytes(s).
+ * A list whose offsets decrease or leave [0, n_sel] is treated as empty, an
+ * index outside [0, ceil(N / 4)) and a weight that is not positive and finite
+ * are skipped; each sets the device error word (BSA_ERR_DEVICE_INDEX). */
+BSA_API bsa_status bsa_attn_fwd_fine(const bsa_shape* s, const void* q, const void* k, const void* v,
+                                     const int64_t* sel_offsets, const int32_t* sel_idx,
+                                     const float* sel_w_or_null, int64_t n_sel, float scale, void* o,
+                                     float* lse_or_null, void* workspace, size_t ws_bytes, bsa_stream_t stream);
 
 /* Same contract as bsa_attn_fwd, computed by the legacy warp-level
  * mma.sync tensor-core kernel instead of the tcgen05 one.  Kept as the measured

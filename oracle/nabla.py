@@ -506,28 +506,53 @@ def radius_mask_from_qk(q: np.ndarray, k: np.ndarray, T: int, H: int, W: int, P:
 
 # --------------------------------------------- fine-grained KV selection
 
+def fine_attention_block(qr: np.ndarray, kh: np.ndarray, vh: np.ndarray, idx: np.ndarray,
+                         w: Optional[np.ndarray], N: int, kblock: int = 4,
+                         scale: Optional[float] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """One query block of fine_attention: rows ``qr`` [n, d] of one head over
+    the keys of the 4-token blocks ``idx`` (weights ``w`` or None) of that
+    head's ``kh``, ``vh`` [Npad, d].  Returns (O [n, d], lse [n]); both zero
+    when the list holds no valid key."""
+    n, d = qr.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    cols, shift = [], []
+    for e, blk in enumerate(np.asarray(idx, dtype=np.int64)):
+        lw = 0.0 if w is None else math.log(float(w[e]))
+        for key in range(int(blk) * kblock, min((int(blk) + 1) * kblock, N)):
+            cols.append(key)
+            shift.append(lw)
+    if not cols:
+        return np.zeros((n, d)), np.zeros(n)
+    cols = np.asarray(cols, dtype=np.int64)
+    s = (qr @ kh[cols, :].T) * scale + np.asarray(shift)[None, :]
+    m = s.max(axis=1, keepdims=True)
+    e_ = np.exp(s - m)
+    z = e_.sum(axis=1, keepdims=True)
+    return (e_ @ vh[cols, :]) / z, (m + np.log(z))[:, 0]
+
+
 def fine_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, sel_offsets: np.ndarray, sel_idx: np.ndarray,
                    sel_w: Optional[np.ndarray], N: int, qblock: int = 128, kblock: int = 4,
                    scale: Optional[float] = None) -> Tuple[np.ndarray, np.ndarray]:
     """Attention over per-query-block lists of small KV blocks, with optional
     inclusion weights.
 
-    AB-Attention article, "la seleccion fina sobre hardware grueso": KV blocks
-    of only 4 tokens, chosen per query block (of 128 tokens) and gathered by
-    index; and SIP: each chosen block counts with the inverse of its inclusion
-    probability w (Horvitz-Thompson), as a logit shift ln w in both the
-    numerator and the normalisation of the softmax:
+    AB-Attention article, "Los tres recursos de AB-Attention": KV blocks of
+    only 4 tokens, chosen per query block (of 128 tokens) and gathered by
+    index (the fine selection on coarse hardware); and SIP: each chosen block
+    counts with the inverse of its inclusion probability w (Horvitz-Thompson),
+    as a logit shift ln w in both the numerator and the normalisation of the
+    softmax:
         O_q = sum_k w_b(k) e^(s_qk) v_k / sum_k w_b(k) e^(s_qk),  s = scale q.k
     over the valid keys k of the chosen blocks.  Lists are CSR: query block r
     of head (b, h) (r = (b * heads + h) * nq + I) uses entries
     sel_offsets[r] .. sel_offsets[r + 1] of sel_idx (block indices, 4-token
     units) and sel_w (None: all 1).  Returns (O, lse) like masked_attention
-    (lse includes the shifts).
+    (lse includes the shifts; rows >= N and rows with no valid key are 0).
     """
     B, heads, Npad, d = q.shape
     nq = Npad // qblock
-    if scale is None:
-        scale = 1.0 / math.sqrt(d)
     O = np.zeros_like(q, dtype=np.float64)
     lse = np.zeros((B, heads, Npad), dtype=np.float64)
     for b in range(B):
@@ -537,22 +562,10 @@ def fine_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, sel_offsets: np.
                 qlo, qhi = I * qblock, min((I + 1) * qblock, N)
                 if qhi <= qlo:
                     continue
-                cols, shift = [], []
-                for e in range(int(sel_offsets[r]), int(sel_offsets[r + 1])):
-                    blk = int(sel_idx[e])
-                    lw = 0.0 if sel_w is None else math.log(float(sel_w[e]))
-                    for key in range(blk * kblock, min((blk + 1) * kblock, N)):
-                        cols.append(key)
-                        shift.append(lw)
-                if not cols:
-                    continue
-                cols = np.asarray(cols, dtype=np.int64)
-                s = (q[b, h, qlo:qhi, :] @ k[b, h, cols, :].T) * scale + np.asarray(shift)[None, :]
-                m = s.max(axis=1, keepdims=True)
-                e_ = np.exp(s - m)
-                z = e_.sum(axis=1, keepdims=True)
-                O[b, h, qlo:qhi, :] = (e_ @ v[b, h, cols, :]) / z
-                lse[b, h, qlo:qhi] = (m + np.log(z))[:, 0]
+                lo, hi = int(sel_offsets[r]), int(sel_offsets[r + 1])
+                O[b, h, qlo:qhi], lse[b, h, qlo:qhi] = fine_attention_block(
+                    q[b, h, qlo:qhi], k[b, h], v[b, h], sel_idx[lo:hi], None if sel_w is None else sel_w[lo:hi],
+                    N, kblock, scale)
     return O, lse
 
 
