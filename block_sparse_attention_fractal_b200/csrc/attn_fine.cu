@@ -15,20 +15,25 @@
 //
 // Roles (384 threads, persistent, one CTA per SM, query blocks from a work
 // counter):
-//   warps 0 and 3  gather K: each thread copies 16-byte pieces of the tile's
-//                  rows with cp.async into the 128-byte swizzled layout the
-//                  MMA descriptors expect (zero-filled past the list's end and
-//                  for keys >= N), waits for its own copies, orders them for
-//                  the tensor core (proxy fence) and arrives on the stage's
-//                  barrier; lane 0 of warp 0 also loads Q by TMA
+//   warps 0 and 3  gather K into three stages: each thread copies 16-byte
+//                  pieces of the tile's rows with cp.async into the 128-byte
+//                  swizzled layout the MMA descriptors expect (zero-filled past
+//                  the list's end and for keys >= N).  It issues tile j's
+//                  copies before it waits for its own copies of tile j - 1,
+//                  so two tiles are in flight; once those have landed it
+//                  orders them for the tensor core (proxy fence) and arrives
+//                  on the stage's barrier.  Lane 0 of warp 0 also loads Q by TMA
 //   warp 2         gathers V the same way
 //   warp 1         issues the MMAs (one elected thread): S(0), S(1), then
 //                  O_w += P(j) V(j) and S(j + 2) into the same TMEM buffer,
 //                  as in the block-sparse kernel
 //   warps 4-11     softmax (two groups on alternating KV tiles) and epilogue;
-//                  each warp turns the tile's 32 entries into 128 column
-//                  shifts (log2 w, or -inf for a missing key) in its own
-//                  shared-memory row, loaded one tile ahead
+//                  the first warp of each group turns the tile's 32 entries
+//                  into 128 column shifts (log2 w, or -inf for a missing key)
+//                  in one of the group's two shared-memory slots, loaded one
+//                  tile ahead, and a named barrier of the group's 128 threads
+//                  (which also carries the group's abort verdict) hands them
+//                  to the other three warps
 // Every mbarrier wait is bounded, with the same abort and drain sequence as
 // the block-sparse kernel.
 #include <cmath>
@@ -56,10 +61,11 @@ constexpr int kKeyBlock = 4;       // tokens of a KV block
 constexpr int kEntries = 128 / kKeyBlock;   // list entries per 128-key tile (one per lane)
 constexpr int kKThreads = 64;      // K gather: warps 0 and 3
 constexpr int kVThreads = 32;      // V gather: warp 2
+constexpr uint32_t kStages = 3;    // K and V stages in shared memory
 
 struct Ctl {
   uint64_t q_full;
-  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
+  uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
   uint64_t s_full[2], p_full[2], pv_done[2];
   uint64_t drain;
   uint32_t tmem_base;
@@ -67,7 +73,9 @@ struct Ctl {
   int len;          // list entries of the current query block
   int abort;
   long long off;    // its first entry
-  alignas(16) float shift[8][128];   // per softmax warp: base-2 logit shift of each key column of its tile
+  // per softmax group, two slots (tiles j with (j / 2) mod 2 = 0, 1): base-2
+  // logit shift of each key column of the tile
+  alignas(16) float shift[2][2][128];
 };
 
 struct FineArgs {
@@ -120,6 +128,23 @@ __device__ __forceinline__ bool pair_sync(int q4, bool ok) {
   return r != 0u;
 }
 
+// Named barrier of the 128 threads of softmax group w; returns the AND of
+// `ok` over them (the group leaves its loop together).
+__device__ __forceinline__ bool group_sync(int w, bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n"
+      ".reg .pred p, q;\n"
+      "setp.ne.u32 q, %1, 0;\n"
+      "bar.red.and.pred p, %2, 128, q;\n"
+      "selp.u32 %0, 1, 0, p;\n"
+      "}\n"
+      : "=r"(r)
+      : "r"((uint32_t)ok), "r"(5 + w)
+      : "memory");
+  return r != 0u;
+}
+
 // List entry `lane` of KV tile j: its block index (-1 past the list's end or
 // when out of range, which is reported) and weight.
 __device__ __forceinline__ int entry_block(const FineArgs& a, long long off, int len, int j, int lane, bool report) {
@@ -147,7 +172,7 @@ __device__ __forceinline__ void gather_tile(uint32_t stage, const __nv_bfloat16*
   const int sub = t / PR, pc = t % PR;
   const uint32_t col = (uint32_t)(pc >> 3) * (128u * 128u);
   const uint32_t cc = (uint32_t)(pc & 7);
-#pragma unroll
+#pragma unroll 8
   for (int r0 = 0; r0 < 128; r0 += RS) {
     const int row = r0 + sub;
     const int blk = __shfl_sync(0xffffffffu, blk_lane, row >> 2);
@@ -171,9 +196,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fine_kernel(const __grid_con
     return;
   }
   uint8_t* sQ = smem_raw;
-  uint8_t* sK = sQ + kTile;            // two stages
-  uint8_t* sV = sQ + 3 * kTile;        // two stages
-  Ctl& c = *reinterpret_cast<Ctl*>(sQ + 5 * kTile);
+  uint8_t* sK = sQ + kTile;                     // kStages stages
+  uint8_t* sV = sK + kStages * kTile;           // kStages stages
+  Ctl& c = *reinterpret_cast<Ctl*>(sV + kStages * kTile);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -183,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fine_kernel(const __grid_con
 
   if (tid == 0) {
     mbar_init(&c.q_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (uint32_t s = 0; s < kStages; ++s) {
       mbar_init(&c.k_full[s], kKThreads);
       mbar_init(&c.k_empty[s], 1);
       mbar_init(&c.v_full[s], kVThreads);
@@ -254,22 +279,35 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fine_kernel(const __grid_con
       }
       const __nv_bfloat16* base = (is_k ? a.k : a.v) + (size_t)bh * a.Npad * D;
       const uint32_t s0 = smem_addr(is_k ? sK : sV);
+      uint64_t* full = is_k ? c.k_full : c.v_full;
+      uint64_t* empty = is_k ? c.k_empty : c.v_empty;
       int blk = (n_tiles > 0) ? entry_block(a, off, len, 0, lane, warp == 0) : -1;
+      int issued = 0;   // tiles of this item whose copies this thread has issued
       for (int j = 0; j < n_tiles; ++j) {
-        const uint32_t jg = jbase + j, s = jg & 1;
-        uint64_t* empty = is_k ? &c.k_empty[s] : &c.v_empty[s];
-        if (jg >= 2 && !wait_warp(empty, ((jg - 2) >> 1) & 1, ctrl, seq)) {
+        const uint32_t jg = jbase + j, s = jg % kStages;
+        if (jg >= kStages && !wait_warp(&empty[s], ((jg - kStages) / kStages) & 1, ctrl, seq)) {
           if (lane == 0) timeout(ctrl, c, seq, is_k ? 10 : 11);
           break;
         }
         if (is_k) gather_tile<D, kKThreads>(s0 + s * kTile, base, blk, (warp == 0 ? 0 : 32) + lane, a.N);
         else gather_tile<D, kVThreads>(s0 + s * kTile, base, blk, lane, a.N);
         cp_async_commit();
+        ++issued;
         // the next tile's entries, in flight while these copies land
         blk = (j + 1 < n_tiles) ? entry_block(a, off, len, j + 1, lane, warp == 0) : -1;
-        cp_async_wait<0>();
-        fence_proxy_async_smem();   // the copies, ordered before the tensor core reads them
-        mbar_arrive(is_k ? &c.k_full[s] : &c.v_full[s]);
+        if (j > 0) {
+          // tile j - 1 has landed once at most one group (tile j) is in flight
+          cp_async_wait<1>();
+          fence_proxy_async_smem();   // the copies, ordered before the tensor core reads them
+          mbar_arrive(&full[(jg - 1) % kStages]);
+        }
+      }
+      // the last tile issued; after a timeout only the wait (nothing may be
+      // left in flight when the item ends)
+      cp_async_wait<0>();
+      if (issued == n_tiles && n_tiles > 0) {
+        fence_proxy_async_smem();
+        mbar_arrive(&full[(jbase + n_tiles - 1) % kStages]);
       }
     } else if (warp == 1) {
       // ---------------------------------------------------------- MMA issuer
@@ -279,9 +317,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fine_kernel(const __grid_con
         const uint64_t dQ = smem_desc_sw128(smem_addr(sQ), 16, 1024);
         const uint32_t aK = smem_addr(sK), aV = smem_addr(sV);
         auto issue_s = [&](int jj) -> bool {
-          const uint32_t jg = jbase + jj, ks = jg & 1;
+          const uint32_t jg = jbase + jj, ks = jg % kStages;
           const int w = jj & 1;
-          if (!wait(&c.k_full[ks], (jg >> 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 21); return false; }
+          if (!wait(&c.k_full[ks], (jg / kStages) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 21); return false; }
           tc_fence_after();
           const uint64_t dK = smem_desc_sw128(aK + ks * kTile, 16, 1024);
 #pragma unroll
@@ -300,11 +338,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fine_kernel(const __grid_con
         }
         for (int jj = 0; go && jj < 2 && jj < n_tiles; ++jj) go = issue_s(jj);
         for (int j = 0; go && j < n_tiles; ++j) {
-          const uint32_t jg = jbase + j, vs = jg & 1;
+          const uint32_t jg = jbase + j, vs = jg % kStages;
           const int w = j & 1;
           const uint32_t gw = gbase[w] + (j >> 1);
           if (!wait(&c.p_full[w], gw & 1, ctrl, seq)) { timeout(ctrl, c, seq, 23); break; }
-          if (!wait(&c.v_full[vs], (jg >> 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 24); break; }
+          if (!wait(&c.v_full[vs], (jg / kStages) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 24); break; }
           tc_fence_after();
           const uint64_t dV = smem_desc_sw128(aV + vs * kTile, kChunk, 1024);
           const uint32_t acc0 = (j >= 2) ? 1u : 0u;
@@ -324,8 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fine_kernel(const __grid_con
       const int r = q4 * 32 + lane;
       const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16);
       const uint32_t tS = trow + 128 * w, tOw = trow + kTmemO + 128 * w;
-      float* shw = c.shift[warp - kSoftmaxWarp0];
-      const float4* shw4 = reinterpret_cast<const float4*>(shw);
+      const bool writer = q4 == 0;   // the group's first warp writes its shifts
       float m = -INFINITY;
       float l = 0.f, lx = 0.f;
       bool ok = true;
@@ -334,15 +371,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fine_kernel(const __grid_con
       // tile ahead
       int blk = -1;
       float wt = 1.f;
-      if (w < n_tiles) {
+      if (writer && w < n_tiles) {
         blk = entry_block(a, off, len, w, lane, false);
         if (a.sel_w != nullptr && w * kEntries + lane < len) wt = __ldg(a.sel_w + off + w * kEntries + lane);
       }
       for (int j = w; j < n_tiles; j += 2, ++mine) {
         const uint32_t gw = gbase[w] + (j >> 1);
-        // column shifts of tile j: log2 w for the block's valid keys, -inf
-        // for keys >= N, missing entries and invalid weights (reported once)
-        {
+        float* shs = c.shift[w][(j >> 1) & 1];
+        if (writer) {
+          // column shifts of tile j: log2 w for the block's valid keys, -inf
+          // for keys >= N, missing entries and invalid weights (reported).
+          // The slot was last read for tile j - 4, before the group barrier
+          // of tile j - 2.
           float sh = -INFINITY;
           int nv = 0;
           if (blk >= 0) {
@@ -352,14 +392,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fine_kernel(const __grid_con
             } else if (wt > 0.f && wt <= 3.0e38f) {
               sh = log2f(wt);
             } else {
-              if (warp == kSoftmaxWarp0 + 4 * w) report_error(ctrl, kErrWeight, (uint32_t)(off + j * kEntries + lane), __float_as_uint(wt), 42u);
+              report_error(ctrl, kErrWeight, (uint32_t)(off + j * kEntries + lane), __float_as_uint(wt), 42u);
               nv = 0;
             }
           }
-          __syncwarp();   // the previous tile's shifts have been read
-          reinterpret_cast<float4*>(shw)[lane] = make_float4(nv > 0 ? sh : -INFINITY, nv > 1 ? sh : -INFINITY,
+          reinterpret_cast<float4*>(shs)[lane] = make_float4(nv > 0 ? sh : -INFINITY, nv > 1 ? sh : -INFINITY,
                                                              nv > 2 ? sh : -INFINITY, nv > 3 ? sh : -INFINITY);
-          __syncwarp();
           const int jn = j + 2;
           blk = -1;
           wt = 1.f;
@@ -368,7 +406,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fine_kernel(const __grid_con
             if (a.sel_w != nullptr && jn * kEntries + lane < len) wt = __ldg(a.sel_w + off + jn * kEntries + lane);
           }
         }
-        if (!wait_warp(&c.s_full[w], gw & 1, ctrl, seq)) { timeout(ctrl, c, seq, 30); ok = false; break; }
+        // the shifts, visible to the whole group; a warp that timed out on
+        // the previous tile makes the whole group leave here
+        ok = group_sync(w, ok);
+        if (!ok) break;
+        const float4* shw4 = reinterpret_cast<const float4*>(shs);
+        if (!wait_warp(&c.s_full[w], gw & 1, ctrl, seq)) {
+          timeout(ctrl, c, seq, 30);
+          ok = false;
+          continue;   // to the next group barrier (or the end of the loop)
+        }
         tc_fence_after();
         // Pass 1: row max of y = s * scale_log2 + shift over the 128 columns.
         const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
@@ -538,8 +585,8 @@ template <int D, bool WITH_LSE>
 cudaError_t launch_fine_t(const FineArgs& a, const void* q, uint64_t bhs, cudaStream_t st) {
   CUtensorMap mq;
   if (!make_map_bf16_3d(&mq, q, D, (uint64_t)a.Npad, bhs, 64, 64)) return cudaErrorInvalidValue;
-  const size_t smem = 5u * 128u * D * 2u + sizeof(Ctl);
-  static_assert(5u * 128u * 128u * 2u + sizeof(Ctl) <= 227u * 1024u, "shared memory layout");
+  const size_t smem = (1u + 2u * kStages) * 128u * D * 2u + sizeof(Ctl);
+  static_assert((1u + 2u * kStages) * 128u * 128u * 2u + sizeof(Ctl) <= 227u * 1024u, "shared memory layout");
   cudaError_t e =
       cudaFuncSetAttribute(attn_fine_kernel<D, WITH_LSE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
