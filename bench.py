@@ -87,7 +87,8 @@ def recorded_traffic(kernel: str, workload: str):
 
 
 class ClockSampler:
-    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+    """Samples SM clocks and throttle reasons while running: NVML every 5 ms
+    (the counters nvidia-smi reports), else nvidia-smi -lms 50."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -99,6 +100,10 @@ class ClockSampler:
         self.lines = []
 
     def __enter__(self):
+        self.t0 = None
+        if self._start_nvml():
+            self.t0 = time.monotonic()
+            return self
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "50"],
@@ -112,6 +117,40 @@ class ClockSampler:
         self.t0 = time.monotonic()
         return self
 
+    def _start_nvml(self) -> bool:
+        """Polls NVML every 5 ms (the same counters nvidia-smi reads) in a
+        thread; False when NVML is not available."""
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            smax = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            return False
+        bits = {"hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
+                "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap}
+        self.stop = threading.Event()
+
+        def poll():
+            while not self.stop.is_set():
+                try:
+                    sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                    rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                except Exception:
+                    break
+                flags = ["Active" if rs & bits[k] else "Not Active" for k in
+                         ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")]
+                self.lines.append((time.monotonic(), ", ".join([str(self.index), str(sm), str(smax), "", hex(rs)]
+                                                               + flags)))
+                time.sleep(0.005)
+
+        self.thread = threading.Thread(target=poll, daemon=True)
+        self.thread.start()
+        self.nvml = True
+        return True
+
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append((time.monotonic(), line.strip()))
@@ -120,6 +159,10 @@ class ClockSampler:
 
     def __exit__(self, *exc):
         self.t1 = time.monotonic()
+        if getattr(self, "nvml", False):
+            self.stop.set()
+            self.thread.join(timeout=2)
+            return
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -149,6 +192,28 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+def plan_work_ratio(bsa, shape, w, plan) -> float:
+    """KV tiles the attention kernel runs (each tile 128 x 128) over the kept
+    (query block, key block) pairs, in pair units: 1 for 128-token blocks;
+    with 64-token blocks two query blocks share a tile and walk the union of
+    their lists."""
+    qb = 128 // w.block
+    per_bh = -(-plan.nb // qb)
+    off = bsa.plan_items_offset(shape)
+    n = w.B * w.heads * per_bh
+    items = plan.ws[off:off + 8 * n].view(torch.int32).view(n, 2).cpu().numpy()
+    keep = lists_to_keep(plan.kv_count.cpu().numpy(), plan.kv_idx.cpu().numpy(), plan.nb).reshape(-1, plan.nb,
+                                                                                                   plan.nb)
+    bh = np.arange(n) // per_bh
+    a = np.clip(items[:, 0], 0, plan.nb - 1)
+    rows = keep[bh, a]
+    if qb == 2:
+        second = items[:, 1] >= 0
+        rows = rows | (keep[bh, np.clip(items[:, 1], 0, plan.nb - 1)] & second[:, None])
+    tiles = -(-rows.sum(axis=1) // qb)
+    return float(tiles.sum() * qb * qb / keep.sum())
 
 
 def lists_to_keep(kv_count: np.ndarray, kv_idx: np.ndarray, nb: int) -> np.ndarray:
@@ -354,6 +419,7 @@ def run_ours(args, w, rank, world, dist):
     if plan.status() != 0:
         raise RuntimeError("device status not OK after warm-up")
     dens = float(plan.kv_count.sum().item()) / (w.B * w.heads * plan.nb * plan.nb)
+    work_ratio = plan_work_ratio(bsa, shape, w, plan)
     flops_step = 4.0 * w.N * w.N * w.d * w.heads * w.B * dens
 
     # ---- device-timed steps
@@ -551,6 +617,7 @@ def run_ours(args, w, rank, world, dist):
             "sta": list(w.sta) if w.sta else None, "density": dens, "parallelism": f"replicas x{world}",
             "attn_kernel": "mma.sync (legacy baseline)" if args.baseline_kernel else "tcgen05",
             "l2": "flushed between steps (write of a 2x L2 buffer, outside the step events)",
+            "plan_work_ratio": work_ratio,
             "attn_ms": attn_ms, "attn_tflops": attn_tf, "attn_pct_bf16_peak": 100.0 * attn_tf / peak_tf,
             "breakdown_ms": {"reorder_pool_qk": qk_ms, "mask": mask_ms, "wait_reorder_v": vjoin_ms, "attn": attn_ms,
                              "inverse_reorder": float(br[4])},

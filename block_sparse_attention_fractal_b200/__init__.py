@@ -18,7 +18,7 @@ from typing import Optional, Tuple
 import torch
 
 from ._lib import (BsaError, Shape, attn_bwd, attn_bwd_workspace_bytes, attn_fwd, attn_fwd_baseline,  # noqa: F401
-                   attn_fwd_fine, attn_fine_workspace_bytes,
+                   attn_fwd_fine, attn_fine_workspace_bytes, plan_items_offset,
                    build_block_mask, build_block_mask_pooled, build_block_mask_subblock, hilbert_order,
                    hilbert_workspace_bytes, inverse_reorder_perm, reorder_perm, reorder_qk_pooled_perm,
                    subblock_workspace_bytes, attn_fwd_entropy, dense_lists, build_block_mask_radius,
@@ -37,6 +37,7 @@ __all__ = ["BsaError", "Shape", "make_shape", "NablaAttention", "reorder", "inve
            "hilbert_order", "hilbert_workspace_bytes", "reorder_perm", "inverse_reorder_perm",
            "reorder_qk_pooled_perm", "build_block_mask_subblock", "subblock_workspace_bytes",
            "attn_fwd_entropy", "dense_lists", "build_block_mask_radius", "attn_fwd_fine", "attn_fine_workspace_bytes",
+           "plan_items_offset",
            "attn_fwd", "attn_fwd_baseline", "check_device_status", "workspace_bytes", "workspace_init", "padded_len", "num_blocks",
            "seq_len", "validate_shape", "get_lib", "LIB_PATH"]
 

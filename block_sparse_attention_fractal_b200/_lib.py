@@ -51,6 +51,7 @@ def _load() -> ctypes.CDLL:
         "bsa_num_blocks": (ctypes.c_int64, [S]),
         "bsa_workspace_bytes": (ctypes.c_size_t, [S]),
         "bsa_workspace_init": (st, [P, ctypes.c_size_t, P]),
+        "bsa_plan_items_offset": (ctypes.c_int64, [S]),
         "bsa_reorder": (st, [S, P, P, P]),
         "bsa_inverse_reorder": (st, [S, P, P, P]),
         "bsa_build_block_mask": (st, [S, P, P, ctypes.c_float, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
@@ -141,6 +142,11 @@ def num_blocks(s: Shape) -> int:
 
 def workspace_bytes(s: Shape) -> int:
     return get_lib().bsa_workspace_bytes(ctypes.byref(s))
+
+
+def plan_items_offset(s: Shape) -> int:
+    """Byte offset of the attention work plan (int2 per 128-row tile) in the workspace."""
+    return get_lib().bsa_plan_items_offset(ctypes.byref(s))
 
 
 def workspace_init(ws: torch.Tensor) -> None:

@@ -109,6 +109,11 @@ size_t bsa_workspace_bytes(const bsa_shape* s) {
   return check_shape(s, &g) == BSA_OK ? workspace_bytes(g) : 0;
 }
 
+int64_t bsa_plan_items_offset(const bsa_shape* s) {
+  Dims g;
+  return check_shape(s, &g) == BSA_OK ? (int64_t)plan_offset(g) : -1;
+}
+
 bsa_status bsa_workspace_init(void* workspace, size_t ws_bytes, bsa_stream_t stream) {
   if (workspace == nullptr || !aligned16(workspace) || ws_bytes < sizeof(Ctrl)) return BSA_ERR_INVALID_ARG;
   return from_cuda(cudaMemsetAsync(workspace, 0, sizeof(Ctrl), (cudaStream_t)stream));

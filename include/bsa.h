@@ -91,6 +91,14 @@ BSA_API int64_t bsa_num_blocks(const bsa_shape* s);
  * invalid shape. */
 BSA_API size_t bsa_workspace_bytes(const bsa_shape* s);
 
+/* Byte offset, inside the workspace, of the work plan that bsa_attn_fwd
+ * writes on every call (-1 for an invalid shape): one int2 per 128-row query
+ * tile of every (batch, head), [B * heads][ceil(nb * block / 128)], in
+ * launch order: the tile's first query block and its second (-1 when the tile
+ * holds one block; blocks of 128 always hold one).  Read-only diagnostics
+ * (e.g. the KV tiles a call runs: the union of each tile's lists). */
+BSA_API int64_t bsa_plan_items_offset(const bsa_shape* s);
+
 /* Clears the control block of a freshly allocated workspace (async memset).
  * Call once after allocation; bsa_check_device_status clears it again. */
 BSA_API bsa_status bsa_workspace_init(void* workspace, size_t ws_bytes, bsa_stream_t stream);
