@@ -494,25 +494,32 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           if (cch < 3) tmem_ld32(tS + 32 * (cch + 1), sc[(cch + 1) & 1]);
           const float* x = reinterpret_cast<const float*>(sc[cch & 1]);
           uint32_t pk[16];
-          if (lim[h] > 0) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              // both arguments in one fma.rn.f32x2 (half the issue slots)
-              const float2 yy = ffma2(make_float2(x[2 * i], x[2 * i + 1]), sc2, nm2);
-              const float y0 = yy.x, y1 = yy.y;
-              float2 p;
-              p.x = ex2f(y0);
-              p.y = ex2f(y1);
-              if (lim[h] < 64) {
-                const int kc = (cch & 1) * 32 + 2 * i;   // key within the half
-                p.x = (kc < lim[h]) ? p.x : 0.f;
-                p.y = (kc + 1 < lim[h]) ? p.y : 0.f;
-              }
-              pk[i] = pack_bf16(p.x, p.y);
-              rs[i & 1] = add_bf16x2(rs[i & 1], pk[i]);
-              if (WITH_LSE) rx += p.x + p.y;
-              if (WITH_ENT) ry = fmaf(p.x, y0, fmaf(p.y, y1, ry));
+          // valid keys of this chunk: all 32 (the common case, no per-key
+          // test in the loop), some, or none
+          const int kc0 = (cch & 1) * 32;
+          const int cl = min(32, max(0, lim[h] - kc0));
+          auto exp_pair = [&](int i, bool masked) {
+            // both arguments in one fma.rn.f32x2 (half the issue slots)
+            const float2 yy = ffma2(make_float2(x[2 * i], x[2 * i + 1]), sc2, nm2);
+            const float y0 = yy.x, y1 = yy.y;
+            float2 p;
+            p.x = ex2f(y0);
+            p.y = ex2f(y1);
+            if (masked) {
+              p.x = (2 * i < cl) ? p.x : 0.f;
+              p.y = (2 * i + 1 < cl) ? p.y : 0.f;
             }
+            pk[i] = pack_bf16(p.x, p.y);
+            rs[i & 1] = add_bf16x2(rs[i & 1], pk[i]);
+            if (WITH_LSE) rx += p.x + p.y;
+            if (WITH_ENT) ry = fmaf(p.x, y0, fmaf(p.y, y1, ry));
+          };
+          if (cl == 32) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) exp_pair(i, false);
+          } else if (cl > 0) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) exp_pair(i, true);
           } else {
 #pragma unroll
             for (int i = 0; i < 16; ++i) pk[i] = 0u;
