@@ -685,6 +685,57 @@ def test_pins_catch_a_radius_mask_without_temporal_decay(monkeypatch):
         test_radius_block_mask_by_brute_force(0.7, 1)
 
 
+def test_subblock_mask_with_whole_blocks_is_the_nabla_mask():
+    """Sub-blocks as large as the blocks: the sub-block mask is NABLA's block
+    mask (reduced map of the block means + CDF rule), reached by another route."""
+    rng = np.random.default_rng(16)
+    T, H, W, P, bs, d = 2, 6, 10, 4, 16, 8
+    N = T * H * W
+    Npad = nabla.padded_len(N, bs)
+    q = rng.standard_normal((1, 2, Npad, d)) * 1.5
+    k = rng.standard_normal((1, 2, Npad, d)) * 1.5
+    q[:, :, N:] = 0
+    k[:, :, N:] = 0
+    keep_sub, amb_sub = oracle.block_mask_subblock(q, k, N, bs, bs, 0.2)
+    keep_nabla, amb_nabla = oracle.block_mask(q, k, T, H, W, P, bs, 0.2)
+    assert np.array_equal(keep_sub, keep_nabla) and np.array_equal(amb_sub, amb_nabla)
+
+
+def test_radius_chain_against_library_entropy_and_brute_force():
+    """The whole chain on reordered Q, K: entropies from torch's categorical
+    entropy, radii from the closed form, the mask by brute force over the
+    original coordinates."""
+    rng = np.random.default_rng(23)
+    T, H, W, P, bs, d = 3, 5, 7, 4, 8, 8
+    N = T * H * W
+    Npad = nabla.padded_len(N, bs)
+    q = rng.standard_normal((1, 1, Npad, d)) * 1.5
+    k = rng.standard_normal((1, 1, Npad, d)) * 1.5
+    q[:, :, N:] = 0
+    k[:, :, N:] = 0
+    tau, gamma = 0.3, 0.6
+    got = oracle.radius_mask_from_qk(q, k, T, H, W, P, bs, tau, gamma, vote=2)[0, 0]
+    logits = torch.from_numpy(q[0, 0, :N] @ k[0, 0, :N].T / math.sqrt(d))
+    ent = torch.distributions.Categorical(logits=logits).entropy().numpy()   # per position
+    order = oracle.fractal_order(T, H, W, P)
+    r_tok = np.zeros(N)
+    for p_ in range(N):
+        n = order[p_]
+        t = n // (H * W)
+        budget = min(max(tau * math.exp(ent[p_]), 1.0), float(N))
+        area = math.pi * sum(math.exp(-2 * gamma * abs(tt - t)) for tt in range(T))
+        r_tok[n] = math.sqrt(budget / area)
+    assert np.array_equal(got, _radius_mask_brute(r_tok, T, H, W, P, bs, gamma, 2))
+
+
+def test_density_and_attention_flops_closed_forms():
+    keep = np.zeros((1, 2, 4, 4), dtype=bool)
+    keep[0, 0, :, 0] = True
+    keep[0, 1] = True
+    assert oracle.density(keep) == (4 + 16) / 32
+    assert oracle.attention_flops(1000, 64, 3, 2, 0.25) == 4.0 * 1000 * 1000 * 64 * 3 * 2 * 0.25
+
+
 # ----------------------------------------------- fine-grained KV selection
 
 def _fine_lists(keep_blocks, per):
@@ -739,6 +790,30 @@ def test_fine_attention_weights_against_library_attention():
     idx_rep = np.concatenate([[idx[0], idx[0]], idx])
     Orep, _ = oracle.fine_attention(q, k, v, np.array([0, idx_rep.size]), idx_rep, None, N)
     assert np.allclose(O3, Orep, atol=1e-13)
+
+
+def test_fine_attention_block_against_library_attention():
+    """One query block alone: rows of a head over the listed 4-token blocks
+    (one straddling N), weights as an additive log mask in torch SDPA."""
+    rng = np.random.default_rng(33)
+    N, d, n = 91, 16, 37
+    kh, vh = rng.standard_normal((96, d)), rng.standard_normal((96, d))
+    qr = rng.standard_normal((n, d))
+    idx = np.array([22, 3, 17, 9])          # block 22 holds keys 88-91: 91 is >= N
+    w = np.array([1.0, 4.0, 1.5, 2.0])
+    O, lse = oracle.fine_attention_block(qr, kh, vh, idx, w, N)
+    cols = np.array([c for b in idx for c in range(4 * b, min(4 * b + 4, N))])
+    wcol = np.array([w[e] for e, b in enumerate(idx) for c in range(4 * b, min(4 * b + 4, N))])
+    s = qr @ kh[cols].T / math.sqrt(d) + np.log(wcol)[None, :]
+    ref = F.scaled_dot_product_attention(torch.from_numpy(qr)[None, None], torch.from_numpy(kh[cols])[None, None],
+                                         torch.from_numpy(vh[cols])[None, None],
+                                         attn_mask=torch.from_numpy(np.log(wcol))[None, :].expand(n, -1)[None, None],
+                                         scale=1 / math.sqrt(d))[0, 0].numpy()
+    assert np.allclose(O, ref, rtol=1e-12, atol=1e-12)
+    assert np.allclose(lse, np.log(np.exp(s).sum(axis=1)), rtol=1e-12, atol=1e-12)
+    # an empty list: zeros
+    O0, lse0 = oracle.fine_attention_block(qr, kh, vh, np.array([], dtype=np.int64), None, N)
+    assert np.all(O0 == 0) and np.all(lse0 == 0)
 
 
 def test_pins_catch_weights_applied_to_the_numerator_only(monkeypatch):
