@@ -453,6 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kernel(
         if (!wait_warp(&c.sdp_full, jg & 1, ctrl, seq)) { timeout(ctrl, c, seq, 30); ok = false; break; }
         tc_fence_after();
         const float* rowL = sRow + s * 256;          // dkdv: L of the tile's 128 query columns, then D
+        const float2 sl2 = make_float2(scale_log2, scale_log2), nlg2 = make_float2(-kLog2e, -kLog2e);
         uint32_t sv[32], dv[32];
 #pragma unroll 1
         for (int cch = 0; cch < 4; ++cch) {
@@ -460,29 +461,41 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kernel(
           tmem_ld32(trow + kTS + 32 * cch, sv);
           tmem_ld32(trow + kTdP + 32 * cch, dv);
           tmem_wait_ld();
+          // valid columns of this chunk: all 32 (no per-column test in the
+          // loop, the common case), some, or none
+          const int cl = min(32, max(0, lim[h] - 32 * (cch & 1)));
           uint32_t pk[16], dk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float p2[2], d2[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int col = 32 * cch + 2 * i + e;            // column of the tile
-              const int kc = col & 63;                          // within its half
-              float l2, dd;
-              if (DKDV) {
-                l2 = rowL[col] * kLog2e;
-                dd = rowL[128 + col];
-              } else {
-                l2 = lse2;
-                dd = drow;
-              }
-              const float x = __uint_as_float(sv[2 * i + e]);
-              const float p = (kc < lim[h]) ? ex2f(fmaf(x, scale_log2, -l2)) : 0.f;
-              p2[e] = p;
-              d2[e] = p * (__uint_as_float(dv[2 * i + e]) - dd);
+          // one pair of columns: p = 2^(x scale log2 e - L log2 e),
+          // dS = p (dP - D), in packed two-lane arithmetic
+          auto pair = [&](int i, bool masked) {
+            const int col = 32 * cch + 2 * i;
+            float2 nl, dd;   // -L log2 e and D
+            if (DKDV) {
+              nl = fmul2(*reinterpret_cast<const float2*>(rowL + col), nlg2);
+              dd = *reinterpret_cast<const float2*>(rowL + 128 + col);
+            } else {
+              nl = make_float2(-lse2, -lse2);
+              dd = make_float2(drow, drow);
             }
-            pk[i] = pack_bf16(p2[0], p2[1]);
-            dk[i] = pack_bf16(d2[0], d2[1]);
+            const float2 y = ffma2(make_float2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), sl2, nl);
+            float2 p = make_float2(ex2f(y.x), ex2f(y.y));
+            if (masked) {
+              p.x = (2 * i < cl) ? p.x : 0.f;
+              p.y = (2 * i + 1 < cl) ? p.y : 0.f;
+            }
+            const float2 ds = fmul2(p, fsub2(make_float2(__uint_as_float(dv[2 * i]), __uint_as_float(dv[2 * i + 1])), dd));
+            pk[i] = pack_bf16(p.x, p.y);
+            dk[i] = pack_bf16(ds.x, ds.y);
+          };
+          if (cl == 32) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pair(i, false);
+          } else if (cl > 0) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pair(i, true);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[i] = dk[i] = 0u;
           }
           // bf16 operands over columns already read: P (dkdv only) over S,
           // dS over dP, two per 32-bit column
