@@ -454,13 +454,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kernel(
         tc_fence_after();
         const float* rowL = sRow + s * 256;          // dkdv: L of the tile's 128 query columns, then D
         const float2 sl2 = make_float2(scale_log2, scale_log2), nlg2 = make_float2(-kLog2e, -kLog2e);
-        uint32_t sv[32], dv[32];
-#pragma unroll 1
+        // two buffers: the next chunk's scores and dP load while this one is
+        // computed
+        uint32_t sv2[2][32], dv2[2][32];
+        tmem_ld32(trow + kTS, sv2[0]);
+        tmem_ld32(trow + kTdP, dv2[0]);
+#pragma unroll
         for (int cch = 0; cch < 4; ++cch) {
           const int h = cch >> 1;
-          tmem_ld32(trow + kTS + 32 * cch, sv);
-          tmem_ld32(trow + kTdP + 32 * cch, dv);
           tmem_wait_ld();
+          if (cch < 3) {
+            tmem_ld32(trow + kTS + 32 * (cch + 1), sv2[(cch + 1) & 1]);
+            tmem_ld32(trow + kTdP + 32 * (cch + 1), dv2[(cch + 1) & 1]);
+          }
+          const uint32_t* sv = sv2[cch & 1];
+          const uint32_t* dv = dv2[cch & 1];
           // valid columns of this chunk: all 32 (no per-column test in the
           // loop, the common case), some, or none
           const int cl = min(32, max(0, lim[h] - 32 * (cch & 1)));
