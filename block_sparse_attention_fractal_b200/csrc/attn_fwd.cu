@@ -117,6 +117,22 @@ __device__ __forceinline__ bool pair_sync(int q4, bool ok) {
   return r != 0u;
 }
 
+// O_w *= alpha for this thread's row, 32 columns at a time (warp-collective
+// TMEM accesses: every lane of the warp calls it).
+template <int D>
+__device__ __forceinline__ void rescale_o_cols(uint32_t tO, float alpha) {
+#pragma unroll 1
+  for (int cc = 0; cc < D; cc += 32) {
+    uint32_t ov[32];
+    tmem_ld32(tO + cc, ov);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+    tmem_st32(tO + cc, ov);
+  }
+  tmem_wait_st();
+}
+
 // MODE 0: O only; 1: O and the LSE; 2: O, the LSE and the entropy of each
 // row's attention distribution.
 template <int D, int BS, int MODE>
@@ -398,6 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       float vx = 0.f;
       bool ok = true;
       int mine = 0;   // KV tiles this group ran in this item
+      auto rescale_o = [&](uint32_t tO, float alpha) { rescale_o_cols<D>(tO, alpha); };
       for (int j = w; j < n_tiles; j += 2, ++mine) {
         const uint32_t gw = gbase[w] + (j >> 1);
         int lim[2];
@@ -418,60 +435,60 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         // previous P.V product, so O_w and the P columns are free as well
         if (!wait_warp(&c.s_full[w], gw & 1, ctrl, seq)) { timeout(ctrl, c, seq, 30); ok = false; break; }
         tc_fence_after();
-        // Pass 1: row max of the raw scores over the kept, real keys (scale > 0
-        // keeps the order), 64 columns at a time.
-        float mh[2];
+        // The row max is needed only to keep 2^(y - m) in range: bf16 P and
+        // the fp32 sums and accumulators hold weights far beyond 2^64.  So the
+        // max pass runs only while a row of the warp has no max yet (its
+        // first kept tile); later tiles use the running max as it stands and
+        // check each chunk's weights before storing them (below).
+        const bool need_max = __any_sync(0xffffffffu, m == -INFINITY);
+        if (need_max) {
+          // Pass 1: row max of the raw scores over the kept, real keys (scale
+          // > 0 keeps the order), 64 columns at a time.
+          float mh[2];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t sr[64];
-          tmem_ld32(tS + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-          tmem_ld32(tS + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-          tmem_wait_ld();
-          const float* xh = reinterpret_cast<const float*>(sr);
-          if (lim[h] == 64) {
-            float m0 = xh[0], m1 = xh[1], m2 = xh[2], m3 = xh[3];
-#pragma unroll
-            for (int i = 4; i < 64; i += 8) {
-              m0 = fmax3(m0, xh[i], xh[i + 1]);
-              m1 = fmax3(m1, xh[i + 2], xh[i + 3]);
-              m2 = fmax3(m2, xh[i + 4], xh[i + 5]);
-              m3 = fmax3(m3, xh[i + 6], xh[i + 7]);
-            }
-            mh[h] = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
-          } else {
-            float mm = -INFINITY;
-            if (lim[h] > 0) {
-#pragma unroll
-              for (int i = 0; i < 64; ++i) mm = (i < lim[h]) ? fmaxf(mm, xh[i]) : mm;
-            }
-            mh[h] = mm;
-          }
-        }
-        const float mnew = fmaxf(m, fmaxf(mh[0], mh[1]) * scale_log2);
-        // The running max moves only when it grows by more than 8 (a factor
-        // 256 in p), or when it is set for the first time.  The O rescale uses
-        // warp-collective TMEM accesses, so the whole warp takes it when any
-        // lane needs it (lanes whose max did not move use alpha = 1).  O_w is
-        // stable: its last P.V product has completed (waited above).
-        const bool grow = mnew > m + 8.0f;
-        if (__any_sync(0xffffffffu, grow && m != -INFINITY)) {
-          const float alpha = (grow && m != -INFINITY) ? ex2f(m - mnew) : 1.0f;
-#pragma unroll 1
-          for (int cc = 0; cc < D; cc += 32) {
-            uint32_t ov[32];
-            tmem_ld32(tOw + cc, ov);
+          for (int h = 0; h < 2; ++h) {
+            uint32_t sr[64];
+            tmem_ld32(tS + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+            tmem_ld32(tS + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
             tmem_wait_ld();
+            const float* xh = reinterpret_cast<const float*>(sr);
+            if (lim[h] == 64) {
+              float m0 = xh[0], m1 = xh[1], m2 = xh[2], m3 = xh[3];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-            tmem_st32(tOw + cc, ov);
+              for (int i = 4; i < 64; i += 8) {
+                m0 = fmax3(m0, xh[i], xh[i + 1]);
+                m1 = fmax3(m1, xh[i + 2], xh[i + 3]);
+                m2 = fmax3(m2, xh[i + 4], xh[i + 5]);
+                m3 = fmax3(m3, xh[i + 6], xh[i + 7]);
+              }
+              mh[h] = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+            } else {
+              float mm = -INFINITY;
+              if (lim[h] > 0) {
+#pragma unroll
+                for (int i = 0; i < 64; ++i) mm = (i < lim[h]) ? fmaxf(mm, xh[i]) : mm;
+              }
+              mh[h] = mm;
+            }
           }
-          tmem_wait_st();
-          if (WITH_ENT && grow && m != -INFINITY) vx = alpha * (vx + (m - mnew) * lx);
-          l *= alpha;
-          lx *= alpha;
+          const float mnew = fmaxf(m, fmaxf(mh[0], mh[1]) * scale_log2);
+          // The running max moves only when it grows by more than 8 (a factor
+          // 256 in p), or when it is set for the first time.  The O rescale
+          // uses warp-collective TMEM accesses, so the whole warp takes it
+          // when any lane needs it (lanes whose max did not move use alpha =
+          // 1).  O_w is stable: its last P.V product has completed (waited
+          // above).
+          const bool grow = mnew > m + 8.0f;
+          if (__any_sync(0xffffffffu, grow && m != -INFINITY)) {
+            const float alpha = (grow && m != -INFINITY) ? ex2f(m - mnew) : 1.0f;
+            rescale_o(tOw, alpha);
+            if (WITH_ENT && grow && m != -INFINITY) vx = alpha * (vx + (m - mnew) * lx);
+            l *= alpha;
+            lx *= alpha;
+          }
+          if (grow) m = mnew;
         }
-        if (grow) m = mnew;
-        const float nm = (m == -INFINITY) ? 0.f : -m;
+        float nm = (m == -INFINITY) ? 0.f : -m;
         // p = 2^(s * scale_log2 - m): one FFMA and one MUFU ex2 per score.  O is
         // normalised by the sum of the bf16-rounded weights the P.V product
         // uses (an exact convex combination of V rows up to accumulation
@@ -484,20 +501,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         // already read into registers.
         float rs[2] = {0.f, 0.f};
         float rx = 0.f, ry = 0.f;
-        const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(nm, nm);
-        uint32_t sc[2][32];
-        tmem_ld32(tS, sc[0]);
-#pragma unroll
-        for (int cch = 0; cch < 4; ++cch) {
-          const int h = cch >> 1;
-          tmem_wait_ld();
-          if (cch < 3) tmem_ld32(tS + 32 * (cch + 1), sc[(cch + 1) & 1]);
-          const float* x = reinterpret_cast<const float*>(sc[cch & 1]);
-          uint32_t pk[16];
-          // valid keys of this chunk: all 32 (the common case, no per-key
-          // test in the loop), some, or none
-          const int kc0 = (cch & 1) * 32;
-          const int cl = min(32, max(0, lim[h] - kc0));
+        float rx_ok = 0.f, ry_ok = 0.f;   // the LSE and entropy sums of the chunks stored so far
+        const float2 sc2 = make_float2(scale_log2, scale_log2);
+        // one chunk's weights from its scores x: pk, and the sums
+        auto exp_chunk = [&](const float* x, int cl, float nmv, uint32_t (&pk)[16]) {
+          const float2 nm2 = make_float2(nmv, nmv);
           auto exp_pair = [&](int i, bool masked) {
             // both arguments in one fma.rn.f32x2 (half the issue slots)
             const float2 yy = ffma2(make_float2(x[2 * i], x[2 * i + 1]), sc2, nm2);
@@ -514,6 +522,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             if (WITH_LSE) rx += p.x + p.y;
             if (WITH_ENT) ry = fmaf(p.x, y0, fmaf(p.y, y1, ry));
           };
+          // valid keys of the chunk: all 32 (the common case, no per-key
+          // test in the loop), some, or none
           if (cl == 32) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) exp_pair(i, false);
@@ -524,7 +534,78 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 #pragma unroll
             for (int i = 0; i < 16; ++i) pk[i] = 0u;
           }
+        };
+        int c_fail = 4;
+        uint32_t sc[2][32];
+        tmem_ld32(tS, sc[0]);
+#pragma unroll
+        for (int cch = 0; cch < 4; ++cch) {
+          const int h = cch >> 1;
+          tmem_wait_ld();
+          if (cch < 3) tmem_ld32(tS + 32 * (cch + 1), sc[(cch + 1) & 1]);
+          uint32_t pk[16];
+          exp_chunk(reinterpret_cast<const float*>(sc[cch & 1]), min(32, max(0, lim[h] - (cch & 1) * 32)), nm, pk);
+          // Without the max pass, a weight of 2^64 or more means this tile's
+          // scores exceed the running max by 64 or more: nothing of this
+          // chunk is stored, and the tile goes on below with a new max.
+          if (!need_max && __any_sync(0xffffffffu, !(rs[0] + rs[1] < 0x1p64f))) {
+            c_fail = cch;
+            break;
+          }
           tmem_st16(tS + 16 * cch, pk);
+          rx_ok = rx;
+          ry_ok = ry;
+        }
+        if (c_fail < 4) {
+          // Rare: the running max moves by 64 or more within a tile.  The new
+          // max comes from the scores of chunks c_fail..3 (columns the P
+          // stores have not reached); O, the row sums and the weights of the
+          // chunks already stored are rescaled by alpha = 2^(m - m_new) (the
+          // stored bf16 weights re-rounded, their sum recomputed from them);
+          // chunks c_fail..3 are then redone with the new max.
+          tmem_wait_ld();                     // the prefetch in flight
+          float mx = -INFINITY;
+#pragma unroll 1
+          for (int cc = c_fail; cc < 4; ++cc) {
+            uint32_t t[32];
+            tmem_ld32(tS + 32 * cc, t);
+            tmem_wait_ld();
+            const int cl = min(32, max(0, lim[cc >> 1] - (cc & 1) * 32));
+#pragma unroll
+            for (int i = 0; i < 32; ++i) mx = (i < cl) ? fmaxf(mx, __uint_as_float(t[i])) : mx;
+          }
+          const float mnew = fmaxf(m, mx * scale_log2);
+          const float alpha = ex2f(m - mnew);   // m is finite here: the max pass ran on an earlier tile
+          rescale_o(tOw, alpha);
+          if (WITH_ENT) vx = alpha * (vx + (m - mnew) * lx);
+          l *= alpha;
+          lx *= alpha;
+          rs[0] = rs[1] = 0.f;
+#pragma unroll 1
+          for (int cc = 0; cc < c_fail; ++cc) {
+            uint32_t pv[16];
+            tmem_ld16(tS + 16 * cc, pv);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              pv[i] = pack_bf16(__uint_as_float(pv[i] << 16) * alpha, __uint_as_float(pv[i] & 0xFFFF0000u) * alpha);
+              rs[i & 1] = add_bf16x2(rs[i & 1], pv[i]);
+            }
+            tmem_st16(tS + 16 * cc, pv);
+          }
+          if (WITH_ENT) ry = alpha * (ry_ok + (m - mnew) * rx_ok);
+          rx = alpha * rx_ok;
+          m = mnew;
+          nm = -m;
+#pragma unroll 1
+          for (int cc = c_fail; cc < 4; ++cc) {
+            uint32_t t[32];
+            tmem_ld32(tS + 32 * cc, t);
+            tmem_wait_ld();
+            uint32_t pk[16];
+            exp_chunk(reinterpret_cast<const float*>(t), min(32, max(0, lim[cc >> 1] - (cc & 1) * 32)), nm, pk);
+            tmem_st16(tS + 16 * cc, pk);
+          }
         }
         l += rs[0] + rs[1];
         if (WITH_LSE) lx += rx;

@@ -367,3 +367,49 @@ def test_running_max_growth_rescales(bsa, w):
         assert np.abs(got - want).mean() <= MEAN_ABS, dens
         lse = to64(plan.lse)[:, :, :w.N]
         assert np.abs(lse - lse_ref[:, :, :w.N]).max() <= LSE_ABS * max(1.0, np.abs(lse_ref).max() / 16.0), dens
+
+
+@pytest.mark.parametrize("w", GROWTH, ids=lambda w: w.name)
+def test_running_max_jump_past_the_unchecked_range(bsa, w):
+    """After a row's first kept tile the kernel skips the max pass and checks
+    each 32-key chunk's weights instead; scores that exceed the running max by
+    64 or more (log2 units) make the warp redo the tile from that chunk with a
+    new max, rescaling O, the sums and the weights already stored.  Keys
+    scaled up steeply along the blocks force that path on most rows: O, LSE and
+    (dense lists, the warm-up pass) the entropy against the oracle."""
+    q, k, v = synth.make_qkv(w)
+    plan = bsa.NablaAttention(_shape(bsa, w), with_lse=True)
+    for src, dst in ((q, plan.q), (k, plan.k), (v, plan.v)):
+        bsa.reorder(plan.shape, src.cuda(), dst)
+    nb = plan.nb
+    blk = torch.arange(plan.k.shape[2], device=plan.k.device) // w.block
+    ramp = 1.0 + 40.0 * (blk.float() / nb) ** 2
+    plan.k.copy_((plan.k.float() * ramp[None, None, :, None]).to(torch.bfloat16))
+    q64, k64, v64 = to64(plan.q), to64(plan.k), to64(plan.v)
+    s = np.einsum("bhnd,bhmd->bhnm", q64[:, :, :w.N], k64[:, :, :w.N]) / math.sqrt(w.d) / math.log(2.0)
+    first = s[..., :2 * w.block].max(axis=-1)
+    assert np.mean(s.max(axis=-1) - first > 64.0) > 0.2
+    cnt, idx = synth.random_block_lists(w.B, w.heads, nb, 1.0, seed=9)
+    plan.kv_count.copy_(cnt)
+    plan.kv_idx.copy_(idx)
+    keep = lists_to_keep(cnt, idx, nb)
+    O_ref, lse_ref = oracle.masked_attention(q64, k64, v64, keep, w.N, w.block)
+    want, lse_want = O_ref[:, :, :w.N], lse_ref[:, :, :w.N]
+    lse_tol = LSE_ABS * max(1.0, np.abs(lse_want).max() / 16.0)
+    plan.attention_step()
+    torch.cuda.synchronize()
+    assert plan.status() == 0
+    got = to64(plan.o)[:, :, :w.N]
+    assert np.all(np.abs(got - want) <= MAX_ABS + _half_ulp_bf16(want))
+    assert np.abs(got - want).mean() <= MEAN_ABS
+    assert np.abs(to64(plan.lse)[:, :, :w.N] - lse_want).max() <= lse_tol
+    ent = torch.full_like(plan.lse, float("nan"))
+    bsa.attn_fwd_entropy(plan.shape, plan.q, plan.k, plan.v, plan.kv_count, plan.kv_idx, 0.0, plan.o, plan.lse, ent,
+                         plan.ws)
+    torch.cuda.synchronize()
+    assert plan.status() == 0
+    got = to64(plan.o)[:, :, :w.N]
+    assert np.all(np.abs(got - want) <= MAX_ABS + _half_ulp_bf16(want))
+    assert np.abs(to64(plan.lse)[:, :, :w.N] - lse_want).max() <= lse_tol
+    H_ref = oracle.attention_entropy(q64, k64, w.N)[:, :, :w.N]
+    assert np.abs(to64(ent)[:, :, :w.N] - H_ref).max() <= 2e-3
