@@ -417,33 +417,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fine_kernel(const __grid_con
           continue;   // to the next group barrier (or the end of the loop)
         }
         tc_fence_after();
-        // Pass 1: row max of y = s * scale_log2 + shift over the 128 columns.
         const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
-        float mh[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t sr[64];
-          tmem_ld32(tS + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-          tmem_ld32(tS + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-          tmem_wait_ld();
-          const float* xh = reinterpret_cast<const float*>(sr);
-          float m0 = -INFINITY, m1 = -INFINITY;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float4 s4 = shw4[16 * h + i];
-            const float2 ya = ffma2(make_float2(xh[4 * i], xh[4 * i + 1]), sc2, make_float2(s4.x, s4.y));
-            const float2 yb = ffma2(make_float2(xh[4 * i + 2], xh[4 * i + 3]), sc2, make_float2(s4.z, s4.w));
-            m0 = fmax3(m0, ya.x, ya.y);
-            m1 = fmax3(m1, yb.x, yb.y);
-          }
-          mh[h] = fmaxf(m0, m1);
-        }
-        const float mnew = fmaxf(m, fmaxf(mh[0], mh[1]));
-        // Lazy rescale, as in the block-sparse kernel: the running max moves
-        // only when it grows by more than 8 (or is set for the first time).
-        const bool grow = mnew > m + 8.0f;
-        if (__any_sync(0xffffffffu, grow && m != -INFINITY)) {
-          const float alpha = (grow && m != -INFINITY) ? ex2f(m - mnew) : 1.0f;
+        auto rescale_o = [&](float alpha) {
 #pragma unroll 1
           for (int cc = 0; cc < D; cc += 32) {
             uint32_t ov[32];
@@ -454,24 +429,51 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fine_kernel(const __grid_con
             tmem_st32(tOw + cc, ov);
           }
           tmem_wait_st();
-          l *= alpha;
-          lx *= alpha;
+        };
+        // As in the block-sparse kernel: the max pass runs only while a row
+        // of the warp has no max yet; later tiles check each chunk's weights.
+        const bool need_max = __any_sync(0xffffffffu, m == -INFINITY);
+        if (need_max) {
+          // Pass 1: row max of y = s * scale_log2 + shift over the 128 columns.
+          float mh[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t sr[64];
+            tmem_ld32(tS + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+            tmem_ld32(tS + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+            tmem_wait_ld();
+            const float* xh = reinterpret_cast<const float*>(sr);
+            float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float4 s4 = shw4[16 * h + i];
+              const float2 ya = ffma2(make_float2(xh[4 * i], xh[4 * i + 1]), sc2, make_float2(s4.x, s4.y));
+              const float2 yb = ffma2(make_float2(xh[4 * i + 2], xh[4 * i + 3]), sc2, make_float2(s4.z, s4.w));
+              m0 = fmax3(m0, ya.x, ya.y);
+              m1 = fmax3(m1, yb.x, yb.y);
+            }
+            mh[h] = fmaxf(m0, m1);
+          }
+          const float mnew = fmaxf(m, fmaxf(mh[0], mh[1]));
+          // Lazy rescale: the running max moves only when it grows by more
+          // than 8 (or is set for the first time).
+          const bool grow = mnew > m + 8.0f;
+          if (__any_sync(0xffffffffu, grow && m != -INFINITY)) {
+            const float alpha = (grow && m != -INFINITY) ? ex2f(m - mnew) : 1.0f;
+            rescale_o(alpha);
+            l *= alpha;
+            lx *= alpha;
+          }
+          if (grow) m = mnew;
         }
-        if (grow) m = mnew;
-        const float nm = (m == -INFINITY) ? 0.f : -m;
+        float nm = (m == -INFINITY) ? 0.f : -m;
         // Pass 2: p = 2^(s * scale_log2 + shift - m), 32 keys at a time; the
         // bf16 weights go to columns [16 c, 16 c + 16) of the same buffer.
         float rs[2] = {0.f, 0.f};
-        float rx = 0.f;
-        const float2 nm2 = make_float2(nm, nm), one2 = make_float2(1.f, 1.f);
-        uint32_t sc[2][32];
-        tmem_ld32(tS, sc[0]);
-#pragma unroll
-        for (int cch = 0; cch < 4; ++cch) {
-          tmem_wait_ld();
-          if (cch < 3) tmem_ld32(tS + 32 * (cch + 1), sc[(cch + 1) & 1]);
-          const float* x = reinterpret_cast<const float*>(sc[cch & 1]);
-          uint32_t pk[16];
+        float rx = 0.f, rx_ok = 0.f;
+        const float2 one2 = make_float2(1.f, 1.f);
+        auto exp_chunk = [&](const float* x, int cch, float nmv, uint32_t (&pk)[16]) {
+          const float2 nm2 = make_float2(nmv, nmv);
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const float4 s4 = shw4[8 * cch + i];
@@ -486,7 +488,75 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fine_kernel(const __grid_con
             rs[1] = add_bf16x2(rs[1], pk[2 * i + 1]);
             if (WITH_LSE) rx += (p0 + p1) + (p2 + p3);
           }
+        };
+        int c_fail = 4;
+        uint32_t sc[2][32];
+        tmem_ld32(tS, sc[0]);
+#pragma unroll
+        for (int cch = 0; cch < 4; ++cch) {
+          tmem_wait_ld();
+          if (cch < 3) tmem_ld32(tS + 32 * (cch + 1), sc[(cch + 1) & 1]);
+          uint32_t pk[16];
+          exp_chunk(reinterpret_cast<const float*>(sc[cch & 1]), cch, nm, pk);
+          // a weight of 2^64 or more: this tile's logits exceed the running
+          // max by 64 or more; nothing of this chunk is stored
+          if (!need_max && __any_sync(0xffffffffu, !(rs[0] + rs[1] < 0x1p64f))) {
+            c_fail = cch;
+            break;
+          }
           tmem_st16(tS + 16 * cch, pk);
+          rx_ok = rx;
+        }
+        if (c_fail < 4) {
+          // Rare: a new max from the logits of chunks c_fail..3, O, the sums
+          // and the stored weights rescaled, chunks c_fail..3 redone (as in
+          // the block-sparse kernel).
+          tmem_wait_ld();
+          float mx = -INFINITY;
+#pragma unroll 1
+          for (int cc = c_fail; cc < 4; ++cc) {
+            uint32_t t[32];
+            tmem_ld32(tS + 32 * cc, t);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float4 s4 = shw4[8 * cc + i];
+              mx = fmax3(mx, fmaf(__uint_as_float(t[4 * i]), a.scale_log2, s4.x),
+                         fmaf(__uint_as_float(t[4 * i + 1]), a.scale_log2, s4.y));
+              mx = fmax3(mx, fmaf(__uint_as_float(t[4 * i + 2]), a.scale_log2, s4.z),
+                         fmaf(__uint_as_float(t[4 * i + 3]), a.scale_log2, s4.w));
+            }
+          }
+          const float mnew = fmaxf(m, mx);
+          const float alpha = ex2f(m - mnew);   // m is finite: the max pass ran on an earlier tile
+          rescale_o(alpha);
+          l *= alpha;
+          lx *= alpha;
+          rs[0] = rs[1] = 0.f;
+#pragma unroll 1
+          for (int cc = 0; cc < c_fail; ++cc) {
+            uint32_t pv[16];
+            tmem_ld16(tS + 16 * cc, pv);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              pv[i] = pack_bf16(__uint_as_float(pv[i] << 16) * alpha, __uint_as_float(pv[i] & 0xFFFF0000u) * alpha);
+              rs[i & 1] = add_bf16x2(rs[i & 1], pv[i]);
+            }
+            tmem_st16(tS + 16 * cc, pv);
+          }
+          rx = alpha * rx_ok;
+          m = mnew;
+          nm = -m;
+#pragma unroll 1
+          for (int cc = c_fail; cc < 4; ++cc) {
+            uint32_t t[32];
+            tmem_ld32(tS + 32 * cc, t);
+            tmem_wait_ld();
+            uint32_t pk[16];
+            exp_chunk(reinterpret_cast<const float*>(t), cc, nm, pk);
+            tmem_st16(tS + 16 * cc, pk);
+          }
         }
         l += rs[0] + rs[1];
         if (WITH_LSE) lx += rx;

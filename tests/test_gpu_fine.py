@@ -237,3 +237,21 @@ def test_wan480p_sampled_query_blocks(bsa):
         mx, mean = compare_outputs(O[b, h, lo:hi].double().numpy(), O_ref)
         assert mx <= MAX_ABS and mean <= MEAN_ABS, ((b, h, I), mx, mean)
         assert np.abs(L[b, h, lo:hi].double().numpy() - lse_ref).max() <= LSE_ABS
+
+
+def test_weights_past_the_unchecked_range(bsa):
+    """Entries of every tile after the first two weighted 2^70: each group's
+    logits jump by 70 (log2 units) after its first tile, past the range the
+    kernel accepts without a max pass, so every query block redoes a tile with
+    a new max (O, sums and stored weights rescaled)."""
+    w = small("fine_jump", 1, 4, 16, 16, 2, 128, 128, 8, 0.0, seed=51)
+    q, k, v = _inputs(w)
+    nq, nkb = w.Npad // 128, -(-w.N // KB)
+    off, idx, wt = synth.random_fine_lists(w.B, w.heads, nq, nkb, 0.6, w.seed)
+    wt = torch.ones_like(wt)
+    for r in range(off.numel() - 1):
+        lo, hi = int(off[r]), int(off[r + 1])
+        wt[lo + 64:hi] = 2.0 ** 70
+    o, l, status = _run(bsa, w, q, k, v, off, idx, wt)
+    assert status == 0
+    _check_all(w, q, k, v, off, idx, wt, o, l)
