@@ -63,11 +63,17 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def attn_source_hash() -> str:
+# the kernel source each recorded traffic figure was taken from (the shared
+# headers count for all of them)
+TRAFFIC_SOURCES = {"attn": "attn_fwd.cu", "fine": "attn_fine.cu"}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    csrc = os.path.join(ROOT, "block_sparse_attention_fractal_b200", "csrc")
     h = hashlib.sha256()
-    for fn in sorted(os.listdir(os.path.join(ROOT, "block_sparse_attention_fractal_b200", "csrc"))):
-        if fn.startswith("attn") or fn.endswith((".cuh", ".h")):
-            with open(os.path.join(ROOT, "block_sparse_attention_fractal_b200", "csrc", fn), "rb") as f:
+    for fn in sorted(os.listdir(csrc)):
+        if fn == TRAFFIC_SOURCES[kernel] or fn.endswith((".cuh", ".h")):
+            with open(os.path.join(csrc, fn), "rb") as f:
                 h.update(fn.encode() + f.read())
     return h.hexdigest()[:16]
 
@@ -81,7 +87,7 @@ def recorded_traffic(kernel: str, workload: str):
     with open(path) as f:
         rec = json.load(f)
     ent = rec.get(kernel)
-    if not ent or ent.get("source_hash") != attn_source_hash() or ent.get("workload") != workload:
+    if not ent or ent.get("source_hash") != kernel_source_hash(kernel) or ent.get("workload") != workload:
         return None
     return ent.get("bytes_per_launch")
 

@@ -21,10 +21,14 @@
 //                dP^T = V dO^T into TMEM, P^T and dS^T written as bf16 over
 //                their own columns, dV += P^T dO and dK += dS^T Q with A from
 //                TMEM.
-// tcgen05.mma operations of one thread execute in issue order: the next
-// tile's S and dP overwrite the bf16 operands of the previous tile's last
-// MMAs only after those have read them.  Both kernels are single-buffered in
-// TMEM (S, dP and the accumulators fill it), so the softmax warps and the
+// tcgen05.mma operations of one thread execute in issue order: a product
+// that overwrites the bf16 operand of an earlier product runs after it.
+// The dq kernel keeps S in two TMEM buffers and writes dS over the S it was
+// computed from, so the next tile's dP (one fixed buffer, free once the
+// softmax warps have read it) is issued as soon as they finish a tile, ahead
+// of that tile's dQ product and the S of the tile after next: only one
+// product sits between two tiles' softmax work.  The dkdv kernel has no TMEM
+// to spare (S, dP and two accumulators fill it), so its softmax warps and
 // tensor pipe take turns within a tile.
 //
 // Small kernels before them: D = rowsum(dO * O) per row (fp32), and the
@@ -54,7 +58,10 @@ constexpr int kSoftmaxWarp0 = 4;
 constexpr uint32_t kGroupThreads = 128;
 constexpr uint64_t kWaitNs = 250ull * 1000ull * 1000ull;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTS = 0, kTdP = 128, kTAcc0 = 256, kTAcc1 = 384;   // TMEM column bases
+// TMEM column bases.  dkdv: S^T (P^T over it), dP^T (dS^T over it), dV, dK.
+// dq: S of even tiles, dP, S of odd tiles (dS over each S), dQ.
+constexpr uint32_t kTS = 0, kTdP = 128, kTAcc0 = 256, kTAcc1 = 384;
+constexpr uint32_t kTS1 = 256, kTdQ = 384;
 constexpr uint16_t kEntBlock = 0x0FFFu;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -137,7 +144,7 @@ __global__ void __launch_bounds__(256) bwd_tlist_kernel(const uint32_t* __restri
 // ------------------------------------------------------- the main kernels
 
 struct Ctl {
-  uint64_t a_full[2], a_empty[2], b_full[2], b_empty[2];   // per-tile operand stages (two each)
+  uint64_t a_full[3], a_empty[3], b_full[2], b_empty[2];   // per-tile operand stages (a: three for dq)
   uint64_t fixed_full;                                      // the item's fixed operands
   uint64_t sdp_full, ds_full, acc_done, drain;
   uint32_t tmem_base;
@@ -163,8 +170,8 @@ __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, Ctrl* 
 
 // One kernel body for both passes.
 //   DKDV = false (dq pass): fixed operands Q and dO (128 query rows), tile
-//     operands K (stage a) and V (stage b) of each KV tile; S = Q K^T,
-//     dP = dO V^T; acc0 = dQ += dS K.
+//     operands K (stage a, three stages: S of a tile is issued a tile ahead)
+//     and V (stage b) of each KV tile; S = Q K^T, dP = dO V^T; dQ += dS K.
 //   DKDV = true (dkdv pass): fixed operands K and V (128 keys), tile operands
 //     Q (a) and dO (b) of each query tile, plus that tile's L and D rows;
 //     S^T = K Q^T, dP^T = V dO^T; acc0 = dV += P^T dO, acc1 = dK += dS^T Q.
@@ -182,6 +189,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kernel(
   constexpr int CH = D / 64;            // 128-byte chunks of a row
   constexpr uint32_t kTile = 128u * D * 2u;
   constexpr uint32_t kChunk = 128u * 128u;
+  constexpr uint32_t NA = DKDV ? 2u : 3u;   // stages of tile operand a
+  constexpr uint32_t kRowBytes = DKDV ? 2u * 256u * sizeof(float) : 0u;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if (smem_addr(smem_raw) & 1023u) {
@@ -190,18 +199,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kernel(
   }
   uint8_t* sF0 = smem_raw;              // fixed operand 0 (Q or K)
   uint8_t* sF1 = sF0 + kTile;           // fixed operand 1 (dO or V)
-  uint8_t* sA = sF0 + 2 * kTile;        // two stages of tile operand a (K or Q)
-  uint8_t* sB = sF0 + 4 * kTile;        // two stages of tile operand b (V or dO)
-  float* sRow = reinterpret_cast<float*>(sF0 + 6 * kTile);   // dkdv: [stage][L 128 | D 128]
-  Ctl& c = *reinterpret_cast<Ctl*>(sF0 + 6 * kTile + 2 * 256 * sizeof(float));
+  uint8_t* sA = sF0 + 2 * kTile;        // NA stages of tile operand a (K or Q)
+  uint8_t* sB = sA + NA * kTile;        // two stages of tile operand b (V or dO)
+  float* sRow = reinterpret_cast<float*>(sB + 2 * kTile);   // dkdv: [stage][L 128 | D 128]
+  Ctl& c = *reinterpret_cast<Ctl*>(sB + 2 * kTile + kRowBytes);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nb = g.nb, nw = (nb + 31) >> 5;
 
   if (tid == 0) {
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < (int)NA; ++s) {
       mbar_init(&c.a_full[s], 1);
       mbar_init(&c.a_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&c.b_full[s], 1);
       mbar_init(&c.b_empty[s], 1);
     }
@@ -329,11 +340,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kernel(
               tma_load_3d(sF1 + ch * kChunk + h * (kChunk / 2), &mfix1, &c.fixed_full, ch * 64, fixed_row0(h), bh);
             }
         }
+        const uint32_t ns = is_a ? NA : 2u;
         for (int j = 0; j < n_tiles; ++j) {
-          const uint32_t jg = jbase + j, s = jg & 1;
+          const uint32_t jg = jbase + j, s = jg % ns;
           uint64_t* full = is_a ? &c.a_full[s] : &c.b_full[s];
           uint64_t* empty = is_a ? &c.a_empty[s] : &c.b_empty[s];
-          if (jg >= 2 && !wait(empty, ((jg - 2) >> 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 10); break; }
+          if (jg >= ns && !wait(empty, ((jg / ns) - 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 10); break; }
           const uint32_t extra = (!is_a && DKDV) ? 2u * 128u * sizeof(float) : 0u;
           mbar_arrive_expect_tx(full, kTile + extra);
           ++armed;
@@ -356,9 +368,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kernel(
       }
     } else if (warp == 1) {
       // ------------------------------------------------------------ MMA issuer
-      // per walked tile j: S_j and dP_j into TMEM; once the softmax warps
-      // have written the bf16 operands, the accumulating products.  Issue
-      // order makes the next tile's S and dP wait for them.
       if (lane == 0 && n_tiles > 0) {
         constexpr uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);
         constexpr uint32_t idO = idesc_bf16_f32(128, D, 0, 1);
@@ -367,36 +376,82 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kernel(
         const uint32_t aA = smem_addr(sA), aB = smem_addr(sB);
         bool go = wait(&c.fixed_full, nfix & 1, ctrl, seq);
         if (!go) timeout(ctrl, c, seq, 20);
-        for (int j = 0; go && j < n_tiles; ++j) {
-          const uint32_t jg = jbase + j, s = jg & 1;
-          if (!wait(&c.a_full[s], (jg >> 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 21); break; }
-          if (!wait(&c.b_full[s], (jg >> 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 22); break; }
-          tc_fence_after();
-          const uint64_t dA = smem_desc_sw128(aA + s * kTile, 16, 1024);
-          const uint64_t dB = smem_desc_sw128(aB + s * kTile, 16, 1024);
-          // dq: S = Q K^T (fixed0 x a), dP = dO V^T (fixed1 x b)
-          // dkdv: S^T = K Q^T (fixed0 x a), dP^T = V dO^T (fixed1 x b)
+        if (!DKDV) {
+          // dq, per walked tile j: S_j = Q K_j^T into the S buffer of j's
+          // parity, issued a tile ahead; dP_j = dO V_j^T as soon as the
+          // softmax warps are done with tile j - 1 (its dP is read); then
+          // dQ += dS_{j-1} K_{j-1} and S_{j+1} over dS_{j-1}.
+          auto issue_s = [&](uint32_t jg) -> bool {
+            const uint32_t sa = jg % NA;
+            if (!wait(&c.a_full[sa], (jg / NA) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 21); return false; }
+            tc_fence_after();
+            const uint64_t dA = smem_desc_sw128(aA + sa * kTile, 16, 1024);
+            const uint32_t col = (jg & 1) ? kTS1 : kTS;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
-            mma_ss(tmem + kTS, smem_desc_add(dF0, off), smem_desc_add(dA, off), idS, kk > 0);
-          }
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
+              mma_ss(tmem + col, smem_desc_add(dF0, off), smem_desc_add(dA, off), idS, kk > 0);
+            }
+            return true;
+          };
+          auto issue_dp = [&](uint32_t jg) -> bool {
+            const uint32_t sb = jg & 1;
+            if (!wait(&c.b_full[sb], (jg >> 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 22); return false; }
+            tc_fence_after();
+            const uint64_t dB = smem_desc_sw128(aB + sb * kTile, 16, 1024);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
-            mma_ss(tmem + kTdP, smem_desc_add(dF1, off), smem_desc_add(dB, off), idS, kk > 0);
-          }
-          mma_commit(&c.sdp_full);
-          if (!wait(&c.ds_full, jg & 1, ctrl, seq)) { timeout(ctrl, c, seq, 23); break; }
-          tc_fence_after();
-          const uint32_t acc = (j > 0) ? 1u : 0u;
-          if (!DKDV) {
-            // dQ += dS K: A = dS (bf16 over the dP columns), B = K (MN-major)
-            const uint64_t dK = smem_desc_sw128(aA + s * kTile, kChunk, 1024);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
+              mma_ss(tmem + kTdP, smem_desc_add(dF1, off), smem_desc_add(dB, off), idS, kk > 0);
+            }
+            mma_commit(&c.sdp_full);    // S_j (issued before) and dP_j
+            mma_commit(&c.b_empty[sb]); // V_j is read by dP_j alone
+            return true;
+          };
+          go = go && issue_s(jbase);
+          go = go && (n_tiles < 2 || issue_s(jbase + 1));
+          go = go && issue_dp(jbase);
+          for (int j = 0; go && j < n_tiles; ++j) {
+            const uint32_t jg = jbase + j, sa = jg % NA;
+            if (!wait(&c.ds_full, jg & 1, ctrl, seq)) { timeout(ctrl, c, seq, 23); break; }
+            tc_fence_after();
+            if (j + 1 < n_tiles && !issue_dp(jg + 1)) break;
+            // dQ += dS K: A = dS (bf16 over the S columns), B = K (MN-major)
+            const uint32_t col = (jg & 1) ? kTS1 : kTS;
+            const uint64_t dK = smem_desc_sw128(aA + sa * kTile, kChunk, 1024);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              mma_ts(tmem + kTAcc0, tmem + kTdP + 8 * kk, smem_desc_add(dK, kk * 2048), idO, kk > 0 ? 1u : acc);
-          } else {
+              mma_ts(tmem + kTdQ, tmem + col + 8 * kk, smem_desc_add(dK, kk * 2048), idO, (kk > 0 || j > 0) ? 1u : 0u);
+            mma_commit(&c.a_empty[sa]);
+            if (j == n_tiles - 1) mma_commit(&c.acc_done);
+            if (j + 2 < n_tiles && !issue_s(jg + 2)) break;
+          }
+        } else {
+          // dkdv, per walked tile j: S^T_j and dP^T_j into TMEM; once the
+          // softmax warps have written P^T and dS^T over them, dV and dK.
+          // Issue order makes the next tile's S^T and dP^T wait for those.
+          for (int j = 0; go && j < n_tiles; ++j) {
+            const uint32_t jg = jbase + j, s = jg & 1;
+            if (!wait(&c.a_full[s], (jg >> 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 21); break; }
+            if (!wait(&c.b_full[s], (jg >> 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 22); break; }
+            tc_fence_after();
+            const uint64_t dA = smem_desc_sw128(aA + s * kTile, 16, 1024);
+            const uint64_t dB = smem_desc_sw128(aB + s * kTile, 16, 1024);
+            // S^T = K Q^T (fixed0 x a), dP^T = V dO^T (fixed1 x b)
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
+              mma_ss(tmem + kTS, smem_desc_add(dF0, off), smem_desc_add(dA, off), idS, kk > 0);
+            }
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
+              mma_ss(tmem + kTdP, smem_desc_add(dF1, off), smem_desc_add(dB, off), idS, kk > 0);
+            }
+            mma_commit(&c.sdp_full);
+            if (!wait(&c.ds_full, jg & 1, ctrl, seq)) { timeout(ctrl, c, seq, 23); break; }
+            tc_fence_after();
+            const uint32_t acc = (j > 0) ? 1u : 0u;
             // dV += P^T dO: A = P^T (over the S columns), B = dO (MN-major);
             // dK += dS^T Q: A = dS^T (over the dP columns), B = Q (MN-major)
             const uint64_t dQt = smem_desc_sw128(aA + s * kTile, kChunk, 1024);
@@ -407,10 +462,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kernel(
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
               mma_ts(tmem + kTAcc1, tmem + kTdP + 8 * kk, smem_desc_add(dQt, kk * 2048), idO, kk > 0 ? 1u : acc);
+            mma_commit(&c.a_empty[s]);
+            mma_commit(&c.b_empty[s]);
+            if (j == n_tiles - 1) mma_commit(&c.acc_done);
           }
-          mma_commit(&c.a_empty[s]);
-          mma_commit(&c.b_empty[s]);
-          if (j == n_tiles - 1) mma_commit(&c.acc_done);
         }
       }
     } else if (warp >= kSoftmaxWarp0) {
@@ -452,19 +507,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kernel(
         }
         if (!wait_warp(&c.sdp_full, jg & 1, ctrl, seq)) { timeout(ctrl, c, seq, 30); ok = false; break; }
         tc_fence_after();
+        const uint32_t tS = trow + (DKDV ? kTS : ((jg & 1) ? kTS1 : kTS));   // this tile's S columns
         const float* rowL = sRow + s * 256;          // dkdv: L of the tile's 128 query columns, then D
         const float2 sl2 = make_float2(scale_log2, scale_log2), nlg2 = make_float2(-kLog2e, -kLog2e);
         // two buffers: the next chunk's scores and dP load while this one is
         // computed
         uint32_t sv2[2][32], dv2[2][32];
-        tmem_ld32(trow + kTS, sv2[0]);
+        tmem_ld32(tS, sv2[0]);
         tmem_ld32(trow + kTdP, dv2[0]);
 #pragma unroll
         for (int cch = 0; cch < 4; ++cch) {
           const int h = cch >> 1;
           tmem_wait_ld();
           if (cch < 3) {
-            tmem_ld32(trow + kTS + 32 * (cch + 1), sv2[(cch + 1) & 1]);
+            tmem_ld32(tS + 32 * (cch + 1), sv2[(cch + 1) & 1]);
             tmem_ld32(trow + kTdP + 32 * (cch + 1), dv2[(cch + 1) & 1]);
           }
           const uint32_t* sv = sv2[cch & 1];
@@ -505,10 +561,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kernel(
 #pragma unroll
             for (int i = 0; i < 16; ++i) pk[i] = dk[i] = 0u;
           }
-          // bf16 operands over columns already read: P (dkdv only) over S,
-          // dS over dP, two per 32-bit column
-          if (DKDV) tmem_st16(trow + kTS + 16 * cch, pk);
-          tmem_st16(trow + kTdP + 16 * cch, dk);
+          // bf16 operands over columns already read, two per 32-bit column:
+          // dkdv P^T over S^T and dS^T over dP^T; dq dS over S (dP is then
+          // free for the next tile's product)
+          if (DKDV) {
+            tmem_st16(tS + 16 * cch, pk);
+            tmem_st16(trow + kTdP + 16 * cch, dk);
+          } else {
+            tmem_st16(tS + 16 * cch, dk);
+          }
         }
         tmem_wait_st();
         tc_fence_before();
@@ -525,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kernel(
         // dq: out0 = dQ (scaled); dkdv: out0 = dV (acc0), out1 = dK (acc1, scaled)
         __nv_bfloat16* dst = (a == 0) ? out0 : out1;
         const float mul = (DKDV && a == 0) ? 1.f : scale;
-        const uint32_t tacc = trow + (a == 0 ? kTAcc0 : kTAcc1);
+        const uint32_t tacc = trow + (DKDV ? (a == 0 ? kTAcc0 : kTAcc1) : kTdQ);
         uint4* orow = reinterpret_cast<uint4*>(dst + ((size_t)bh * g.Npad + (store ? frow : 0)) * D);
 #pragma unroll 1
         for (int cc = 0; cc < D; cc += 16) {
@@ -557,7 +618,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kernel(
   if (lane == 0) {
     if (warp == 0) {
       mbar_drain_ring(&c.fixed_full, 1, nfix, kWaitNs);
-      mbar_drain_ring(c.a_full, 2, armed, kWaitNs);
+      mbar_drain_ring(c.a_full, NA, armed, kWaitNs);
     } else if (warp == 2) {
       mbar_drain_ring(c.b_full, 2, armed, kWaitNs);
     } else if (warp == 1) {
@@ -586,8 +647,11 @@ cudaError_t launch_pass(const Dims& g, const void* fix0, const void* fix1, const
     return cudaErrorInvalidValue;
   const int items_per_bh = (BS == 64) ? (g.nb + 1) / 2 : g.nb;
   const int n_items = (int)(bhs * items_per_bh);
-  const size_t smem = 6u * 128u * D * 2u + 2u * 256u * sizeof(float) + sizeof(Ctl);
+  // Q/K and dO/V, the stages of a (three for dq, two for dkdv) and of b, the
+  // dkdv L and D rows, the control block
+  const size_t smem = (DKDV ? 6u : 7u) * 128u * D * 2u + (DKDV ? 2u * 256u * sizeof(float) : 0u) + sizeof(Ctl);
   static_assert(6u * 128u * 128u * 2u + 2u * 256u * sizeof(float) + sizeof(Ctl) <= 227u * 1024u, "smem layout");
+  static_assert(7u * 128u * 128u * 2u + sizeof(Ctl) <= 227u * 1024u, "smem layout");
   cudaError_t e =
       cudaFuncSetAttribute(attn_bwd_kernel<D, BS, DKDV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
