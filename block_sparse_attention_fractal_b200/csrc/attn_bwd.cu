@@ -28,8 +28,11 @@
 // softmax warps have read it) is issued as soon as they finish a tile, ahead
 // of that tile's dQ product and the S of the tile after next: only one
 // product sits between two tiles' softmax work.  The dkdv kernel has no TMEM
-// to spare (S, dP and two accumulators fill it), so its softmax warps and
-// tensor pipe take turns within a tile.
+// to spare (S, dP and two accumulators fill it); its softmax warps work in two
+// phases instead: P^T from S^T alone (the exponentials), then dS^T from the
+// bf16 P^T kept in registers once dP^T is there.  dV and the next S^T run
+// after the first phase, dK and the next dP^T after the second, so the next
+// tile's exponentials overlap dK and dP^T.
 //
 // Small kernels before them: D = rowsum(dO * O) per row (fp32), and the
 // transposed lists (for each KV block, the ascending list of query blocks
@@ -147,6 +150,7 @@ struct Ctl {
   uint64_t a_full[3], a_empty[3], b_full[2], b_empty[2];   // per-tile operand stages (a: three for dq)
   uint64_t fixed_full;                                      // the item's fixed operands
   uint64_t sdp_full, ds_full, acc_done, drain;
+  uint64_t dp_full, p_full;                                 // dkdv: dP^T in TMEM; P^T written
   uint32_t tmem_base;
   int n_ent;
   int item;
@@ -219,6 +223,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kernel(
     mbar_init(&c.fixed_full, 1);
     mbar_init(&c.sdp_full, 1);
     mbar_init(&c.ds_full, kGroupThreads);
+    mbar_init(&c.dp_full, 1);
+    mbar_init(&c.p_full, kGroupThreads);
     mbar_init(&c.acc_done, 1);
     mbar_init(&c.drain, 1);
     c.abort = 0;
@@ -427,44 +433,61 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kernel(
             if (j + 2 < n_tiles && !issue_s(jg + 2)) break;
           }
         } else {
-          // dkdv, per walked tile j: S^T_j and dP^T_j into TMEM; once the
-          // softmax warps have written P^T and dS^T over them, dV and dK.
-          // Issue order makes the next tile's S^T and dP^T wait for those.
-          for (int j = 0; go && j < n_tiles; ++j) {
-            const uint32_t jg = jbase + j, s = jg & 1;
-            if (!wait(&c.a_full[s], (jg >> 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 21); break; }
-            if (!wait(&c.b_full[s], (jg >> 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 22); break; }
+          // dkdv, per walked tile j: S^T_j = K Q_j^T, then dP^T_j = V dO_j^T,
+          // each on a barrier of its own; once the softmax warps have written
+          // P^T_j over S^T_j, dV += P^T dO and S^T_{j+1} over it; once they
+          // have written dS^T_j over dP^T_j, dK += dS^T Q and dP^T_{j+1}.
+          // The softmax warps compute P^T_{j+1} while dK and dP^T_{j+1} run.
+          auto issue_s = [&](uint32_t jg) -> bool {
+            const uint32_t s = jg & 1;
+            if (!wait(&c.a_full[s], (jg >> 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 21); return false; }
             tc_fence_after();
             const uint64_t dA = smem_desc_sw128(aA + s * kTile, 16, 1024);
-            const uint64_t dB = smem_desc_sw128(aB + s * kTile, 16, 1024);
-            // S^T = K Q^T (fixed0 x a), dP^T = V dO^T (fixed1 x b)
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
               mma_ss(tmem + kTS, smem_desc_add(dF0, off), smem_desc_add(dA, off), idS, kk > 0);
             }
+            mma_commit(&c.sdp_full);
+            return true;
+          };
+          auto issue_dp = [&](uint32_t jg) -> bool {
+            const uint32_t s = jg & 1;
+            if (!wait(&c.b_full[s], (jg >> 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 22); return false; }
+            tc_fence_after();
+            const uint64_t dB = smem_desc_sw128(aB + s * kTile, 16, 1024);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
               mma_ss(tmem + kTdP, smem_desc_add(dF1, off), smem_desc_add(dB, off), idS, kk > 0);
             }
-            mma_commit(&c.sdp_full);
-            if (!wait(&c.ds_full, jg & 1, ctrl, seq)) { timeout(ctrl, c, seq, 23); break; }
-            tc_fence_after();
+            mma_commit(&c.dp_full);
+            return true;
+          };
+          go = go && issue_s(jbase) && issue_dp(jbase);
+          for (int j = 0; go && j < n_tiles; ++j) {
+            const uint32_t jg = jbase + j, s = jg & 1;
             const uint32_t acc = (j > 0) ? 1u : 0u;
-            // dV += P^T dO: A = P^T (over the S columns), B = dO (MN-major);
-            // dK += dS^T Q: A = dS^T (over the dP columns), B = Q (MN-major)
-            const uint64_t dQt = smem_desc_sw128(aA + s * kTile, kChunk, 1024);
+            if (!wait(&c.p_full, jg & 1, ctrl, seq)) { timeout(ctrl, c, seq, 23); break; }
+            tc_fence_after();
+            // dV += P^T dO: A = P^T (bf16 over the S columns), B = dO (MN-major)
             const uint64_t dOt = smem_desc_sw128(aB + s * kTile, kChunk, 1024);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
               mma_ts(tmem + kTAcc0, tmem + kTS + 8 * kk, smem_desc_add(dOt, kk * 2048), idO, kk > 0 ? 1u : acc);
+            if (j + 1 < n_tiles && !issue_s(jg + 1)) break;
+            if (!wait(&c.ds_full, jg & 1, ctrl, seq)) { timeout(ctrl, c, seq, 24); break; }
+            tc_fence_after();
+            // dK += dS^T Q: A = dS^T (bf16 over the dP columns), B = Q (MN-major)
+            const uint64_t dQt = smem_desc_sw128(aA + s * kTile, kChunk, 1024);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
               mma_ts(tmem + kTAcc1, tmem + kTdP + 8 * kk, smem_desc_add(dQt, kk * 2048), idO, kk > 0 ? 1u : acc);
+            // the stages (and this tile's L and D rows) are free once dK has read Q
             mma_commit(&c.a_empty[s]);
             mma_commit(&c.b_empty[s]);
             if (j == n_tiles - 1) mma_commit(&c.acc_done);
+            if (j + 1 < n_tiles && !issue_dp(jg + 1)) break;
           }
         }
       }
@@ -507,68 +530,118 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kernel(
         }
         if (!wait_warp(&c.sdp_full, jg & 1, ctrl, seq)) { timeout(ctrl, c, seq, 30); ok = false; break; }
         tc_fence_after();
-        const uint32_t tS = trow + (DKDV ? kTS : ((jg & 1) ? kTS1 : kTS));   // this tile's S columns
-        const float* rowL = sRow + s * 256;          // dkdv: L of the tile's 128 query columns, then D
-        const float2 sl2 = make_float2(scale_log2, scale_log2), nlg2 = make_float2(-kLog2e, -kLog2e);
-        // two buffers: the next chunk's scores and dP load while this one is
-        // computed
-        uint32_t sv2[2][32], dv2[2][32];
-        tmem_ld32(tS, sv2[0]);
-        tmem_ld32(trow + kTdP, dv2[0]);
+        const float2 sl2 = make_float2(scale_log2, scale_log2);
+        if (!DKDV) {
+          // dq: S and dP are both in TMEM; per pair of columns
+          // p = 2^(x scale log2 e - L log2 e), dS = p (dP - D) in packed
+          // two-lane arithmetic, dS as bf16 over the S columns already read
+          // (dP is then free for the next tile's product).  Two buffers: the
+          // next chunk's scores and dP load while this one is computed.
+          const uint32_t tS = trow + ((jg & 1) ? kTS1 : kTS);
+          const float2 nl = make_float2(-lse2, -lse2), dd = make_float2(drow, drow);
+          uint32_t sv2[2][32], dv2[2][32];
+          tmem_ld32(tS, sv2[0]);
+          tmem_ld32(trow + kTdP, dv2[0]);
 #pragma unroll
-        for (int cch = 0; cch < 4; ++cch) {
-          const int h = cch >> 1;
-          tmem_wait_ld();
-          if (cch < 3) {
-            tmem_ld32(tS + 32 * (cch + 1), sv2[(cch + 1) & 1]);
-            tmem_ld32(trow + kTdP + 32 * (cch + 1), dv2[(cch + 1) & 1]);
-          }
-          const uint32_t* sv = sv2[cch & 1];
-          const uint32_t* dv = dv2[cch & 1];
-          // valid columns of this chunk: all 32 (no per-column test in the
-          // loop, the common case), some, or none
-          const int cl = min(32, max(0, lim[h] - 32 * (cch & 1)));
-          uint32_t pk[16], dk[16];
-          // one pair of columns: p = 2^(x scale log2 e - L log2 e),
-          // dS = p (dP - D), in packed two-lane arithmetic
-          auto pair = [&](int i, bool masked) {
-            const int col = 32 * cch + 2 * i;
-            float2 nl, dd;   // -L log2 e and D
-            if (DKDV) {
-              nl = fmul2(*reinterpret_cast<const float2*>(rowL + col), nlg2);
-              dd = *reinterpret_cast<const float2*>(rowL + 128 + col);
+          for (int cch = 0; cch < 4; ++cch) {
+            tmem_wait_ld();
+            if (cch < 3) {
+              tmem_ld32(tS + 32 * (cch + 1), sv2[(cch + 1) & 1]);
+              tmem_ld32(trow + kTdP + 32 * (cch + 1), dv2[(cch + 1) & 1]);
+            }
+            const uint32_t* sv = sv2[cch & 1];
+            const uint32_t* dv = dv2[cch & 1];
+            // valid columns of this chunk: all 32 (no per-column test in the
+            // loop, the common case), some, or none
+            const int cl = min(32, max(0, lim[cch >> 1] - 32 * (cch & 1)));
+            uint32_t dk[16];
+            auto pair = [&](int i, bool masked) {
+              const float2 y = ffma2(make_float2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), sl2, nl);
+              float2 p = make_float2(ex2f(y.x), ex2f(y.y));
+              if (masked) {
+                p.x = (2 * i < cl) ? p.x : 0.f;
+                p.y = (2 * i + 1 < cl) ? p.y : 0.f;
+              }
+              const float2 ds = fmul2(p, fsub2(make_float2(__uint_as_float(dv[2 * i]), __uint_as_float(dv[2 * i + 1])), dd));
+              dk[i] = pack_bf16(ds.x, ds.y);
+            };
+            if (cl == 32) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) pair(i, false);
+            } else if (cl > 0) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) pair(i, true);
             } else {
-              nl = make_float2(-lse2, -lse2);
-              dd = make_float2(drow, drow);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) dk[i] = 0u;
             }
-            const float2 y = ffma2(make_float2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), sl2, nl);
-            float2 p = make_float2(ex2f(y.x), ex2f(y.y));
-            if (masked) {
-              p.x = (2 * i < cl) ? p.x : 0.f;
-              p.y = (2 * i + 1 < cl) ? p.y : 0.f;
-            }
-            const float2 ds = fmul2(p, fsub2(make_float2(__uint_as_float(dv[2 * i]), __uint_as_float(dv[2 * i + 1])), dd));
-            pk[i] = pack_bf16(p.x, p.y);
-            dk[i] = pack_bf16(ds.x, ds.y);
-          };
-          if (cl == 32) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) pair(i, false);
-          } else if (cl > 0) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) pair(i, true);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) pk[i] = dk[i] = 0u;
-          }
-          // bf16 operands over columns already read, two per 32-bit column:
-          // dkdv P^T over S^T and dS^T over dP^T; dq dS over S (dP is then
-          // free for the next tile's product)
-          if (DKDV) {
-            tmem_st16(tS + 16 * cch, pk);
-            tmem_st16(trow + kTdP + 16 * cch, dk);
-          } else {
             tmem_st16(tS + 16 * cch, dk);
+          }
+        } else {
+          // dkdv phase 1, S^T alone: P^T = 2^(x scale log2 e - L log2 e) per
+          // pair of columns, as bf16 over the S^T columns already read and
+          // kept in registers; then the dV product may run.
+          // L and D of the tile's 128 query columns land with its dO stage,
+          // which S^T does not wait for
+          if (!wait_warp(&c.b_full[s], (jg >> 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 33); ok = false; break; }
+          const float* rowL = sRow + s * 256;
+          const float2 nlg2 = make_float2(-kLog2e, -kLog2e);
+          uint32_t pk[4][16];
+          {
+            uint32_t sv2[2][32];
+            tmem_ld32(trow + kTS, sv2[0]);
+#pragma unroll
+            for (int cch = 0; cch < 4; ++cch) {
+              tmem_wait_ld();
+              if (cch < 3) tmem_ld32(trow + kTS + 32 * (cch + 1), sv2[(cch + 1) & 1]);
+              const uint32_t* sv = sv2[cch & 1];
+              const int cl = min(32, max(0, lim[cch >> 1] - 32 * (cch & 1)));
+              auto pair = [&](int i, bool masked) {
+                const float2 nl = fmul2(*reinterpret_cast<const float2*>(rowL + 32 * cch + 2 * i), nlg2);
+                const float2 y = ffma2(make_float2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), sl2, nl);
+                float2 p = make_float2(ex2f(y.x), ex2f(y.y));
+                if (masked) {
+                  p.x = (2 * i < cl) ? p.x : 0.f;
+                  p.y = (2 * i + 1 < cl) ? p.y : 0.f;
+                }
+                pk[cch][i] = pack_bf16(p.x, p.y);
+              };
+              if (cl == 32) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pair(i, false);
+              } else if (cl > 0) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pair(i, true);
+              } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pk[cch][i] = 0u;
+              }
+              tmem_st16(trow + kTS + 16 * cch, pk[cch]);
+            }
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&c.p_full);
+          // phase 2, once dP^T is in TMEM: dS^T = P^T (dP^T - D) from the
+          // bf16 P^T (the operand dV uses), as bf16 over the dP^T columns
+          if (!wait_warp(&c.dp_full, jg & 1, ctrl, seq)) { timeout(ctrl, c, seq, 32); ok = false; break; }
+          tc_fence_after();
+          uint32_t dv2[2][32];
+          tmem_ld32(trow + kTdP, dv2[0]);
+#pragma unroll
+          for (int cch = 0; cch < 4; ++cch) {
+            tmem_wait_ld();
+            if (cch < 3) tmem_ld32(trow + kTdP + 32 * (cch + 1), dv2[(cch + 1) & 1]);
+            const uint32_t* dv = dv2[cch & 1];
+            uint32_t dk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float2 p = make_float2(__uint_as_float(pk[cch][i] << 16), __uint_as_float(pk[cch][i] & 0xFFFF0000u));
+              const float2 dd = *reinterpret_cast<const float2*>(rowL + 128 + 32 * cch + 2 * i);
+              const float2 ds = fmul2(p, fsub2(make_float2(__uint_as_float(dv[2 * i]), __uint_as_float(dv[2 * i + 1])), dd));
+              dk[i] = pack_bf16(ds.x, ds.y);
+            }
+            tmem_st16(trow + kTdP + 16 * cch, dk);
           }
         }
         tmem_wait_st();
