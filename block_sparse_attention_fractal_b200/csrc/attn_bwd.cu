@@ -150,7 +150,8 @@ struct Ctl {
   uint64_t a_full[3], a_empty[3], b_full[2], b_empty[2];   // per-tile operand stages (a: three for dq)
   uint64_t fixed_full;                                      // the item's fixed operands
   uint64_t sdp_full, ds_full, acc_done, drain;
-  uint64_t dp_full, p_full;                                 // dkdv: dP^T in TMEM; P^T written
+  uint64_t dp_full, p_full;                                 // dP (dP^T) in TMEM; dkdv: P^T written
+  uint64_t s_full[2];                                       // dq: S in TMEM buffer 0 / 1
   uint32_t tmem_base;
   int n_ent;
   int item;
@@ -225,6 +226,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kernel(
     mbar_init(&c.ds_full, kGroupThreads);
     mbar_init(&c.dp_full, 1);
     mbar_init(&c.p_full, kGroupThreads);
+    mbar_init(&c.s_full[0], 1);
+    mbar_init(&c.s_full[1], 1);
     mbar_init(&c.acc_done, 1);
     mbar_init(&c.drain, 1);
     c.abort = 0;
@@ -384,9 +387,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kernel(
         if (!go) timeout(ctrl, c, seq, 20);
         if (!DKDV) {
           // dq, per walked tile j: S_j = Q K_j^T into the S buffer of j's
-          // parity, issued a tile ahead; dP_j = dO V_j^T as soon as the
-          // softmax warps are done with tile j - 1 (its dP is read); then
-          // dQ += dS_{j-1} K_{j-1} and S_{j+1} over dS_{j-1}.
+          // parity (each buffer with a barrier of its own), issued a tile
+          // ahead; dP_j = dO V_j^T as soon as the softmax warps are done with
+          // tile j - 1 (its dP is read); then dQ += dS_{j-1} K_{j-1} and
+          // S_{j+1} over dS_{j-1}.
           auto issue_s = [&](uint32_t jg) -> bool {
             const uint32_t sa = jg % NA;
             if (!wait(&c.a_full[sa], (jg / NA) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 21); return false; }
@@ -398,6 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kernel(
               const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
               mma_ss(tmem + col, smem_desc_add(dF0, off), smem_desc_add(dA, off), idS, kk > 0);
             }
+            mma_commit(&c.s_full[jg & 1]);
             return true;
           };
           auto issue_dp = [&](uint32_t jg) -> bool {
@@ -410,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kernel(
               const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
               mma_ss(tmem + kTdP, smem_desc_add(dF1, off), smem_desc_add(dB, off), idS, kk > 0);
             }
-            mma_commit(&c.sdp_full);    // S_j (issued before) and dP_j
+            mma_commit(&c.dp_full);
             mma_commit(&c.b_empty[sb]); // V_j is read by dP_j alone
             return true;
           };
@@ -528,49 +533,78 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kernel(
           }
           lim[h] = (kept && frow_ok) ? max(0, min(64, g.N - col0)) : 0;
         }
-        if (!wait_warp(&c.sdp_full, jg & 1, ctrl, seq)) { timeout(ctrl, c, seq, 30); ok = false; break; }
-        tc_fence_after();
         const float2 sl2 = make_float2(scale_log2, scale_log2);
         if (!DKDV) {
-          // dq: S and dP are both in TMEM; per pair of columns
-          // p = 2^(x scale log2 e - L log2 e), dS = p (dP - D) in packed
-          // two-lane arithmetic, dS as bf16 over the S columns already read
-          // (dP is then free for the next tile's product).  Two buffers: the
-          // next chunk's scores and dP load while this one is computed.
+          // dq phase 1, S alone (in TMEM a tile ahead): per pair of columns
+          // p = 2^(x scale log2 e - L log2 e) in packed two-lane arithmetic,
+          // written as fp32 over the S just read.  Two buffers: the next
+          // chunk's scores load while this one is computed.
+          if (!wait_warp(&c.s_full[jg & 1], (jg >> 1) & 1, ctrl, seq)) { timeout(ctrl, c, seq, 30); ok = false; break; }
+          tc_fence_after();
           const uint32_t tS = trow + ((jg & 1) ? kTS1 : kTS);
-          const float2 nl = make_float2(-lse2, -lse2), dd = make_float2(drow, drow);
-          uint32_t sv2[2][32], dv2[2][32];
-          tmem_ld32(tS, sv2[0]);
+          {
+            const float2 nl = make_float2(-lse2, -lse2);
+            uint32_t sv2[2][32];
+            tmem_ld32(tS, sv2[0]);
+#pragma unroll
+            for (int cch = 0; cch < 4; ++cch) {
+              tmem_wait_ld();
+              if (cch < 3) tmem_ld32(tS + 32 * (cch + 1), sv2[(cch + 1) & 1]);
+              uint32_t* sv = sv2[cch & 1];
+              // valid columns of this chunk: all 32 (no per-column test in
+              // the loop, the common case), some, or none (stored as they
+              // are: phase 2 writes zeros there).  cl differs between the
+              // lanes of a warp at the ragged end, so the warp-collective
+              // TMEM store below runs in every case.
+              const int cl = min(32, max(0, lim[cch >> 1] - 32 * (cch & 1)));
+              auto pair = [&](int i, bool masked) {
+                const float2 y = ffma2(make_float2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), sl2, nl);
+                float2 p = make_float2(ex2f(y.x), ex2f(y.y));
+                if (masked) {
+                  p.x = (2 * i < cl) ? p.x : 0.f;
+                  p.y = (2 * i + 1 < cl) ? p.y : 0.f;
+                }
+                sv[2 * i] = __float_as_uint(p.x);
+                sv[2 * i + 1] = __float_as_uint(p.y);
+              };
+              if (cl == 32) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pair(i, false);
+              } else if (cl > 0) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pair(i, true);
+              }
+              tmem_st32(tS + 32 * cch, sv2[cch & 1]);
+            }
+          }
+          tmem_wait_st();
+          // phase 2, once dP is in TMEM: dS = p (dP - D) from the fp32 p,
+          // as bf16 over the columns already read (dP is then free for the
+          // next tile's product)
+          if (!wait_warp(&c.dp_full, jg & 1, ctrl, seq)) { timeout(ctrl, c, seq, 34); ok = false; break; }
+          tc_fence_after();
+          const float2 dd = make_float2(drow, drow);
+          uint32_t pv2[2][32], dv2[2][32];
+          tmem_ld32(tS, pv2[0]);
           tmem_ld32(trow + kTdP, dv2[0]);
 #pragma unroll
           for (int cch = 0; cch < 4; ++cch) {
             tmem_wait_ld();
             if (cch < 3) {
-              tmem_ld32(tS + 32 * (cch + 1), sv2[(cch + 1) & 1]);
+              tmem_ld32(tS + 32 * (cch + 1), pv2[(cch + 1) & 1]);
               tmem_ld32(trow + kTdP + 32 * (cch + 1), dv2[(cch + 1) & 1]);
             }
-            const uint32_t* sv = sv2[cch & 1];
+            const uint32_t* pv = pv2[cch & 1];
             const uint32_t* dv = dv2[cch & 1];
-            // valid columns of this chunk: all 32 (no per-column test in the
-            // loop, the common case), some, or none
             const int cl = min(32, max(0, lim[cch >> 1] - 32 * (cch & 1)));
             uint32_t dk[16];
-            auto pair = [&](int i, bool masked) {
-              const float2 y = ffma2(make_float2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), sl2, nl);
-              float2 p = make_float2(ex2f(y.x), ex2f(y.y));
-              if (masked) {
-                p.x = (2 * i < cl) ? p.x : 0.f;
-                p.y = (2 * i + 1 < cl) ? p.y : 0.f;
+            if (cl > 0) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float2 ds = fmul2(make_float2(__uint_as_float(pv[2 * i]), __uint_as_float(pv[2 * i + 1])),
+                                        fsub2(make_float2(__uint_as_float(dv[2 * i]), __uint_as_float(dv[2 * i + 1])), dd));
+                dk[i] = pack_bf16(ds.x, ds.y);
               }
-              const float2 ds = fmul2(p, fsub2(make_float2(__uint_as_float(dv[2 * i]), __uint_as_float(dv[2 * i + 1])), dd));
-              dk[i] = pack_bf16(ds.x, ds.y);
-            };
-            if (cl == 32) {
-#pragma unroll
-              for (int i = 0; i < 16; ++i) pair(i, false);
-            } else if (cl > 0) {
-#pragma unroll
-              for (int i = 0; i < 16; ++i) pair(i, true);
             } else {
 #pragma unroll
               for (int i = 0; i < 16; ++i) dk[i] = 0u;
@@ -578,6 +612,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_kernel(
             tmem_st16(tS + 16 * cch, dk);
           }
         } else {
+          if (!wait_warp(&c.sdp_full, jg & 1, ctrl, seq)) { timeout(ctrl, c, seq, 30); ok = false; break; }
+          tc_fence_after();
           // dkdv phase 1, S^T alone: P^T = 2^(x scale log2 e - L log2 e) per
           // pair of columns, as bf16 over the S^T columns already read and
           // kept in registers; then the dV product may run.
