@@ -14,7 +14,7 @@
 //   dq kernel    the forward's 128-row query tiles (the same plan), walking
 //                the union of their KV lists: S = Q K^T and dP = dO V^T into
 //                TMEM, P and dS by the softmax warps (dS written as bf16 over
-//                the dP columns), dQ += dS K with A = dS from TMEM;
+//                the S columns), dQ += dS K with A = dS from TMEM;
 //   dkdv kernel  128-key tiles (one block of 128, or two blocks of 64 paired
 //                by the same planner run on the transposed lists), walking the
 //                union of the query blocks that keep them: S^T = K Q^T and
@@ -26,8 +26,10 @@
 // The dq kernel keeps S in two TMEM buffers and writes dS over the S it was
 // computed from, so the next tile's dP (one fixed buffer, free once the
 // softmax warps have read it) is issued as soon as they finish a tile, ahead
-// of that tile's dQ product and the S of the tile after next: only one
-// product sits between two tiles' softmax work.  The dkdv kernel has no TMEM
+// of that tile's dQ product and the S of the tile after next.  Its softmax
+// warps work in two phases: fp32 P in place over S (S is in TMEM a tile
+// ahead), then dS once dP is there, so only the dP product's wait sits
+// between two tiles' softmax work, and the exponentials overlap it.  The dkdv kernel has no TMEM
 // to spare (S, dP and two accumulators fill it); its softmax warps work in two
 // phases instead: P^T from S^T alone (the exponentials), then dS^T from the
 // bf16 P^T kept in registers once dP^T is there.  dV and the next S^T run
