@@ -17,9 +17,9 @@
 //   O_w += P V     tcgen05.mma with A = P from TMEM and B = V (MN-major) from
 //                  shared memory, O_w in TMEM
 // Shared memory then carries only the TMA tiles and the MMA reads of Q, K and
-// V: about 160 KB per KV tile against 1024 cycles of tensor work, where
-// staging P in shared memory as well (written by the softmax, read by the
-// MMA) costs another 64 KB per tile of its 128 bytes per clock.
+// V, and one thread issues every MMA: staging P in shared memory instead
+// (written by the softmax, read by the MMA from there) measured the same speed
+// with a second issuer and 64 KB more shared-memory traffic per KV tile.
 //
 // One thread issues every MMA of the CTA, in this order: S(0), S(1), then for
 // each j: O_w += P(j) V(j), S(j + 2) into the same buffer w.  tcgen05.mma
