@@ -36,6 +36,7 @@ constexpr int kOverlapRows = 32;     // rows whose weights one overlap CTA write
 constexpr int kOverlapThreads = kOverlapRows * kWindow;  // 1024
 constexpr int kMatchThreads = 1024;
 static_assert(kMatchThreads >= BSA_MAX_BLOCKS, "match_kernel handles one block row per thread");
+static_assert(kWindow % 2 == 0 && kMatchThreads % 64 == 0, "two lanes per row split the window in halves");
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -153,24 +154,40 @@ __global__ void __launch_bounds__(kMatchThreads) match_kernel(const int32_t* __r
   __syncthreads();
 
   if (QB == 2) {
-    for (int round = 0; round < kRounds; ++round) {
-      for (int r = threadIdx.x; r < nb; r += kMatchThreads) {
-        int best = -1, bestw = -1;
-        if (partner[r] < 0) {
-          for (int off = 1; off <= kWindow; ++off) {
-            const int lo = r - off, hi = r + off;
-            // ties keep the nearer, then the lower, index
-            if (lo >= 0 && partner[lo] < 0) {
-              const int w = wts[(off - 1) * S + lo];
-              if (w > bestw) { bestw = w; best = lo; }
-            }
-            if (hi < nb && partner[hi] < 0) {
-              const int w = wts[(off - 1) * S + r];
-              if (w > bestw) { bestw = w; best = hi; }
-            }
-          }
+    // Each unmatched row's heaviest free partner within the window, offsets
+    // scanned nearest first (lower index first at equal offset), a strictly
+    // heavier weight replacing the pick: ties keep the nearer, then the
+    // lower, index.  Up to kMatchThreads / 2 rows, two adjacent lanes scan
+    // half the offsets each and the far half's pick wins only when strictly
+    // heavier, which is the same rule.
+    const bool split = nb <= kMatchThreads / 2;
+    auto scan = [&](int r, int off0, int off1, int& best, int& bestw) {
+      for (int off = off0; off <= off1; ++off) {
+        const int lo = r - off, hi = r + off;
+        if (lo >= 0 && partner[lo] < 0) {
+          const int w = wts[(off - 1) * S + lo];
+          if (w > bestw) { bestw = w; best = lo; }
         }
-        choice[r] = best;
+        if (hi < nb && partner[hi] < 0) {
+          const int w = wts[(off - 1) * S + r];
+          if (w > bestw) { bestw = w; best = hi; }
+        }
+      }
+    };
+    for (int round = 0; round < kRounds; ++round) {
+      if (split) {
+        const int r = threadIdx.x >> 1, part = threadIdx.x & 1;
+        int best = -1, bestw = -1;
+        if (r < nb && partner[r] < 0) scan(r, 1 + part * (kWindow / 2), (part + 1) * (kWindow / 2), best, bestw);
+        const int far_w = __shfl_down_sync(0xffffffffu, bestw, 1);
+        const int far_b = __shfl_down_sync(0xffffffffu, best, 1);
+        if (part == 0 && r < nb) choice[r] = (far_w > bestw) ? far_b : best;
+      } else {
+        for (int r = threadIdx.x; r < nb; r += kMatchThreads) {
+          int best = -1, bestw = -1;
+          if (partner[r] < 0) scan(r, 1, kWindow, best, bestw);
+          choice[r] = best;
+        }
       }
       __syncthreads();
       int formed = 0;
