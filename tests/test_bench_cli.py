@@ -43,3 +43,30 @@ def test_package_import_maps_the_library_only_on_first_call():
     r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.split() == ["False", "True", "True"]
+
+
+def test_recorded_traffic_follows_the_measured_kernel_source(tmp_path, monkeypatch):
+    """The bench line's `traffic` comes from the committed ncu record only while
+    the measured kernel's source and the shared headers are those it was taken
+    from: a change to that kernel voids it, a change to another kernel does not."""
+    import shutil
+    sys.path.insert(0, ROOT)
+    import bench
+    rec = json.load(open(os.path.join(ROOT, "profiles", "dram_traffic.json")))
+    assert bench.recorded_traffic("attn", "wan480p") == rec["attn"]["bytes_per_launch"]
+    assert bench.recorded_traffic("attn", "hunyuan720p") is None      # recorded on another workload
+    csrc = tmp_path / "block_sparse_attention_fractal_b200" / "csrc"
+    shutil.copytree(os.path.join(ROOT, "block_sparse_attention_fractal_b200", "csrc"), csrc)
+    shutil.copytree(os.path.join(ROOT, "profiles"), tmp_path / "profiles")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.recorded_traffic("attn", "wan480p") == rec["attn"]["bytes_per_launch"]
+    with open(csrc / "attn_bwd.cu", "a") as f:
+        f.write("\n// another kernel's change\n")
+    assert bench.recorded_traffic("attn", "wan480p") == rec["attn"]["bytes_per_launch"]
+    with open(csrc / "attn_fwd.cu", "a") as f:
+        f.write("\n// the measured kernel's change\n")
+    assert bench.recorded_traffic("attn", "wan480p") is None
+    assert bench.recorded_traffic("fine", "wan480p") == rec["fine"]["bytes_per_launch"]
+    with open(csrc / "sm100.cuh", "a") as f:
+        f.write("\n// a shared header's change\n")
+    assert bench.recorded_traffic("fine", "wan480p") is None
